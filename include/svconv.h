@@ -1,0 +1,179 @@
+/*
+ * svconv — SparseConv2D on frame-wise pruned ViT tokens, B200 (sm_100a).
+ *
+ * C ABI of the CUDA library (libsvconv.so).  The operation is the native sparse
+ * 3x3 convolution of SV-TAD (papernotes.org, "SV-TAD: Native Sparse Convolutions
+ * for Efficient Temporal Action Detection", Method, Key Designs 1 and 2), which
+ * convolves a packed, pruned token sequence directly through a neighbour table
+ * and never rebuilds the dense H x W grid.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tokens are packed frame by frame: frame t owns packed rows
+ *    frame_off[t] .. frame_off[t+1]-1 (frame_off is int32, CSR style, T+1 entries).
+ *    coords is int32 [n][3] = (t, y, x) per token.  Within a frame any token
+ *    order is accepted.
+ *  - Taps j = 0..8 are row-major over (dy, dx) in {-1,0,1}^2: j = (dy+1)*3 + (dx+1).
+ *    j = 4 is the token itself and 8-j is the mirrored offset (-dy, -dx).
+ *  - The neighbour table nbr is int32 [n][9]; nbr[k][j] is the GLOBAL packed row
+ *    of the token at (t, y_k+dy_j, x_k+dx_j), or -1 if that cell was pruned or lies
+ *    outside the frame.  Neighbours never cross frames.
+ *  - Features are row-major with channels contiguous: X [n][C_in], Y [n][C_out].
+ *    Weights are W [C_out][9][C_in] (torch conv2d weight w[o][i][dy+1][dx+1] maps
+ *    to W[o][(dy+1)*3+(dx+1)][i]); the operator is a cross-correlation, like conv2d.
+ *  - All pointers are DEVICE pointers owned by the caller unless stated otherwise;
+ *    the library allocates no device memory and every call is asynchronous on the
+ *    given CUDA stream (a cudaStream_t passed as void*; NULL = legacy stream).
+ *  - dtype SVCONV_F32: fp32 in/out, fp32 accumulate, CUDA cores.
+ *    dtype SVCONV_BF16: bf16 in/out, fp32 accumulate on tcgen05 tensor cores;
+ *    requires C_in % 64 == 0 and C_out % 64 == 0 and 16-byte aligned pointers.
+ *    Unsupported shapes are rejected with SVCONV_ERR_UNSUPPORTED (no fallback).
+ *  - Return value: SVCONV_OK (0) or a negative host-detected error.  Problems found
+ *    inside kernels (bad coordinates, an index outside the table, a bounded wait
+ *    that ran out) never fault: they set bits in a device status word (see
+ *    SVCONV_STATUS_*) and leave the outputs undefined.
+ */
+#ifndef SVCONV_H_
+#define SVCONV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVCONV_API __attribute__((visibility("default")))
+#else
+#define SVCONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define SVCONV_F32 0
+#define SVCONV_BF16 1
+
+/* host-side return codes */
+#define SVCONV_OK 0
+#define SVCONV_ERR_NULL (-1)        /* a required pointer is NULL */
+#define SVCONV_ERR_SIZE (-2)        /* negative or too large size / count */
+#define SVCONV_ERR_UNSUPPORTED (-3) /* dtype or channel count not supported */
+#define SVCONV_ERR_ALIGN (-4)       /* pointer not 16-byte aligned (bf16 paths) */
+#define SVCONV_ERR_WORKSPACE (-5)   /* workspace NULL or smaller than the query says */
+#define SVCONV_ERR_CUDA (-6)        /* CUDA runtime / launch error */
+#define SVCONV_ERR_DEVICE (-7)      /* current device is not an sm_100 GPU */
+
+/* device status bits (OR-ed into an int32 word in device memory) */
+#define SVCONV_STATUS_BAD_COORD 1       /* y or x outside the H x W frame */
+#define SVCONV_STATUS_DUPLICATE 2       /* two tokens at the same (t, y, x) */
+#define SVCONV_STATUS_BAD_FRAME 4       /* coords[k].t differs from the frame holding k */
+#define SVCONV_STATUS_BAD_OFFSETS 8     /* frame_off not 0..n and non-decreasing */
+#define SVCONV_STATUS_TIMEOUT 16        /* a kernel's bounded wait ran out; it returned early */
+#define SVCONV_STATUS_BAD_INDEX 32      /* a neighbour index outside the feature rows; read as 0 */
+#define SVCONV_STATUS_CHUNK_OVERFLOW 64 /* adapter chunk holds more rows than max_chunk_rows */
+
+/*
+ * Neighbour-index build (Key Design 1: the lookup map M per frame, filled with -1,
+ * then M[y_k, x_k] = k; then N[k, j] = M[y_k+dy_j, x_k+dx_j], or -1 when the
+ * neighbour was pruned or is out of bounds).  One CTA per frame keeps M in shared
+ * memory; nothing returns to the host.
+ *   coords     [n][3] int32 device, frame_off [T+1] int32 device.
+ *   nbr        [n][9] int32 device, written.
+ *   M          [T][H][W] int32 device or NULL; if given, written with the map
+ *              (global packed indices, -1 elsewhere).  With duplicate
+ *              coordinates the cell holds the largest k and DUPLICATE is set.
+ *   dev_status int32 device or NULL; SVCONV_STATUS_BAD_* bits are OR-ed in (the
+ *              caller zeroes it).  Rows of tokens with bad coordinates are -1.
+ *   Limits: H*W <= 16384, T >= 0, n >= 0.
+ */
+SVCONV_API int svconv_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,
+                       int32_t* nbr, int32_t* M, int32_t* dev_status, void* stream);
+
+/*
+ * Forward (Key Design 2: y_k = sum_j W_j x[N[k,j]], N = -1 read as zero padding),
+ * plus an optional bias: Y[k][o] = bias[o] + sum_j sum_i W[o][j][i] * X[N[k][j]][i].
+ *   X [n][Cin], Y [n][Cout] of dtype; Wt [Cout][9][Cin] of dtype;
+ *   bias [Cout] fp32 device or NULL.  Y must not alias X.
+ *   fp32 limit: 9*Cin*Cout <= 49152.  bf16: Cin, Cout multiples of 64, Cout <= 4096.
+ */
+SVCONV_API int svconv_fwd(int dtype, const void* X, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt,
+               const float* bias, void* Y, void* stream);
+
+/*
+ * Backward w.r.t. the input features.  The page names backward kernels but prints
+ * no formula; this is the adjoint of svconv_fwd written as a GATHER through the
+ * mirrored offset:  dX[k] = sum_j W_j^T dY[N[k][8-j]]  (N[m][j] = k  <=>  N[k][8-j] = m
+ * for tokens of one frame), so it is deterministic and uses no atomics.
+ *   dY [n][Cout], dX [n][Cin] of dtype; Wt as in svconv_fwd.  dX must not alias dY.
+ *   Limits as svconv_fwd.  No workspace.
+ */
+SVCONV_API int svconv_bwd_data(int dtype, const void* dY, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt,
+                    void* dX, void* stream);
+
+/*
+ * Backward w.r.t. the weights and bias (adjoint of svconv_fwd):
+ *   dW[o][j][i] = sum_k dY[k][o] * X[N[k][j]][i],   db[o] = sum_k dY[k][o].
+ * A GEMM over K = n tokens with the gather on the X side, split over token ranges
+ * into fp32 partials in the workspace, then reduced in a fixed order: the result
+ * is deterministic (bitwise identical across runs) and atomic-free.
+ *   dY [n][Cout], X [n][Cin] of dtype; dW [Cout][9][Cin] fp32 and db [Cout] fp32
+ *   (db may be NULL) are overwritten.
+ *   workspace: device, at least svconv_bwd_weight_workspace_size(...) bytes,
+ *   16-byte aligned, no initial contents required.
+ */
+SVCONV_API int svconv_bwd_weight(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
+                      float* dW, float* db, void* workspace, size_t ws_bytes, void* stream);
+SVCONV_API size_t svconv_bwd_weight_workspace_size(int dtype, int n, int Cin, int Cout);
+
+/*
+ * Chunked bottleneck adapter forward (Key Design 2, "chunked execution" that
+ * keeps memory flat in the number of frames; the adapter is the "lightweight
+ * bottleneck adapter" with "down-projected" features of the Overall Architecture
+ * and Key Design 3).  For each chunk of chunk_T frames, in order:
+ *     H1 = bf16(X Wd^T)                         Wd [R][D]
+ *     H2 = bf16(GELU(SparseConv3x3(H1) + bc))   Wc [R][9][R], bc [R] fp32 or NULL
+ *     X  = bf16(X + H2 Wu^T)   (in place)       Wu [D][R]
+ * GELU is the erf form 0.5 x (1 + erf(x / sqrt 2)).  All of X, Wd, Wc, Wu are
+ * bf16; accumulation is fp32.
+ *   X          [n][D] bf16 device, read and overwritten in place.
+ *   nbr        [n][9] global neighbour table (svconv_build_index).
+ *   frame_off  [T+1] int32 DEVICE; chunk bounds are read on the device.
+ *   max_chunk_rows  upper bound on the tokens of any chunk; a larger chunk sets
+ *              SVCONV_STATUS_CHUNK_OVERFLOW and only its first max_chunk_rows rows
+ *              are processed.
+ *   workspace  >= svconv_adapter_workspace_size(R, max_chunk_rows) bytes.
+ *   dev_status int32 device or NULL (status bits are OR-ed in).
+ *   Limits: D, R multiples of 64, R <= 4096.
+ */
+SVCONV_API int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
+                       const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T,
+                       int max_chunk_rows, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
+SVCONV_API size_t svconv_adapter_workspace_size(int R, int max_chunk_rows);
+
+/*
+ * The library's own device error word (per device): kernels without a caller
+ * status pointer (fwd, bwd_data, bwd_weight) OR SVCONV_STATUS_TIMEOUT and
+ * SVCONV_STATUS_BAD_INDEX into it.  Reading it synchronizes the current device,
+ * copies the word to *out and clears it.
+ */
+SVCONV_API int svconv_read_error_word(int32_t* out);
+
+/*
+ * Failure-detection check: launches one CTA whose mbarrier wait can never
+ * complete (nothing arrives), bounded by timeout_us microseconds.  The kernel
+ * gives up, records SVCONV_STATUS_TIMEOUT into *dev_status and returns normally,
+ * leaving the context usable.
+ */
+SVCONV_API int svconv_selftest_timeout(int32_t* dev_status, int timeout_us, void* stream);
+
+/* Static text for a return code or a status bit. */
+SVCONV_API const char* svconv_status_str(int code);
+
+/* Library ABI version (major * 100 + minor). */
+SVCONV_API int svconv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVCONV_H_ */

@@ -58,6 +58,7 @@ def _load():
         lib.orc_round_bf16.restype = ctypes.c_double
         lib.orc_adapter_fwd.argtypes = [P, P, I, I, I, I, P, P, P, P, P]
         lib.orc_dense_conv.argtypes = [P, I, I, I, I, P, P, P]
+        lib.orc_bwd_bias.argtypes = [P, I, I, P]
         _lib = lib
     return _lib
 
@@ -139,6 +140,15 @@ def bwd_weight_entries(dY, X, nbr, entries):
     out = np.empty((ent.shape[0],), dtype=np.float64)
     lib.orc_bwd_weight_entries(_p(dY), _p(X), _p(nbr), n, Cin, Cout, _p(ent), ent.shape[0], _p(out))
     return out
+
+
+def bwd_bias(dY):
+    lib = _load()
+    dY = _f64(dY)
+    n, Cout = dY.shape
+    db = np.empty((Cout,), dtype=np.float64)
+    lib.orc_bwd_bias(_p(dY), n, Cout, _p(db))
+    return db
 
 
 def round_bf16(v: float) -> float:

@@ -269,3 +269,11 @@ void orc_dense_conv(const double *G, int H, int W, int Cin, int Cout, const doub
                 Y[((size_t)y * W + x) * Cout + o] = acc;
             }
 }
+
+/* Bias gradient alone: db[o] = sum_k dY[k][o]. */
+void orc_bwd_bias(const double *dY, int n, int Cout, double *db)
+{
+    for (int o = 0; o < Cout; ++o) db[o] = 0.0;
+    for (int k = 0; k < n; ++k)
+        for (int o = 0; o < Cout; ++o) db[o] += dY[(size_t)k * Cout + o];
+}

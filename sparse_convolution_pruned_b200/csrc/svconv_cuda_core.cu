@@ -1,0 +1,158 @@
+// fp32 path on CUDA cores (exact fp32 arithmetic; TF32 tensor cores would not
+// meet an fp32 tolerance), plus the fixed-order split reduction shared by both
+// weight-gradient paths.
+//
+//  * f32_conv_kernel: one thread per (token, output channel).  The 9 x C_src x
+//    C_dst weight block sits in shared memory, laid out so that a warp's
+//    consecutive output channels read consecutive words (no bank conflicts); the
+//    neighbour row of the source features is read once per warp (broadcast).
+//    The same kernel computes the forward (gather through N[k][j]) and the data
+//    gradient (gather through the mirrored column N[k][8-j] with W_j transposed).
+//  * f32_wgrad_partial_kernel: each split of tokens writes its partial dW rows
+//    (row m = j*C_in + i, row 9*C_in = db) to the workspace.
+//  * wgrad_reduce_kernel: sums the splits in index order (deterministic) and
+//    transposes to dW[o][j][i] through a 32x32 shared tile.
+#include "svconv_internal.h"
+
+namespace svc {
+namespace {
+
+__global__ void __launch_bounds__(256) f32_conv_kernel(const float* __restrict__ src, const int32_t* __restrict__ nbr,
+                                                       int n, int Csrc, int Cdst, const float* __restrict__ Wt,
+                                                       int Cin, int Cout, int mirror, const float* __restrict__ bias,
+                                                       float* __restrict__ dst, int* err) {
+  extern __shared__ float sW[];  // [9][Csrc][Cdst]
+  const int total_w = 9 * Cin * Cout;
+  for (int e = threadIdx.x; e < total_w; e += blockDim.x) {
+    const int o = e / (9 * Cin);
+    const int j = (e / Cin) % 9;
+    const int i = e % Cin;
+    const float w = Wt[e];
+    if (!mirror)
+      sW[((size_t)j * Cin + i) * Cout + o] = w;  // forward: src = X (Cin), dst = Y (Cout)
+    else
+      sW[((size_t)j * Cout + o) * Cin + i] = w;  // data grad: src = dY (Cout), dst = dX (Cin)
+  }
+  __syncthreads();
+  const long long total = (long long)n * Cdst;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int k = (int)(e / Cdst);
+    const int c = (int)(e - (long long)k * Cdst);
+    float acc = bias ? bias[c] : 0.0f;
+    for (int j = 0; j < 9; ++j) {
+      const int m = nbr[(size_t)k * 9 + (mirror ? 8 - j : j)];
+      if (m < 0) continue;
+      if (m >= n) {
+        atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+        continue;
+      }
+      const float* s = src + (size_t)m * Csrc;
+      const float* w = sW + (size_t)j * Csrc * Cdst + c;
+      for (int q = 0; q < Csrc; ++q) acc = fmaf(w[(size_t)q * Cdst], s[q], acc);
+    }
+    dst[e] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __restrict__ dY,
+                                                                const float* __restrict__ X,
+                                                                const int32_t* __restrict__ nbr, int n, int Cin,
+                                                                int Cout, float* __restrict__ partial, int splits,
+                                                                int rows_pad, int* err) {
+  const int sp = blockIdx.y;
+  const int k0 = (int)((long long)n * sp / splits), k1 = (int)((long long)n * (sp + 1) / splits);
+  const int rows = 9 * Cin + 1;
+  const long long total = (long long)rows * Cout;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int m = (int)(e / Cout);
+    const int o = (int)(e - (long long)m * Cout);
+    float acc = 0.0f;
+    if (m < 9 * Cin) {
+      const int j = m / Cin, i = m - j * Cin;
+      for (int k = k0; k < k1; ++k) {
+        const int nb = nbr[(size_t)k * 9 + j];
+        if (nb < 0) continue;
+        if (nb >= n) {
+          atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+          continue;
+        }
+        acc = fmaf(dY[(size_t)k * Cout + o], X[(size_t)nb * Cin + i], acc);
+      }
+    } else {
+      for (int k = k0; k < k1; ++k) acc += dY[(size_t)k * Cout + o];
+    }
+    partial[((size_t)sp * rows_pad + m) * Cout + o] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
+                                                           int rows_pad, int Cin, int Cout, float* __restrict__ dW,
+                                                           float* __restrict__ db) {
+  __shared__ float tile[32][33];
+  const int rows = 9 * Cin + 1;
+  const int m0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int r = ty; r < 32; r += 8) {
+    const int m = m0 + r, o = o0 + tx;
+    float s = 0.0f;
+    if (m < rows && o < Cout)
+      for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * rows_pad + m) * Cout + o];
+    tile[r][tx] = s;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int o = o0 + r, m = m0 + tx;
+    if (o >= Cout) continue;
+    if (m < 9 * Cin)
+      dW[(size_t)o * 9 * Cin + m] = tile[tx][r];
+    else if (m == 9 * Cin && db)
+      db[o] = tile[tx][r];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_f32_conv(bool mirror_bwd, const float* src, const int32_t* nbr, int n, int Csrc, int Cdst,
+                            const float* Wt, int Cin, int Cout, const float* bias, float* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * 9 * (size_t)Cin * Cout;
+  static int done[64];
+  cudaError_t e = ensure_smem_attr(f32_conv_kernel, smem, done);
+  if (e != cudaSuccess) return e;
+  long long blocks = ((long long)n * Cdst + 255) / 256;
+  const long long cap = (long long)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  f32_conv_kernel<<<(int)blocks, 256, smem, s>>>(src, nbr, n, Csrc, Cdst, Wt, Cin, Cout, mirror_bwd ? 1 : 0, bias,
+                                                 dst, device_error_word());
+  return cudaGetLastError();
+}
+
+size_t f32_wgrad_splits(int n) {
+  int sp = (n + 127) / 128;
+  if (sp > 128) sp = 128;
+  if (sp < 1) sp = 1;
+  return (size_t)sp;
+}
+
+cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int32_t* nbr, int n, int Cin, int Cout,
+                                      float* partial, int splits, int rows_pad, cudaStream_t s) {
+  const long long total = (long long)(9 * Cin + 1) * Cout;
+  long long bx = (total + 255) / 256;
+  if (bx > 64) bx = 64;
+  dim3 grid((unsigned)bx, (unsigned)splits);
+  f32_wgrad_partial_kernel<<<grid, 256, 0, s>>>(dY, X, nbr, n, Cin, Cout, partial, splits, rows_pad,
+                                                device_error_word());
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, float* dW,
+                                float* db, cudaStream_t s) {
+  const int rows = 9 * Cin + 1;
+  dim3 grid((rows + 31) / 32, (Cout + 31) / 32);
+  wgrad_reduce_kernel<<<grid, dim3(32, 8), 0, s>>>(partial, splits, rows_pad, Cin, Cout, dW, db);
+  return cudaGetLastError();
+}
+
+}  // namespace svc

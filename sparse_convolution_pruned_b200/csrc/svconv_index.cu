@@ -1,0 +1,92 @@
+// Neighbour-index build on the GPU (SV-TAD page, Key Design 1: the per-frame
+// lookup map M, filled with -1 and then M[y_k, x_k] = k, and the neighbour table
+// N[k, j] = M[y_k + dy_j, x_k + dx_j] or -1).  The page builds both on the CPU;
+// here one CTA per frame keeps that frame's M in shared memory, so the table is
+// produced next to the features with no host round trip.
+//
+// Traffic per token: 12 B of coordinates read (twice, the second time from L1/L2)
+// and 36 B of N written; the writes are fully coalesced because consecutive
+// threads produce consecutive (k, j) entries of the frame's contiguous N rows.
+#include "svconv_internal.h"
+
+namespace svc {
+namespace {
+
+__global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restrict__ coords,
+                                                          const int32_t* __restrict__ frame_off, int T, int H,
+                                                          int W, int n, int32_t* __restrict__ nbr,
+                                                          int32_t* __restrict__ Mout, int32_t* status) {
+  extern __shared__ int32_t sM[];  // [H][W] of this frame
+  __shared__ int s_flags;
+  __shared__ int s_lo, s_hi;
+  const int t = blockIdx.x;
+  const int HW = H * W;
+  if (threadIdx.x == 0) {
+    int flags = 0;
+    int lo = frame_off[t], hi = frame_off[t + 1];
+    if (lo < 0 || hi < lo || hi > n) flags |= SVCONV_STATUS_BAD_OFFSETS;
+    if (t == 0 && lo != 0) flags |= SVCONV_STATUS_BAD_OFFSETS;
+    if (t == T - 1 && hi != n) flags |= SVCONV_STATUS_BAD_OFFSETS;
+    if (flags) lo = hi = 0;  // a segment that cannot be trusted is not touched
+    s_flags = flags;
+    s_lo = lo;
+    s_hi = hi;
+  }
+  for (int c = threadIdx.x; c < HW; c += blockDim.x) sM[c] = -1;
+  __syncthreads();
+  const int lo = s_lo, hi = s_hi;
+
+  // step 1: M[y_k][x_k] = k.  With duplicates the largest k wins (deterministic).
+  for (int k = lo + threadIdx.x; k < hi; k += blockDim.x) {
+    const int tt = coords[3 * k], y = coords[3 * k + 1], x = coords[3 * k + 2];
+    if (tt != t) {
+      atomicOr(&s_flags, SVCONV_STATUS_BAD_FRAME);
+      continue;
+    }
+    if (y < 0 || y >= H || x < 0 || x >= W) {
+      atomicOr(&s_flags, SVCONV_STATUS_BAD_COORD);
+      continue;
+    }
+    atomicMax(&sM[y * W + x], k);
+  }
+  __syncthreads();
+
+  // step 2: the 9 lookups, one (k, j) entry per thread, coalesced writes.
+  const long long cnt = (long long)(hi - lo) * 9;
+  int32_t* out = nbr + (size_t)lo * 9;
+  for (long long e = threadIdx.x; e < cnt; e += blockDim.x) {
+    const int k = lo + (int)(e / 9);
+    const int j = (int)(e - (long long)(k - lo) * 9);
+    const int tt = coords[3 * k], y = coords[3 * k + 1], x = coords[3 * k + 2];
+    int32_t v = -1;
+    if (tt == t && y >= 0 && y < H && x >= 0 && x < W) {
+      if (j == 4 && sM[y * W + x] != k) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
+      const int yy = y + j / 3 - 1, xx = x + j % 3 - 1;
+      if (yy >= 0 && yy < H && xx >= 0 && xx < W) v = sM[yy * W + xx];
+    }
+    out[e] = v;
+  }
+  if (Mout) {
+    int32_t* dst = Mout + (size_t)t * HW;
+    for (int c = threadIdx.x; c < HW; c += blockDim.x) dst[c] = sM[c];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && s_flags && status) atomicOr(status, s_flags);
+}
+
+}  // namespace
+
+cudaError_t launch_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,
+                               int32_t* nbr, int32_t* M, int32_t* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const size_t smem = sizeof(int32_t) * (size_t)H * W;
+  if (smem > 48 * 1024) {
+    static int done[64];
+    cudaError_t e = ensure_smem_attr(build_index_kernel, smem, done);
+    if (e != cudaSuccess) return e;
+  }
+  build_index_kernel<<<T, 256, smem, s>>>(coords, frame_off, T, H, W, n, nbr, M, status);
+  return cudaGetLastError();
+}
+
+}  // namespace svc

@@ -1,0 +1,90 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "svconv.h"
+
+namespace svc {
+
+// The library's per-device error word (defined in svconv_api.cu).
+int* device_error_word();
+int sm_count();
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s for any single bounded wait
+
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// call is skipped afterwards, which keeps launches cheap and capturable).
+template <typename Kernel>
+inline cudaError_t ensure_smem_attr(Kernel kernel, size_t bytes, int* done_bytes /* [64] per device */) {
+  int d = 0;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return e;
+  if (d >= 0 && d < 64 && done_bytes[d] >= (int)bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && d >= 0 && d < 64) done_bytes[d] = (int)bytes;
+  return e;
+}
+
+// ---------------------------------------------------------------- index build
+cudaError_t launch_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,
+                               int32_t* nbr, int32_t* M, int32_t* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- fp32 CUDA-core path
+cudaError_t launch_f32_conv(bool mirror_bwd, const float* src, const int32_t* nbr, int n, int Csrc, int Cdst,
+                            const float* Wt, int Cin, int Cout, const float* bias, float* dst, cudaStream_t s);
+size_t f32_wgrad_splits(int n);
+cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int32_t* nbr, int n, int Cin, int Cout,
+                                      float* partial, int splits, int rows_pad, cudaStream_t s);
+// partial [splits][rows_pad][Cout] with row m = j*Cin + i (m = 9*Cin holds db)
+cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, float* dW,
+                                float* db, cudaStream_t s);
+
+// ---------------------------------------------------------------- tcgen05 bf16 path
+struct TcConvArgs {
+  // A operand: rows gathered (taps = 9) or read densely (taps = 1)
+  const void* A;          // bf16 [rows][lda]
+  int lda;
+  int a_rows;             // number of valid rows in A (range check for gathered indices)
+  const int32_t* nbr;     // [*][9] or nullptr for dense
+  int taps;               // 9 or 1
+  int mirror;             // gather uses column 8-j
+  int Kc;                 // channels per tap (multiple of 64)
+  // B operand (weights), described by a TMA tensor map built on the host
+  int b_mn_major;         // 0: W[o][j*Kc + c] K-major 2D map; 1: W[c][j][n] MN-major 3D map
+  // rows
+  int M;                  // rows to compute (upper bound when row pointers are given)
+  const int32_t* row_lo;  // device pointers (chunked adapter) or nullptr
+  const int32_t* row_hi;
+  int a_abs;              // dense A row = lo + r (else r)
+  int nbr_abs;            // neighbour table row = lo + r and values are rebased by -lo
+  int out_abs;            // output row = lo + r (else r)
+  int N;                  // output columns
+  // epilogue
+  const float* bias;      // [N] or nullptr
+  int gelu;
+  const void* residual;   // bf16 [rows][ldo] or nullptr (added before the store; may alias out)
+  void* out;              // bf16 [rows][ldo]
+  int ldo;
+  int out_rows;           // rows of out / residual (range check of absolute output rows)
+  int32_t* status;        // caller status word or nullptr (library word used otherwise)
+};
+cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s);
+
+struct TcWgradArgs {
+  const void* dY;     // bf16 [n][Cout]
+  const void* X;      // bf16 [n][Cin]
+  const int32_t* nbr; // [n][9]
+  int n, Cin, Cout;
+  float* partial;     // [splits][rows_pad][Cout]
+  int splits, rows_pad;
+};
+void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn);
+cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s);
+
+// failure-detection self test
+cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace svc

@@ -1,0 +1,770 @@
+// bf16 SparseConv2D on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// After the gather, each output tile is a dense contraction (SV-TAD page, Key
+// Design 2: y_k = sum_j W_j x[N[k,j]] is a GEMM with K = 9 * C_in whose A rows
+// are gathered through the neighbour table), so it runs as a warp-specialised,
+// persistent implicit GEMM:
+//
+//   warps 4-7 (producers)  gather A: for K-block (tap j, 64 channels) each
+//                          128-token tile row is one 128-byte segment of a
+//                          neighbour's feature row, copied with 16-byte cp.async
+//                          into the 128B-swizzled K-major layout; -1 neighbours
+//                          are zero-filled by the copy itself.  One thread also
+//                          issues the TMA load of the matching weight tile B.
+//   warp 8 (MMA)           one thread issues tcgen05.mma (M=128, N=BN, K=16) into
+//                          a double-buffered fp32 accumulator in TMEM and
+//                          releases smem stages with tcgen05.commit.
+//   warps 0-3 (epilogue)   tcgen05.ld the accumulator (warp w owns TMEM lanes
+//                          32w..32w+31 = tile rows), add bias / GELU / residual,
+//                          convert to bf16 and store, overlapping the next
+//                          tile's main loop.
+//
+// The data gradient uses the same kernel: the gather goes through the mirrored
+// column N[k][8-j] of dY, and B = W_j^T is read straight from W[o][j][i] as an
+// MN-major operand (3-D TMA box over (i, j, o)), so no transposed copy of W is
+// made.  The dense adapter projections are the same kernel with one tap and the
+// identity "gather".
+//
+// The weight gradient dW^T[(j,i)][o] = sum_k X[N[k,j]][i] dY[k][o] is a GEMM with
+// K = tokens: A (gathered X) and B (dY, by TMA) are both MN-major tiles.  The
+// bias gradient comes out of the same MMAs: the A row after the last (j, i) row
+// is all ones, so its accumulator row is sum_k dY[k][o].  Token ranges are split
+// over CTAs into fp32 partials, reduced afterwards in a fixed order.
+//
+// No TMA multicast is used anywhere.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstring>
+
+#include "svconv_internal.h"
+#include "svconv_ptx.cuh"
+
+namespace svc {
+
+constexpr int kBM = 128;                 // tile rows (tokens / dW rows) = TMEM lanes
+constexpr int kBK = 64;                  // bf16 elements per K-block (one 128-byte row)
+constexpr int kABytes = kBM * kBK * 2;   // 16 KB per A stage
+constexpr int kThreads = 9 * 32;         // 4 epilogue + 4 producer + 1 MMA warp
+constexpr int kLag = 2;                  // cp.async groups kept in flight per producer thread
+constexpr int kMaxStages = 8;
+
+struct __align__(8) TcBarriers {
+  uint64_t full[kMaxStages];    // producers' cp.async data landed (one arrival per producer warp)
+  uint64_t bfull[kMaxStages];   // TMA weight tile landed (expect_tx)
+  uint64_t empty[kMaxStages];   // MMA finished reading the stage (tcgen05.commit)
+  uint64_t tfull[2];            // accumulator buffer ready for the epilogue
+  uint64_t tempty[2];           // epilogue drained the accumulator buffer (one arrival per epilogue warp)
+  uint64_t done;                // final MMA drain before TMEM is released
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct TcConvParams {
+  CUtensorMap tmap_b;
+  const __nv_bfloat16* A;
+  const int32_t* nbr;
+  const int32_t* row_lo;
+  const int32_t* row_hi;
+  const float* bias;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* out;
+  int* status;
+  unsigned long long timeout_ns;
+  int lda, a_rows, taps, mirror, Kc;
+  int M, a_abs, nbr_abs, out_abs, N;
+  int gelu, ldo, out_rows, stages;
+};
+
+struct TcWgradParams {
+  CUtensorMap tmap_dy;
+  const __nv_bfloat16* X;
+  const int32_t* nbr;
+  float* partial;
+  int* status;
+  unsigned long long timeout_ns;
+  int n, Cin, Cout, splits, rows_pad, stages;
+};
+
+__host__ __device__ constexpr int tmem_cols_for(int bn) {
+  return (2 * bn) <= 32 ? 32 : (2 * bn) <= 64 ? 64 : (2 * bn) <= 128 ? 128 : (2 * bn) <= 256 ? 256 : 512;
+}
+
+__host__ __device__ constexpr size_t stage_bytes(int bn) { return (size_t)kABytes + (size_t)bn * kBK * 2; }
+
+static size_t smem_bytes(int bn, int stages) {
+  return 1024 /* alignment slack */ + stage_bytes(bn) * stages + sizeof(int32_t) * kBM * 9 + sizeof(TcBarriers);
+}
+
+struct TileCarve {
+  uint8_t* a;
+  uint8_t* b;
+  int32_t* idx;
+  TcBarriers* bar;
+};
+
+template <int BN>
+__device__ __forceinline__ TileCarve carve(uint8_t* smem_raw, int stages) {
+  const uint32_t base = smem_u32(smem_raw);
+  const uint32_t pad = ((base + 1023u) & ~1023u) - base;
+  uint8_t* s = smem_raw + pad;
+  TileCarve c;
+  c.a = s;
+  c.b = s + (size_t)stages * kABytes;
+  c.idx = reinterpret_cast<int32_t*>(c.b + (size_t)stages * BN * kBK * 2);
+  c.bar = reinterpret_cast<TcBarriers*>(c.idx + kBM * 9);
+  return c;
+}
+
+__device__ __forceinline__ void init_barriers(TcBarriers* b, int stages) {
+  for (int s = 0; s < stages; ++s) {
+    mbar_init(&b->full[s], 4);
+    mbar_init(&b->bfull[s], 1);
+    mbar_init(&b->empty[s], 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(&b->tfull[i], 1);
+    mbar_init(&b->tempty[i], 4);
+  }
+  mbar_init(&b->done, 1);
+  b->abort_flag = 0;
+  fence_barrier_init();
+  fence_proxy_async_smem();
+}
+
+// Lane 0 of the warp waits, the verdict is broadcast: control flow stays
+// warp-uniform even when a wait gives up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                          uint64_t timeout_ns) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, err, timeout_ns);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Every thread has made its cp.async / st.shared writes to a stage visible to the
+// async proxy; lane 0 then arrives once for the warp.
+__device__ __forceinline__ void warp_publish(uint64_t* bar) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Producer exit: land every cp.async, publish the stages still owed to the MMA
+// warp, or (on abort) let lane 0 of producer warp 0 wait for its own TMA loads
+// still in flight.
+__device__ __forceinline__ void producer_drain(TcBarriers* bar, uint32_t it, int stages, int pwarp, bool aborted,
+                                               int* err, uint64_t timeout_ns) {
+  cp_async_wait<0>();
+  const uint32_t first = it >= (uint32_t)kLag ? it - kLag : 0u;
+  if (!aborted) {
+    for (uint32_t q = first; q < it; ++q) warp_publish(&bar->full[q % stages]);
+  } else if (pwarp == 0 && (threadIdx.x & 31) == 0) {
+    volatile int never = 0;
+    const uint32_t lo = it >= (uint32_t)stages ? it - stages : 0u;
+    for (uint32_t q = lo; q < it; ++q) mbar_wait(&bar->bfull[q % stages], (q / stages) & 1u, &never, err, timeout_ns);
+  }
+  __syncwarp();
+}
+
+// ============================================================================ conv / dense GEMM
+template <int BN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const int S = p.stages;
+  TileCarve sm = carve<BN>(smem_raw, S);
+  TcBarriers* bar = sm.bar;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* err = p.status;
+  constexpr uint32_t kBBytes = BN * kBK * 2;
+  constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+
+  // rows handled by this launch (device-side bounds for the chunked adapter)
+  int lo = 0, M = p.M;
+  if (p.row_lo) {
+    lo = *p.row_lo;
+    int m = *p.row_hi - lo;
+    if (m > p.M) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(err, SVCONV_STATUS_CHUNK_OVERFLOW);
+      m = p.M;
+    }
+    M = m < 0 ? 0 : m;
+  }
+  const int m_tiles = (M + kBM - 1) / kBM;
+  const int n_tiles = p.N / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int kb_per_tap = p.Kc / kBK;
+  const int num_kb = p.taps * kb_per_tap;
+  const bool gather = p.nbr != nullptr;
+
+  if (threadIdx.x == 0) {
+    init_barriers(bar, S);
+    prefetch_tmap(&p.tmap_b);
+  }
+  if (warp == 8) {
+    tmem_alloc(&bar->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bar->tmem_base;
+  volatile int* abort_flag = &bar->abort_flag;
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ producers
+    // Producer warp pw owns tile rows r = 4*pw + (lane >> 3) + 16*q (q = 0..7);
+    // lane & 7 picks the 16-byte chunk of the 128-byte row.  The warp loads the
+    // neighbour indices of exactly its own rows, so only __syncwarp is needed.
+    const int pw = warp - 4;
+    const int chunk = lane & 7;
+    const int rsub = pw * 4 + (lane >> 3);
+    uint32_t it = 0;
+    bool aborted = false;
+    const int nbr_base = p.nbr_abs ? lo : 0;
+    const int a_base = p.a_abs ? lo : 0;
+    for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
+      const int m0 = (tile / n_tiles) * kBM;
+      const int n0 = (tile % n_tiles) * BN;
+      if (gather) {
+        __syncwarp();
+        for (int e = lane; e < 32 * 9; e += 32) {
+          const int lr = e / 9, j = e - lr * 9;
+          const int r = pw * 4 + (lr & 3) + 16 * (lr >> 2);
+          const int row = m0 + r;
+          int v = -1;
+          if (row < M) {
+            v = p.nbr[(size_t)(nbr_base + row) * 9 + j];
+            if (v >= 0) {
+              v -= nbr_base;
+              if ((unsigned)v >= (unsigned)p.a_rows) {
+                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+                v = -1;
+              }
+            }
+          }
+          sm.idx[r * 9 + j] = v;
+        }
+        __syncwarp();
+      }
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const int j = kb / kb_per_tap;
+        const int cb = kb - j * kb_per_tap;
+        uint8_t* sb = sm.b + (size_t)s * kBBytes;
+        if (pw == 0 && lane == 0) {
+          mbar_arrive_expect_tx(&bar->bfull[s], kBBytes);
+          if constexpr (!B_MN) {
+            tma_load_2d(smem_u32(sb), &p.tmap_b, &bar->bfull[s], j * p.Kc + cb * kBK, n0);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_3d(smem_u32(sb + q * 8192), &p.tmap_b, &bar->bfull[s], n0 + q * 64, j, cb * kBK);
+          }
+        }
+        const int jj = p.mirror ? 8 - j : j;
+        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int r = rsub + 16 * q;
+          int src_row;
+          if (gather) {
+            src_row = sm.idx[r * 9 + jj];
+          } else {
+            const int ar = a_base + m0 + r;
+            src_row = (m0 + r < M && ar >= 0 && ar < p.a_rows) ? ar : -1;
+          }
+          const __nv_bfloat16* src =
+              p.A + (size_t)(src_row < 0 ? 0 : src_row) * p.lda + cb * kBK + chunk * 8;
+          cp_async_16(sa + r * 128 + ((chunk ^ (r & 7)) << 4), src, src_row >= 0 ? 16u : 0u);
+        }
+        cp_async_commit();
+        if (it >= (uint32_t)kLag) {
+          cp_async_wait<kLag>();
+          warp_publish(&bar->full[(it - kLag) % S]);
+        }
+      }
+    }
+    producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, B_MN ? 1 : 0);
+      uint32_t it = 0, tc = 0;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+        const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
+        if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * BN;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&bar->full[s], ph, abort_flag, err, p.timeout_ns) ||
+              !mbar_wait(&bar->bfull[s], ph, abort_flag, err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
+          const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024) : smem_desc_sw128(b0 + k * 32, 16, 1024);
+            tc_mma_bf16(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc_commit(&bar->empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&bar->tfull[ab]);
+      }
+      if (issued) {
+        volatile int never = 0;
+        tc_commit(&bar->done);
+        mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    uint32_t tc = 0;
+    const int out_base = p.out_abs ? lo : 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+      const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
+      if (!warp_wait(&bar->tfull[ab], aph, abort_flag, err, p.timeout_ns)) break;
+      tc_fence_after();
+      const int m0 = (tile / n_tiles) * kBM;
+      const int n0 = (tile % n_tiles) * BN;
+      const int row = m0 + warp * 32 + lane;
+      const int orow_i = out_base + row;
+      const bool valid = row < M && orow_i >= 0 && orow_i < p.out_rows;
+      const size_t orow = (size_t)orow_i;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
+        tmem_ld_wait();
+        if (valid) {
+          float f[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
+          if (p.bias) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c0 + q);
+          }
+          if (p.gelu) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) f[q] = 0.5f * f[q] * (1.0f + erff(f[q] * 0.70710678118654752f));
+          }
+          if (p.residual) {
+            const uint4* rp = reinterpret_cast<const uint4*>(p.residual + orow * p.ldo + n0 + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 u = rp[q];
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float2 x2 = __bfloat1622float2(h[e]);
+                f[q * 8 + 2 * e] += x2.x;
+                f[q * 8 + 2 * e + 1] += x2.y;
+              }
+            }
+          }
+          uint4* op = reinterpret_cast<uint4*>(p.out + orow * p.ldo + n0 + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[q * 8 + 2 * e], f[q * 8 + 2 * e + 1]);
+            op[q] = u;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ============================================================================ weight gradient
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_constant__ TcWgradParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const int S = p.stages;
+  TileCarve sm = carve<BN>(smem_raw, S);
+  TcBarriers* bar = sm.bar;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* err = p.status;
+  constexpr uint32_t kBBytes = BN * kBK * 2;
+  constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+
+  const int m_tiles = p.rows_pad / kBM;
+  const int n_tiles = p.Cout / BN;
+  const int num_units = m_tiles * n_tiles * p.splits;
+  const int kbt = (p.n + kBK - 1) / kBK;  // token blocks in total
+  const int wrows = 9 * p.Cin;             // real dW rows; row wrows is db
+
+  if (threadIdx.x == 0) {
+    init_barriers(bar, S);
+    prefetch_tmap(&p.tmap_dy);
+  }
+  if (warp == 8) {
+    tmem_alloc(&bar->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bar->tmem_base;
+  volatile int* abort_flag = &bar->abort_flag;
+
+  // unit -> (split, m-tile, n-tile); units of one split run side by side so the
+  // tiles of dY and the gathered X rows they share are hot in L2.
+  auto decode = [&](int u, int& sp, int& m0, int& n0, int& kb0, int& kb1) {
+    const int nt = u % n_tiles;
+    const int rest = u / n_tiles;
+    const int mt = rest % m_tiles;
+    sp = rest / m_tiles;
+    m0 = mt * kBM;
+    n0 = nt * BN;
+    kb0 = (int)((long long)kbt * sp / p.splits);
+    kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
+  };
+
+  if (warp >= 4 && warp < 8) {
+    const int pw = warp - 4;
+    const int chunk = lane & 7;
+    const int rsub = pw * 4 + (lane >> 3);  // token rows rsub + 16q, q = 0..3
+    uint32_t it = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+      int sp, m0, n0, kb0, kb1;
+      decode(u, sp, m0, n0, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const int k0 = kb * kBK;
+        uint8_t* sb = sm.b + (size_t)s * kBBytes;
+        if (pw == 0 && lane == 0) {
+          mbar_arrive_expect_tx(&bar->bfull[s], kBBytes);
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q) tma_load_2d(smem_u32(sb + q * 8192), &p.tmap_dy, &bar->bfull[s], n0 + q * 64, k0);
+        }
+        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int mh = m0 + 64 * h;  // first dW row of this 64-row half
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int kk = rsub + 16 * q;
+            const int k = k0 + kk;
+            const uint32_t dst = sa + h * 8192 + kk * 128 + ((chunk ^ (kk & 7)) << 4);
+            if (mh < wrows) {
+              const int j = mh / p.Cin, i0 = mh - j * p.Cin;
+              int src_row = -1;
+              if (k < p.n) {
+                src_row = p.nbr[(size_t)k * 9 + j];
+                if (src_row >= p.n) {
+                  atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+                  src_row = -1;
+                }
+              }
+              const __nv_bfloat16* src = p.X + (size_t)(src_row < 0 ? 0 : src_row) * p.Cin + i0 + chunk * 8;
+              cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
+            } else {
+              // the all-ones row (db) sits at dW row 9*Cin; the rest is zero padding
+              const uint32_t one = (mh == wrows && chunk == 0 && k < p.n) ? 0x3F80u : 0u;
+              st_shared_16(dst, one, 0u, 0u, 0u);
+            }
+          }
+        }
+        cp_async_commit();
+        if (it >= (uint32_t)kLag) {
+          cp_async_wait<kLag>();
+          warp_publish(&bar->full[(it - kLag) % S]);
+        }
+      }
+    }
+    producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
+  } else if (warp == 8) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 1, 1);
+      uint32_t it = 0, tc = 0;
+      bool issued = false;
+      for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+        int sp, m0, n0, kb0, kb1;
+        decode(u, sp, m0, n0, kb0, kb1);
+        const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
+        if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * BN;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&bar->full[s], ph, abort_flag, err, p.timeout_ns) ||
+              !mbar_wait(&bar->bfull[s], ph, abort_flag, err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
+          const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a0 + k * 2048, 8192, 1024);
+            const uint64_t bd = smem_desc_sw128(b0 + k * 2048, 8192, 1024);
+            tc_mma_bf16(d, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+          }
+          issued = true;
+          tc_commit(&bar->empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&bar->tfull[ab]);
+      }
+      if (issued) {
+        volatile int never = 0;
+        tc_commit(&bar->done);
+        mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    uint32_t tc = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+      int sp, m0, n0, kb0, kb1;
+      decode(u, sp, m0, n0, kb0, kb1);
+      const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
+      const bool empty_range = kb1 <= kb0;  // no MMA ran for this unit: its partial is zero
+      if (!warp_wait(&bar->tfull[ab], aph, abort_flag, err, p.timeout_ns)) break;
+      tc_fence_after();
+      const int row = m0 + warp * 32 + lane;
+      float* dst = p.partial + ((size_t)sp * p.rows_pad + row) * p.Cout + n0;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
+        tmem_ld_wait();
+        float4* o4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 w;
+          w.x = empty_range ? 0.f : __uint_as_float(v[4 * q]);
+          w.y = empty_range ? 0.f : __uint_as_float(v[4 * q + 1]);
+          w.z = empty_range ? 0.f : __uint_as_float(v[4 * q + 2]);
+          w.w = empty_range ? 0.f : __uint_as_float(v[4 * q + 3]);
+          o4[q] = w;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ============================================================================ failure-detection self test
+__global__ void timeout_selftest_kernel(int32_t* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // nothing ever arrives
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, (volatile int*)&abort_flag, status, timeout_ns);
+}
+
+// ============================================================================ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims / strides innermost first (strides in bytes, rank-1 of them).
+static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                      const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int pick_stages(int bn) {
+  const size_t budget = 220 * 1024;
+  const size_t fixed = 1024 + sizeof(int32_t) * kBM * 9 + sizeof(TcBarriers);
+  int s = (int)((budget - fixed) / stage_bytes(bn));
+  if (s > kMaxStages) s = kMaxStages;
+  return s;
+}
+
+template <int BN, bool B_MN>
+static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
+  prm.stages = pick_stages(BN);
+  const size_t smem = smem_bytes(BN, prm.stages);
+  static int done[64];
+  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, B_MN>, smem, done);
+  if (e != cudaSuccess) return e;
+  tc_conv_kernel<BN, B_MN><<<grid, kThreads, smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s) {
+  TcConvParams prm;
+  memset(&prm, 0, sizeof(prm));
+  // B operand tensor map
+  if (!a.b_mn_major) {
+    // W viewed as [w_rows][w_cols] (rows = output channels, K contiguous)
+    const uint64_t dims[2] = {(uint64_t)w_cols, (uint64_t)w_rows};
+    const uint64_t strides[1] = {(uint64_t)w_cols * 2};
+    const uint32_t box[2] = {64u, (uint32_t)bn};
+    if (!make_tmap(&prm.tmap_b, Wt, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  } else {
+    // W [Kc rows (o)][9][N cols (i)]: dims (i, j, o), box (64, 1, 64)
+    const uint64_t dims[3] = {(uint64_t)a.N, 9u, (uint64_t)a.Kc};
+    const uint64_t strides[2] = {(uint64_t)a.N * 2, (uint64_t)a.N * 9 * 2};
+    const uint32_t box[3] = {64u, 1u, 64u};
+    if (!make_tmap(&prm.tmap_b, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  prm.A = static_cast<const __nv_bfloat16*>(a.A);
+  prm.nbr = a.nbr;
+  prm.row_lo = a.row_lo;
+  prm.row_hi = a.row_hi;
+  prm.bias = a.bias;
+  prm.residual = static_cast<const __nv_bfloat16*>(a.residual);
+  prm.out = static_cast<__nv_bfloat16*>(a.out);
+  prm.status = a.status ? a.status : device_error_word();
+  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.lda = a.lda;
+  prm.a_rows = a.a_rows;
+  prm.taps = a.taps;
+  prm.mirror = a.mirror;
+  prm.Kc = a.Kc;
+  prm.M = a.M;
+  prm.a_abs = a.a_abs;
+  prm.nbr_abs = a.nbr_abs;
+  prm.out_abs = a.out_abs;
+  prm.N = a.N;
+  prm.gelu = a.gelu;
+  prm.ldo = a.ldo;
+  prm.out_rows = a.out_rows;
+  const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / bn);
+  if (tiles == 0) return cudaSuccess;
+  int grid = sm_count();
+  if (grid > tiles) grid = tiles;
+  if (bn == 256) return a.b_mn_major ? launch_conv_inst<256, true>(prm, grid, s) : launch_conv_inst<256, false>(prm, grid, s);
+  if (bn == 128) return a.b_mn_major ? launch_conv_inst<128, true>(prm, grid, s) : launch_conv_inst<128, false>(prm, grid, s);
+  if (bn == 64) return a.b_mn_major ? launch_conv_inst<64, true>(prm, grid, s) : launch_conv_inst<64, false>(prm, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+static int wgrad_bn(int Cout) { return Cout % 256 == 0 ? 256 : Cout % 128 == 0 ? 128 : 64; }
+
+void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn) {
+  const int b = wgrad_bn(Cout);
+  const int rp = ((9 * Cin + 1 + kBM - 1) / kBM) * kBM;
+  const int base_units = (rp / kBM) * (Cout / b);
+  const int kbt = (n + kBK - 1) / kBK;
+  int sp = sm_count() / base_units;
+  if (sp < 1) sp = 1;
+  if (sp > kbt) sp = kbt > 0 ? kbt : 1;
+  *splits = sp;
+  *rows_pad = rp;
+  *bn = b;
+}
+
+template <int BN>
+static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t s) {
+  prm.stages = pick_stages(BN);
+  const size_t smem = smem_bytes(BN, prm.stages);
+  static int done[64];
+  cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
+  if (e != cudaSuccess) return e;
+  tc_wgrad_kernel<BN><<<grid, kThreads, smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
+  TcWgradParams prm;
+  memset(&prm, 0, sizeof(prm));
+  int splits, rows_pad, bn;
+  tc_wgrad_plan(a.n, a.Cin, a.Cout, &splits, &rows_pad, &bn);
+  if (splits != a.splits || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
+  const uint64_t dims[2] = {(uint64_t)a.Cout, (uint64_t)a.n};
+  const uint64_t strides[1] = {(uint64_t)a.Cout * 2};
+  const uint32_t box[2] = {64u, 64u};
+  if (!make_tmap(&prm.tmap_dy, a.dY, 2, dims, strides, box)) return cudaErrorInvalidValue;
+  prm.X = static_cast<const __nv_bfloat16*>(a.X);
+  prm.nbr = a.nbr;
+  prm.partial = a.partial;
+  prm.status = device_error_word();
+  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.n = a.n;
+  prm.Cin = a.Cin;
+  prm.Cout = a.Cout;
+  prm.splits = splits;
+  prm.rows_pad = rows_pad;
+  const int units = (rows_pad / kBM) * (a.Cout / bn) * splits;
+  int grid = sm_count();
+  if (grid > units) grid = units;
+  if (bn == 256) return launch_wgrad_inst<256>(prm, grid, s);
+  if (bn == 128) return launch_wgrad_inst<128>(prm, grid, s);
+  return launch_wgrad_inst<64>(prm, grid, s);
+}
+
+cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s) {
+  timeout_selftest_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace svc

@@ -1,0 +1,77 @@
+"""CPU-side checks of the C ABI library: it builds for sm_100a, loads, exports
+every entry point the header declares, and rejects bad arguments on the host
+before touching any device (no GPU is needed for any of this)."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from sparse_convolution_pruned_b200 import build as svbuild
+from sparse_convolution_pruned_b200 import svconv as sv
+
+
+@pytest.fixture(scope="module")
+def L():
+    svbuild.build()
+    return sv.lib()
+
+
+def test_library_exports_every_declared_symbol(L):
+    declared = sv.declared_symbols()
+    assert len(declared) >= 11
+    out = subprocess.run(["nm", "-D", "--defined-only", sv.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_version_and_status_strings(L):
+    assert sv.svconv_version() == 100
+    assert sv.status_str(0) == "ok"
+    assert "NULL" in sv.status_str(-1)
+    assert "wait" in sv.status_str(sv.STATUS_TIMEOUT)
+
+
+def test_host_validation_runs_before_any_device_call(L):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # negative sizes
+    assert L.svconv_fwd(sv.BF16, fake, fake, -1, 64, 64, fake, None, fake, None) == -2
+    assert L.svconv_build_index(fake, fake, -1, 4, 4, 0, fake, None, None, None) == -2
+    assert L.svconv_build_index(fake, fake, 1, 200, 200, 0, fake, None, None, None) == -2  # H*W > 16384
+    # empty problems are no-ops
+    assert L.svconv_fwd(sv.BF16, None, None, 0, 64, 64, None, None, None, None) == 0
+    assert L.svconv_bwd_data(sv.BF16, None, None, 0, 64, 64, None, None, None) == 0
+    # NULL pointers
+    assert L.svconv_fwd(sv.BF16, None, fake, 10, 64, 64, fake, None, fake, None) == -1
+    assert L.svconv_bwd_data(sv.BF16, fake, None, 10, 64, 64, fake, fake, None) == -1
+    # adapter: channel counts must be multiples of 64
+    assert L.svconv_adapter_fwd(fake, fake, fake, 4, 10, 1000, 256, fake, fake, None, fake, 2, 64, fake, 1 << 20,
+                                None, None) == -3
+    # workspace sizes (pure host arithmetic for fp32)
+    assert sv.svconv_bwd_weight_workspace_size(sv.F32, 128, 16, 16) == 1 * (9 * 16 + 1) * 16 * 4
+    assert sv.svconv_bwd_weight_workspace_size(sv.F32, 0, 16, 16) == 0
+    assert sv.svconv_adapter_workspace_size(256, 100) == 2 * 128 * 256 * 2
+
+
+def test_no_device_means_cuda_error_not_crash(L):
+    """Without a GPU the first device query fails and the call reports it."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    fake = ctypes.c_void_p(0x1000)
+    rc = L.svconv_fwd(sv.BF16, fake, fake, 10, 64, 64, fake, None, fake, None)
+    assert rc in (-6, -7)
+
+
+def test_product_never_imports_oracle():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "sparse_convolution_pruned_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "svconv_oracle" not in text, f

@@ -1,0 +1,313 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bars (from the workload definitions): the neighbour table N and the map M are
+bit-exact; fp32 outputs satisfy |err| <= 1e-5 * (1 + |ref|) element by element;
+bf16-input outputs (fp32 accumulation) satisfy max|err| <= 2e-2 * max|ref| per
+tensor.  Full-size configurations are checked on sampled rows / entries the
+oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_convolution_pruned_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+BF16_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def sv():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_convolution_pruned_b200 import build, svconv
+    build.build()
+    assert svconv.svconv_read_error_word() == 0
+    return svconv
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def check_f32(got, ref, what):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref)
+    bad = err > F32_TOL * (1.0 + np.abs(ref))
+    assert not bad.any(), f"{what}: {bad.sum()} elements out of tolerance, max err {err.max():.3e}"
+
+
+def check_bf16(got, ref, what):
+    got = np.asarray(got, np.float64)
+    err = np.abs(got - ref).max() if ref.size else 0.0
+    lim = BF16_TOL * (np.abs(ref).max() if ref.size else 0.0)
+    assert err <= lim, f"{what}: max err {err:.4e} > {lim:.4e}"
+
+
+def gpu_index(sv, w, want_map=True):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nbr, M = sv.svconv_build_index(dev(w.coords), dev(w.frame_off), w.T, w.H, w.W, want_map=want_map, status=st)
+    torch.cuda.synchronize()
+    return nbr, M, int(st.item())
+
+
+# ------------------------------------------------------------------ index build
+INDEX_CASES = [
+    ("tiny", lambda: wl.tiny_f32()),
+    ("small_c", lambda: wl.small_c_bf16()),
+    ("large_c_fwd", lambda: wl.large_c_fwd_bf16()),
+    ("large_c_bwd", lambda: wl.large_c_bwd_bf16()),
+    ("all_kept_7x13", lambda: wl.custom_conv(seed=5, T=3, H=7, W=13, keep_frac=1.0, Cin=4, Cout=4, dtype="f32")),
+    ("one_per_frame", lambda: wl.custom_conv(seed=6, T=9, H=5, W=5, keep_frac=1 / 25, Cin=4, Cout=4, dtype="f32")),
+    ("shuffled_empty", lambda: wl.custom_conv(seed=7, T=6, H=16, W=16, keep_frac=0.4, Cin=4, Cout=4, dtype="f32",
+                                              shuffle=True, empty_frames=(0, 3, 5))),
+    ("max_grid_128x128", lambda: wl.custom_conv(seed=8, T=2, H=128, W=128, keep_frac=0.3, Cin=4, Cout=4,
+                                                dtype="f32", shuffle=True)),
+    ("single_row_1x40", lambda: wl.custom_conv(seed=9, T=4, H=1, W=40, keep_frac=0.5, Cin=4, Cout=4, dtype="f32")),
+]
+
+
+@pytest.mark.parametrize("name,make", INDEX_CASES, ids=[c[0] for c in INDEX_CASES])
+def test_index_bit_exact(sv, orc, name, make):
+    w = make()
+    ref_n, ref_m, ref_st = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W)
+    assert ref_st == 0
+    nbr, M, st = gpu_index(sv, w)
+    assert st == 0
+    np.testing.assert_array_equal(nbr.cpu().numpy(), ref_n)
+    np.testing.assert_array_equal(M.cpu().numpy(), ref_m)
+
+
+def test_index_adapter_size_and_empty(sv, orc):
+    a = wl.adapter_bf16(T=3072, D=64, R=64)  # long-video token layout; features unused here
+    ref_n, _, _ = orc.build_index(a.coords, a.frame_off, a.T, a.H, a.W, want_map=False)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nbr, _ = sv.svconv_build_index(dev(a.coords), dev(a.frame_off), a.T, a.H, a.W, status=st)
+    np.testing.assert_array_equal(nbr.cpu().numpy(), ref_n)
+    assert st.item() == 0
+    # no tokens at all: M is all -1
+    coords = torch.zeros((0, 3), dtype=torch.int32, device="cuda")
+    off = torch.zeros(5, dtype=torch.int32, device="cuda")
+    nbr, M = sv.svconv_build_index(coords, off, 4, 3, 3, want_map=True, status=st)
+    assert nbr.shape == (0, 9) and bool((M == -1).all()) and st.item() == 0
+
+
+def test_index_error_flags_match_oracle(sv, orc):
+    base = np.array([[0, 0, 0], [0, 1, 1], [1, 0, 0], [1, 1, 0]], np.int32)
+    off = np.array([0, 2, 4], np.int32)
+    cases = []
+    c = base.copy(); c[1, 2] = 2; cases.append((c, off))            # x out of range
+    c = base.copy(); c[1] = c[0]; cases.append((c, off))            # duplicate
+    c = base.copy(); c[2, 0] = 0; cases.append((c, off))            # wrong frame
+    cases.append((base, np.array([0, 3, 2], np.int32)))             # non-monotone offsets
+    cases.append((base, np.array([0, 2, 3], np.int32)))             # offsets do not end at n
+    for coords, fo in cases:
+        _, _, ref_st = orc.build_index(coords, fo, 2, 2, 2)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sv.svconv_build_index(dev(coords), dev(fo), 2, 2, 2, status=st)
+        assert int(st.item()) == ref_st, (coords.tolist(), fo.tolist(), int(st.item()), ref_st)
+    # valid input afterwards still works and leaves the library word clean
+    assert sv.svconv_read_error_word() == 0
+
+
+# ------------------------------------------------------------------ fp32 path
+F32_CASES = [
+    ("tiny_config", lambda: wl.tiny_f32()),
+    ("ragged_7x13_C8x24", lambda: wl.custom_conv(seed=21, T=5, H=7, W=13, keep_frac=0.45, Cin=8, Cout=24,
+                                                dtype="f32", shuffle=True, empty_frames=(2,))),
+    ("all_kept_C32", lambda: wl.custom_conv(seed=22, T=2, H=8, W=8, keep_frac=1.0, Cin=32, Cout=16, dtype="f32")),
+    ("C64", lambda: wl.custom_conv(seed=23, T=8, H=16, W=16, keep_frac=0.3, Cin=64, Cout=64, dtype="f32")),
+]
+
+
+@pytest.mark.parametrize("name,make", F32_CASES, ids=[c[0] for c in F32_CASES])
+def test_f32_fwd_bwd(sv, orc, name, make):
+    w = make()
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    nbr, _, _ = gpu_index(sv, w, want_map=False)
+    X, Wt, dY = dev(w.X), dev(w.Wt), dev(w.dY)
+    b = dev(w.bias) if w.bias is not None else None
+    Y = sv.svconv_fwd(X, nbr, Wt, b)
+    dX = sv.svconv_bwd_data(dY, nbr, Wt)
+    dW, db = sv.svconv_bwd_weight(dY, X, nbr)
+    torch.cuda.synchronize()
+    check_f32(Y.cpu().numpy(), orc.fwd(w.X, ref_n, w.Wt, w.bias), "Y")
+    check_f32(dX.cpu().numpy(), orc.bwd_data(w.dY, ref_n, w.Wt), "dX")
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    check_f32(dW.cpu().numpy(), rdW, "dW")
+    check_f32(db.cpu().numpy(), rdb, "db")
+    assert sv.svconv_read_error_word() == 0
+
+
+# ------------------------------------------------------------------ bf16 tensor-core path
+def run_bf16(sv, w):
+    nbr, _, st = gpu_index(sv, w, want_map=False)
+    assert st == 0
+    X, Wt, dY = dev(w.X, torch.bfloat16), dev(w.Wt, torch.bfloat16), dev(w.dY, torch.bfloat16)
+    b = dev(w.bias) if w.bias is not None else None
+    Y = sv.svconv_fwd(X, nbr, Wt, b)
+    dX = sv.svconv_bwd_data(dY, nbr, Wt)
+    dW, db = sv.svconv_bwd_weight(dY, X, nbr)
+    torch.cuda.synchronize()
+    return nbr, Y.float().cpu().numpy(), dX.float().cpu().numpy(), dW.cpu().numpy(), db.cpu().numpy()
+
+
+BF16_FULL_CASES = [
+    ("small_c_config", lambda: wl.small_c_bf16()),
+    ("C256_T24_bias", lambda: wl.large_c_fwd_bf16(T=24)),
+    ("C128x192_ragged", lambda: wl.custom_conv(seed=31, T=7, H=9, W=14, keep_frac=0.55, Cin=128, Cout=192,
+                                               dtype="bf16", shuffle=True, empty_frames=(3,))),
+    ("C64x256_one_tile_tail", lambda: wl.custom_conv(seed=32, T=3, H=6, W=7, keep_frac=0.9, Cin=64, Cout=256,
+                                                     dtype="bf16")),
+    ("C320x64_allkept", lambda: wl.custom_conv(seed=33, T=2, H=12, W=12, keep_frac=1.0, Cin=320, Cout=64,
+                                               dtype="bf16")),
+]
+
+
+@pytest.mark.parametrize("name,make", BF16_FULL_CASES, ids=[c[0] for c in BF16_FULL_CASES])
+def test_bf16_full(sv, orc, name, make):
+    w = make()
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    nbr, Y, dX, dW, db = run_bf16(sv, w)
+    check_bf16(Y, orc.fwd(w.X, ref_n, w.Wt, w.bias), "Y")
+    check_bf16(dX, orc.bwd_data(w.dY, ref_n, w.Wt), "dX")
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    check_bf16(dW, rdW, "dW")
+    check_bf16(db, rdb, "db")
+    assert sv.svconv_read_error_word() == 0
+
+
+@pytest.mark.parametrize("make", [wl.large_c_fwd_bf16, wl.large_c_bwd_bf16], ids=["large_c_fwd", "large_c_bwd"])
+def test_bf16_full_size_sampled(sv, orc, make):
+    w = make()
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    nbr, Y, dX, dW, db = run_bf16(sv, w)
+    rng = np.random.default_rng(123)
+    rows = np.unique(np.concatenate([rng.choice(w.n, 384, replace=False), [0, w.n - 1]])).astype(np.int64)
+    check_bf16(Y[rows], orc.fwd(w.X, ref_n, w.Wt, w.bias, rows=rows), "Y rows")
+    check_bf16(dX[rows], orc.bwd_data(w.dY, ref_n, w.Wt, rows=rows), "dX rows")
+    ent = np.stack([rng.integers(0, w.Cout, 1500), rng.integers(0, 9, 1500), rng.integers(0, w.Cin, 1500)], 1)
+    ent = np.concatenate([ent, [[0, 0, 0], [w.Cout - 1, 8, w.Cin - 1], [w.Cout - 1, 4, 0]]]).astype(np.int32)
+    check_bf16(dW[ent[:, 0], ent[:, 1], ent[:, 2]], orc.bwd_weight_entries(w.dY, w.X, ref_n, ent), "dW entries")
+    check_bf16(db, orc.bwd_bias(w.dY), "db")
+    assert sv.svconv_read_error_word() == 0
+
+
+def test_bf16_deterministic(sv):
+    w = wl.large_c_bwd_bf16(T=48)
+    a = run_bf16(sv, w)
+    b = run_bf16(sv, w)
+    for x, y in zip(a[1:], b[1:]):
+        assert np.array_equal(x, y)
+
+
+def test_bf16_one_token_and_empty_frames(sv, orc):
+    w = wl.custom_conv(seed=41, T=5, H=4, W=4, keep_frac=[0.0, 1 / 16, 0.0, 1.0, 0.5], Cin=64, Cout=64, dtype="bf16")
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    nbr, Y, dX, dW, db = run_bf16(sv, w)
+    check_bf16(Y, orc.fwd(w.X, ref_n, w.Wt, w.bias), "Y")
+    check_bf16(dX, orc.bwd_data(w.dY, ref_n, w.Wt), "dX")
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    check_bf16(dW, rdW, "dW")
+
+
+def test_bwd_weight_empty_input_zeroes(sv):
+    X = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    dY = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    nbr = torch.zeros((0, 9), dtype=torch.int32, device="cuda")
+    dW = torch.full((64, 9, 64), 7.0, device="cuda")
+    db = torch.full((64,), 7.0, device="cuda")
+    sv.svconv_bwd_weight(dY, X, nbr, dW=dW, db=db)
+    assert float(dW.abs().max()) == 0.0 and float(db.abs().max()) == 0.0
+
+
+# ------------------------------------------------------------------ adapter
+def adapter_gpu(sv, a, chunk_T):
+    nbr, _, st = gpu_index(sv, a, want_map=False)
+    assert st == 0
+    off = a.frame_off.astype(np.int64)
+    max_rows = int(max(off[min(t + chunk_T, a.T)] - off[t] for t in range(0, a.T, chunk_T)))
+    X = dev(a.X, torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sv.svconv_adapter_fwd(X, nbr, dev(a.frame_off), a.T, dev(a.Wd, torch.bfloat16), dev(a.Wc, torch.bfloat16),
+                          dev(a.Wu, torch.bfloat16), chunk_T=chunk_T, max_chunk_rows=max_rows, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return X
+
+
+def test_adapter_small_full(sv, orc):
+    a = wl.adapter_bf16(seed=11, T=20, D=256, R=128)
+    ref_n, _, _ = orc.build_index(a.coords, a.frame_off, a.T, a.H, a.W, want_map=False)
+    out = adapter_gpu(sv, a, chunk_T=6).float().cpu().numpy()
+    ref = orc.adapter_fwd(a.X, ref_n, 0, a.n, a.Wd, a.Wc, a.Wu)
+    check_bf16(out, ref, "adapter out")
+    check_bf16(out - a.X, ref - a.X, "adapter delta")
+
+
+def test_adapter_long_video_config(sv, orc):
+    torch.cuda.reset_peak_memory_stats()
+    a = wl.adapter_bf16()
+    ref_n, _, _ = orc.build_index(a.coords, a.frame_off, a.T, a.H, a.W, want_map=False)
+    out = adapter_gpu(sv, a, chunk_T=512)
+    peak = torch.cuda.max_memory_allocated()
+    assert peak <= 1 << 30, f"peak {peak / 2**20:.0f} MiB"
+    out = out.float().cpu().numpy()
+    for f0, f1 in [(0, 12), (a.T - 12, a.T)]:
+        r0, r1 = int(a.frame_off[f0]), int(a.frame_off[f1])
+        # whole frames are independent: hand the oracle just these rows, indices rebased
+        sub_n = np.where(ref_n[r0:r1] >= 0, ref_n[r0:r1] - r0, -1)
+        ref = orc.adapter_fwd(a.X[r0:r1], sub_n, 0, r1 - r0, a.Wd, a.Wc, a.Wu)
+        check_bf16(out[r0:r1], ref, f"adapter rows {r0}:{r1}")
+        check_bf16(out[r0:r1] - a.X[r0:r1], ref - a.X[r0:r1], f"adapter delta {r0}:{r1}")
+
+
+# ------------------------------------------------------------------ failure detection / host errors
+def test_bounded_wait_times_out_cleanly(sv):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sv.svconv_selftest_timeout(st, 20000)  # 20 ms on a barrier nothing arrives at
+    torch.cuda.synchronize()
+    assert int(st.item()) & sv.STATUS_TIMEOUT
+    # the context is still usable
+    w = wl.tiny_f32()
+    nbr, _, s2 = gpu_index(sv, w)
+    assert s2 == 0
+
+
+def test_host_errors_on_device(sv):
+    X = torch.zeros((10, 96), dtype=torch.bfloat16, device="cuda")
+    nbr = torch.zeros((10, 9), dtype=torch.int32, device="cuda")
+    Wt = torch.zeros((64, 9, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sv.SvconvError) as e:
+        sv.svconv_fwd(X, nbr, Wt)  # C_in = 96 is not a multiple of 64
+    assert e.value.code == -3
+    Wt2 = torch.zeros((64, 9, 64), dtype=torch.bfloat16, device="cuda")
+    X3 = torch.zeros((10 * 64 + 4,), dtype=torch.bfloat16, device="cuda")[4:].view(10, 64)
+    with pytest.raises(sv.SvconvError) as e:
+        sv.svconv_fwd(X3, nbr, Wt2)  # 8-byte offset: rejected
+    assert e.value.code == -4
+    dW = torch.empty((64, 9, 64), device="cuda")
+    ws = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    X4 = torch.zeros((10, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sv.SvconvError) as e:
+        sv.svconv_bwd_weight(X4, X4, nbr, dW=dW, workspace=ws)
+    assert e.value.code == -5
+
+
+def test_bad_neighbour_index_is_flagged_not_faulted(sv):
+    w = wl.custom_conv(seed=51, T=2, H=8, W=8, keep_frac=0.5, Cin=64, Cout=64, dtype="bf16")
+    nbr, _, _ = gpu_index(sv, w, want_map=False)
+    nbr[3, 2] = w.n + 1000  # outside the feature rows
+    nbr[5, 7] = -77         # negative but not -1: still zero padding
+    X = dev(w.X, torch.bfloat16)
+    Wt = dev(w.Wt, torch.bfloat16)
+    sv.svconv_fwd(X, nbr, Wt)
+    sv.svconv_bwd_data(X, nbr, Wt)
+    sv.svconv_bwd_weight(X, X, nbr)
+    assert sv.svconv_read_error_word() & sv.STATUS_BAD_INDEX
+    assert sv.svconv_read_error_word() == 0  # reading clears it

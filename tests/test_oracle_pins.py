@@ -190,6 +190,7 @@ def test_bwd_vs_torch_autograd(orc, seed, T, H, W, frac, Cin, Cout):
     np.testing.assert_allclose(dX, Xt.grad.numpy(), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(dW, Wtt.grad.numpy(), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(db, bt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(orc.bwd_bias(w.dY), bt.grad.numpy(), rtol=1e-12, atol=1e-12)
     rows = np.array([w.n - 1, 0, 3], np.int64)
     np.testing.assert_allclose(orc.bwd_data(w.dY, nbr, w.Wt, rows=rows), dX[rows], rtol=1e-13, atol=1e-13)
     ent = np.array([[0, 0, 0], [Cout - 1, 8, Cin - 1], [1, 4, 2]], np.int32)
