@@ -84,6 +84,8 @@ extern "C" {
  *              coordinates the cell holds the largest k and DUPLICATE is set.
  *   dev_status int32 device or NULL; SVCONV_STATUS_BAD_* bits are OR-ed in (the
  *              caller zeroes it).  Rows of tokens with bad coordinates are -1.
+ *              Frames are validated independently, so when BAD_OFFSETS is set
+ *              other bits may be set as well and nbr / M are undefined.
  *   Limits: H*W <= 16384, T >= 0, n >= 0.
  */
 SVCONV_API int svconv_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,

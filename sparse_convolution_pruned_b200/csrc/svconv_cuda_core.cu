@@ -2,6 +2,13 @@
 // meet an fp32 tolerance), plus the fixed-order split reduction shared by both
 // weight-gradient paths.
 //
+// Sums are compensated: every dot product uses the "Dot2" scheme of Ogita, Rump
+// and Oishi ("Accurate sum and dot product", SIAM J. Sci. Comput. 2005): the
+// rounding error of each product (recovered exactly with an FMA) and of each
+// addition (Knuth's TwoSum) is carried in a second fp32 word.  The result is as
+// accurate as if accumulated in about twice the working precision, so outputs
+// with heavy cancellation still meet an fp32 tolerance relative to the result.
+//
 //  * f32_conv_kernel: one thread per (token, output channel).  The 9 x C_src x
 //    C_dst weight block sits in shared memory, laid out so that a warp's
 //    consecutive output channels read consecutive words (no bank conflicts); the
@@ -16,6 +23,24 @@
 
 namespace svc {
 namespace {
+
+// The _rn intrinsics are never contracted into FMAs, which the error-free
+// transformations below rely on.
+struct Dot2 {
+  float s = 0.0f, c = 0.0f;
+  __device__ __forceinline__ void add(float v) {  // TwoSum(s, v), error into c
+    const float t = __fadd_rn(s, v);
+    const float z = __fsub_rn(t, s);
+    c = __fadd_rn(c, __fadd_rn(__fsub_rn(s, __fsub_rn(t, z)), __fsub_rn(v, z)));
+    s = t;
+  }
+  __device__ __forceinline__ void fma(float a, float b) {  // TwoProduct(a, b), then add
+    const float p = __fmul_rn(a, b);
+    c = __fadd_rn(c, __fmaf_rn(a, b, -p));
+    add(p);
+  }
+  __device__ __forceinline__ float value() const { return __fadd_rn(s, c); }
+};
 
 __global__ void __launch_bounds__(256) f32_conv_kernel(const float* __restrict__ src, const int32_t* __restrict__ nbr,
                                                        int n, int Csrc, int Cdst, const float* __restrict__ Wt,
@@ -39,7 +64,8 @@ __global__ void __launch_bounds__(256) f32_conv_kernel(const float* __restrict__
        e += (long long)gridDim.x * blockDim.x) {
     const int k = (int)(e / Cdst);
     const int c = (int)(e - (long long)k * Cdst);
-    float acc = bias ? bias[c] : 0.0f;
+    Dot2 acc;
+    if (bias) acc.add(bias[c]);
     for (int j = 0; j < 9; ++j) {
       const int m = nbr[(size_t)k * 9 + (mirror ? 8 - j : j)];
       if (m < 0) continue;
@@ -49,9 +75,9 @@ __global__ void __launch_bounds__(256) f32_conv_kernel(const float* __restrict__
       }
       const float* s = src + (size_t)m * Csrc;
       const float* w = sW + (size_t)j * Csrc * Cdst + c;
-      for (int q = 0; q < Csrc; ++q) acc = fmaf(w[(size_t)q * Cdst], s[q], acc);
+      for (int q = 0; q < Csrc; ++q) acc.fma(w[(size_t)q * Cdst], s[q]);
     }
-    dst[e] = acc;
+    dst[e] = acc.value();
   }
 }
 
@@ -68,7 +94,7 @@ __global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __r
        e += (long long)gridDim.x * blockDim.x) {
     const int m = (int)(e / Cout);
     const int o = (int)(e - (long long)m * Cout);
-    float acc = 0.0f;
+    Dot2 acc;
     if (m < 9 * Cin) {
       const int j = m / Cin, i = m - j * Cin;
       for (int k = k0; k < k1; ++k) {
@@ -78,12 +104,12 @@ __global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __r
           atomicOr(err, SVCONV_STATUS_BAD_INDEX);
           continue;
         }
-        acc = fmaf(dY[(size_t)k * Cout + o], X[(size_t)nb * Cin + i], acc);
+        acc.fma(dY[(size_t)k * Cout + o], X[(size_t)nb * Cin + i]);
       }
     } else {
-      for (int k = k0; k < k1; ++k) acc += dY[(size_t)k * Cout + o];
+      for (int k = k0; k < k1; ++k) acc.add(dY[(size_t)k * Cout + o]);
     }
-    partial[((size_t)sp * rows_pad + m) * Cout + o] = acc;
+    partial[((size_t)sp * rows_pad + m) * Cout + o] = acc.value();
   }
 }
 
@@ -96,10 +122,10 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
   const int tx = threadIdx.x, ty = threadIdx.y;
   for (int r = ty; r < 32; r += 8) {
     const int m = m0 + r, o = o0 + tx;
-    float s = 0.0f;
+    Dot2 s;
     if (m < rows && o < Cout)
-      for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * rows_pad + m) * Cout + o];
-    tile[r][tx] = s;
+      for (int sp = 0; sp < splits; ++sp) s.add(partial[((size_t)sp * rows_pad + m) * Cout + o]);
+    tile[r][tx] = s.value();
   }
   __syncthreads();
   for (int r = ty; r < 32; r += 8) {
