@@ -161,9 +161,20 @@ def dist_setup(n_gpus):
     return rank, local, world
 
 
-def make_inputs(seed):
+WORKLOADS = {
+    # name: (generator, base seed)
+    "small_c": ("small_c_bf16", 1),
+    "large_c_fwd": ("large_c_fwd_bf16", 2),
+    "large_c_bwd": ("large_c_bwd_bf16", 3),
+    "adapter": ("adapter_bf16", 4),
+}
+WORKLOAD = "small_c"
+
+
+def make_inputs(seed_offset=0, workload=None):
     from sparse_convolution_pruned_b200 import workloads as wl
-    return wl.small_c_bf16(seed=seed)
+    gen, seed = WORKLOADS[workload or WORKLOAD]
+    return getattr(wl, gen)(seed=seed + seed_offset)
 
 
 # ----------------------------------------------------------------------------- reference arm (CPU oracle)
@@ -181,14 +192,22 @@ def cpu_oracle_step(w, frames):
     return time.perf_counter() - t0, r1
 
 
+def oracle_frames(w, mac_budget):
+    """How many leading frames of the workload fit a budget of oracle multiply-adds."""
+    per_token = 3 * 9 * w.Cin * w.Cout  # fwd + bwd_data + bwd_weight
+    per_frame = per_token * w.n / max(1, w.T)
+    return int(max(1, min(w.T, mac_budget // max(1, per_frame))))
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import oracle
     oracle.build()
-    w = make_inputs(1)
-    frames = 96  # each step: the first 96 of the 384 frames (a quarter of the workload)
+    w = make_inputs(0)
+    # each step: the first frames of the workload, about 4e9 multiply-adds (a few seconds)
+    frames = oracle_frames(w, 4e9)
     for _ in range(args.warmup):
         cpu_oracle_step(w, frames)
     tot, toks = 0.0, 0
@@ -220,7 +239,7 @@ def run_b200(args):
 
     rank, local, world = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
-    w = make_inputs(1 + rank)  # weak scaling: each rank owns its own batch of frames
+    w = make_inputs(rank)  # weak scaling: each rank owns its own batch of frames
     n, T, Cin, Cout = w.n, w.T, w.Cin, w.Cout
 
     # pinned host inputs (the e2e leg copies these every step)
@@ -229,6 +248,7 @@ def run_b200(args):
     h_X = torch.from_numpy(w.X).to(torch.bfloat16).pin_memory()
     h_W = torch.from_numpy(w.Wt).to(torch.bfloat16).pin_memory()
     h_dY = torch.from_numpy(w.dY).to(torch.bfloat16).pin_memory()
+    bias = torch.from_numpy(w.bias).to(dev) if w.bias is not None else None
 
     coords = h_coords.to(dev)
     off = h_off.to(dev)
@@ -250,7 +270,7 @@ def run_b200(args):
 
     def step_kernels():
         sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
-        sv.svconv_fwd(X, nbr, Wt, None, Y=Y)
+        sv.svconv_fwd(X, nbr, Wt, bias, Y=Y)
         sv.svconv_bwd_data(dY, nbr, Wt, dX=dX)
         sv.svconv_bwd_weight(dY, X, nbr, dW=dW, db=db, workspace=ws)
 
@@ -265,7 +285,7 @@ def run_b200(args):
         g_fwd = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_fwd, stream=stream, capture_error_mode="relaxed"):
             sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
-            sv.svconv_fwd(X, nbr, Wt, None, Y=Y)
+            sv.svconv_fwd(X, nbr, Wt, bias, Y=Y)
     torch.cuda.synchronize()
 
     def one_step():
@@ -310,7 +330,7 @@ def run_b200(args):
     # per-kernel durations (events between the library calls on the launching stream)
     names = ["build_index", "fwd", "bwd_data", "bwd_weight"]
     calls = [lambda: sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status),
-             lambda: sv.svconv_fwd(X, nbr, Wt, None, Y=Y),
+             lambda: sv.svconv_fwd(X, nbr, Wt, bias, Y=Y),
              lambda: sv.svconv_bwd_data(dY, nbr, Wt, dX=dX),
              lambda: sv.svconv_bwd_weight(dY, X, nbr, dW=dW, db=db, workspace=ws)]
     per = {k: 0.0 for k in names}
@@ -372,18 +392,24 @@ def run_b200(args):
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        reps, dt, toks = 5, 0.0, 0
-        for _ in range(reps):  # the whole workload, 5 times (about 10 s of CPU work)
-            d, r = cpu_oracle_step(w, w.T)
+        # about 1.6e10 multiply-adds of oracle work (10-15 s on one core)
+        frames = oracle_frames(w, 1.6e10)
+        per = 3 * 9 * Cin * Cout * int(w.frame_off[frames])
+        reps = int(max(1, round(1.6e10 / per)))
+        dt, toks = 0.0, 0
+        for _ in range(reps):
+            d, r = cpu_oracle_step(w, frames)
             dt += d
             toks += r
         cpu = {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"index+fwd+bwd_data+bwd_weight on all {w.T} frames ({w.n} tokens), repeated {reps} "
-                         f"times; single-threaded C, fp64"}
+               "sample": f"index+fwd+bwd_data+bwd_weight on the first {frames} of {w.T} frames "
+                         f"({int(w.frame_off[frames])} tokens), {reps} time(s); single-threaded C, fp64"}
 
     if rank == 0:
         peaks = load_peaks()
         work = algorithmic_work(n, T, Cin, Cout)
+        if bias is not None:
+            work["fwd"]["bytes"] += 4 * Cout
         kern = {k: dict(ms=per[k], **roofline_entry(k, work[k], per[k], peaks)) for k in names}
         top = max(names, key=lambda k: per[k])
         roof = dict(kern[top])
@@ -426,7 +452,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="small_c",
+                    help="small_c (default: the headline configuration), large_c_fwd, large_c_bwd")
     args = ap.parse_args()
+    global WORKLOAD
+    WORKLOAD = args.workload
+    if args.workload == "adapter":
+        raise SystemExit("the adapter workload is timed by its own step; not wired yet")
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

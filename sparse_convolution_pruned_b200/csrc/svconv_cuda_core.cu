@@ -17,8 +17,8 @@
 //    gradient (gather through the mirrored column N[k][8-j] with W_j transposed).
 //  * f32_wgrad_partial_kernel: each split of tokens writes its partial dW rows
 //    (row m = j*C_in + i, row 9*C_in = db) to the workspace.
-//  * wgrad_reduce_kernel: sums the splits in index order (deterministic) and
-//    transposes to dW[o][j][i] through a 32x32 shared tile.
+//  * wgrad_reduce_kernel: sums the splits in index order (deterministic, and
+//    compensated) and transposes to dW[o][j][i] through a 32x32 shared tile.
 #include "svconv_internal.h"
 
 namespace svc {
@@ -113,28 +113,42 @@ __global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __r
   }
 }
 
-__global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
-                                                           int rows_pad, int Cin, int Cout, float* __restrict__ dW,
-                                                           float* __restrict__ db) {
+// One thread per (dW row m, output channel o); 32 x 32 tiles so that both the
+// partial reads (along o) and the transposed dW writes (along m) are coalesced.
+// The split sums are issued 8 loads at a time so they overlap.
+__global__ void __launch_bounds__(1024) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
+                                                            int rows_pad, int Cin, int Cout, float* __restrict__ dW,
+                                                            float* __restrict__ db) {
   __shared__ float tile[32][33];
   const int rows = 9 * Cin + 1;
   const int m0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;
-  for (int r = ty; r < 32; r += 8) {
-    const int m = m0 + r, o = o0 + tx;
+  {
+    const int m = m0 + ty, o = o0 + tx;
     Dot2 s;
-    if (m < rows && o < Cout)
-      for (int sp = 0; sp < splits; ++sp) s.add(partial[((size_t)sp * rows_pad + m) * Cout + o]);
-    tile[r][tx] = s.value();
+    if (m < rows && o < Cout) {
+      const size_t stride = (size_t)rows_pad * Cout;
+      const float* src = partial + (size_t)m * Cout + o;
+      for (int sp0 = 0; sp0 < splits; sp0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = (sp0 + q < splits) ? __ldg(src + (size_t)(sp0 + q) * stride) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (sp0 + q < splits) s.add(v[q]);
+      }
+    }
+    tile[ty][tx] = s.value();
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int o = o0 + r, m = m0 + tx;
-    if (o >= Cout) continue;
-    if (m < 9 * Cin)
-      dW[(size_t)o * 9 * Cin + m] = tile[tx][r];
-    else if (m == 9 * Cin && db)
-      db[o] = tile[tx][r];
+  {
+    const int o = o0 + ty, m = m0 + tx;
+    if (o < Cout) {
+      if (m < 9 * Cin)
+        dW[(size_t)o * 9 * Cin + m] = tile[tx][ty];
+      else if (m == 9 * Cin && db)
+        db[o] = tile[tx][ty];
+    }
   }
 }
 
@@ -177,7 +191,7 @@ cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, 
                                 float* db, cudaStream_t s) {
   const int rows = 9 * Cin + 1;
   dim3 grid((rows + 31) / 32, (Cout + 31) / 32);
-  wgrad_reduce_kernel<<<grid, dim3(32, 8), 0, s>>>(partial, splits, rows_pad, Cin, Cout, dW, db);
+  wgrad_reduce_kernel<<<grid, dim3(32, 32), 0, s>>>(partial, splits, rows_pad, Cin, Cout, dW, db);
   return cudaGetLastError();
 }
 

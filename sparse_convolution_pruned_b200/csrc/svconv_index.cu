@@ -16,11 +16,15 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
                                                           const int32_t* __restrict__ frame_off, int T, int H,
                                                           int W, int n, int32_t* __restrict__ nbr,
                                                           int32_t* __restrict__ Mout, int32_t* status) {
-  extern __shared__ int32_t sM[];  // [H][W] of this frame
+  // shared: M of this frame [H*W], then each token's packed cell (y*W + x, or -1
+  // when its coordinates are invalid) [H*W]; a valid frame holds at most H*W tokens.
+  extern __shared__ int32_t smem[];
+  const int HW = H * W;
+  int32_t* sM = smem;
+  int32_t* sCell = smem + HW;
   __shared__ int s_flags;
   __shared__ int s_lo, s_hi;
   const int t = blockIdx.x;
-  const int HW = H * W;
   if (threadIdx.x == 0) {
     int flags = 0;
     int lo = frame_off[t], hi = frame_off[t + 1];
@@ -28,6 +32,9 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
     if (t == 0 && lo != 0) flags |= SVCONV_STATUS_BAD_OFFSETS;
     if (t == T - 1 && hi != n) flags |= SVCONV_STATUS_BAD_OFFSETS;
     if (flags) lo = hi = 0;  // a segment that cannot be trusted is not touched
+    if (hi - lo > HW) {      // more tokens than cells: duplicates; only the first HW are mapped
+      flags |= SVCONV_STATUS_DUPLICATE;
+    }
     s_flags = flags;
     s_lo = lo;
     s_hi = hi;
@@ -35,32 +42,37 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   for (int c = threadIdx.x; c < HW; c += blockDim.x) sM[c] = -1;
   __syncthreads();
   const int lo = s_lo, hi = s_hi;
+  const int cnt = hi - lo;
 
   // step 1: M[y_k][x_k] = k.  With duplicates the largest k wins (deterministic).
-  for (int k = lo + threadIdx.x; k < hi; k += blockDim.x) {
+  for (int q = threadIdx.x; q < cnt; q += blockDim.x) {
+    const int k = lo + q;
     const int tt = coords[3 * k], y = coords[3 * k + 1], x = coords[3 * k + 2];
+    int cell = -1;
     if (tt != t) {
       atomicOr(&s_flags, SVCONV_STATUS_BAD_FRAME);
-      continue;
-    }
-    if (y < 0 || y >= H || x < 0 || x >= W) {
+    } else if (y < 0 || y >= H || x < 0 || x >= W) {
       atomicOr(&s_flags, SVCONV_STATUS_BAD_COORD);
-      continue;
+    } else {
+      cell = y * W + x;
+      atomicMax(&sM[cell], k);
     }
-    atomicMax(&sM[y * W + x], k);
+    if (q < HW) sCell[q] = cell;
   }
   __syncthreads();
 
   // step 2: the 9 lookups, one (k, j) entry per thread, coalesced writes.
-  const long long cnt = (long long)(hi - lo) * 9;
+  const int mapped = cnt < HW ? cnt : HW;
+  const long long total = (long long)cnt * 9;
   int32_t* out = nbr + (size_t)lo * 9;
-  for (long long e = threadIdx.x; e < cnt; e += blockDim.x) {
-    const int k = lo + (int)(e / 9);
-    const int j = (int)(e - (long long)(k - lo) * 9);
-    const int tt = coords[3 * k], y = coords[3 * k + 1], x = coords[3 * k + 2];
+  for (long long e = threadIdx.x; e < total; e += blockDim.x) {
+    const int q = (int)(e / 9);
+    const int j = (int)(e - (long long)q * 9);
     int32_t v = -1;
-    if (tt == t && y >= 0 && y < H && x >= 0 && x < W) {
-      if (j == 4 && sM[y * W + x] != k) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
+    const int cell = q < mapped ? sCell[q] : -1;
+    if (cell >= 0) {
+      const int y = cell / W, x = cell - y * W;
+      if (j == 4 && sM[cell] != lo + q) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
       const int yy = y + j / 3 - 1, xx = x + j % 3 - 1;
       if (yy >= 0 && yy < H && xx >= 0 && xx < W) v = sM[yy * W + xx];
     }
@@ -79,7 +91,7 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
 cudaError_t launch_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,
                                int32_t* nbr, int32_t* M, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const size_t smem = sizeof(int32_t) * (size_t)H * W;
+  const size_t smem = 2 * sizeof(int32_t) * (size_t)H * W;
   if (smem > 48 * 1024) {
     static int done[64];
     cudaError_t e = ensure_smem_attr(build_index_kernel, smem, done);

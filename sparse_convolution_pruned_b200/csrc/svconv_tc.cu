@@ -9,8 +9,11 @@
 //                          128-token tile row is one 128-byte segment of a
 //                          neighbour's feature row, copied with 16-byte cp.async
 //                          into the 128B-swizzled K-major layout; -1 neighbours
-//                          are zero-filled by the copy itself.  One thread also
-//                          issues the TMA load of the matching weight tile B.
+//                          are zero-filled by the copy itself.  Each thread then
+//                          arms cp.async.mbarrier.arrive, so a stage is published
+//                          when its copies land and the producers never stall on
+//                          their own loads (all pipeline stages fill at once).
+//                          One thread also issues the TMA load of the weight tile.
 //   warp 8 (MMA)           one thread issues tcgen05.mma (M=128, N=BN, K=16) into
 //                          a double-buffered fp32 accumulator in TMEM and
 //                          releases smem stages with tcgen05.commit.
@@ -46,11 +49,10 @@ constexpr int kBM = 128;                 // tile rows (tokens / dW rows) = TMEM 
 constexpr int kBK = 64;                  // bf16 elements per K-block (one 128-byte row)
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB per A stage
 constexpr int kThreads = 9 * 32;         // 4 epilogue + 4 producer + 1 MMA warp
-constexpr int kLag = 2;                  // cp.async groups kept in flight per producer thread
 constexpr int kMaxStages = 8;
 
 struct __align__(8) TcBarriers {
-  uint64_t full[kMaxStages];    // producers' cp.async data landed (one arrival per producer warp)
+  uint64_t full[kMaxStages];    // producers' cp.async data landed (one arrival per producer thread)
   uint64_t bfull[kMaxStages];   // TMA weight tile landed (expect_tx)
   uint64_t empty[kMaxStages];   // MMA finished reading the stage (tcgen05.commit)
   uint64_t tfull[2];            // accumulator buffer ready for the epilogue
@@ -118,7 +120,7 @@ __device__ __forceinline__ TileCarve carve(uint8_t* smem_raw, int stages) {
 
 __device__ __forceinline__ void init_barriers(TcBarriers* b, int stages) {
   for (int s = 0; s < stages; ++s) {
-    mbar_init(&b->full[s], 4);
+    mbar_init(&b->full[s], 128);
     mbar_init(&b->bfull[s], 1);
     mbar_init(&b->empty[s], 1);
   }
@@ -141,30 +143,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Every thread has made its cp.async / st.shared writes to a stage visible to the
-// async proxy; lane 0 then arrives once for the warp.
-__device__ __forceinline__ void warp_publish(uint64_t* bar) {
-  fence_proxy_async_smem();
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
-// Producer exit: land every cp.async, publish the stages still owed to the MMA
-// warp, or (on abort) let lane 0 of producer warp 0 wait for its own TMA loads
-// still in flight.
+// Producer exit: make sure no cp.async of this thread is still in flight and,
+// on abort, let lane 0 of producer warp 0 wait for the TMA loads it issued.
 __device__ __forceinline__ void producer_drain(TcBarriers* bar, uint32_t it, int stages, int pwarp, bool aborted,
                                                int* err, uint64_t timeout_ns) {
-  cp_async_wait<0>();
-  const uint32_t first = it >= (uint32_t)kLag ? it - kLag : 0u;
-  if (!aborted) {
-    for (uint32_t q = first; q < it; ++q) warp_publish(&bar->full[q % stages]);
-  } else if (pwarp == 0 && (threadIdx.x & 31) == 0) {
+  cp_async_wait_all();
+  if (aborted && pwarp == 0 && (threadIdx.x & 31) == 0) {
     volatile int never = 0;
     const uint32_t lo = it >= (uint32_t)stages ? it - stages : 0u;
     for (uint32_t q = lo; q < it; ++q) mbar_wait(&bar->bfull[q % stages], (q / stages) & 1u, &never, err, timeout_ns);
   }
   __syncwarp();
 }
+
+// A 16-byte row head holding bf16 1.0 followed by zeros: the source of the
+// all-ones A row that turns the weight-gradient GEMM's last row into db.
+__device__ __align__(16) uint32_t kOnesHead[4] = {0x3F80u, 0u, 0u, 0u};
 
 // ============================================================================ conv / dense GEMM
 template <int BN, bool B_MN>
@@ -282,11 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               p.A + (size_t)(src_row < 0 ? 0 : src_row) * p.lda + cb * kBK + chunk * 8;
           cp_async_16(sa + r * 128 + ((chunk ^ (r & 7)) << 4), src, src_row >= 0 ? 16u : 0u);
         }
-        cp_async_commit();
-        if (it >= (uint32_t)kLag) {
-          cp_async_wait<kLag>();
-          warp_publish(&bar->full[(it - kLag) % S]);
-        }
+        cp_async_arrive_noinc(&bar->full[s]);
       }
     }
     producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
@@ -310,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             ok = false;
             break;
           }
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
           const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
@@ -493,16 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
               cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
             } else {
               // the all-ones row (db) sits at dW row 9*Cin; the rest is zero padding
-              const uint32_t one = (mh == wrows && chunk == 0 && k < p.n) ? 0x3F80u : 0u;
-              st_shared_16(dst, one, 0u, 0u, 0u);
+              const bool one = mh == wrows && chunk == 0 && k < p.n;
+              cp_async_16(dst, kOnesHead, one ? 16u : 0u);
             }
           }
         }
-        cp_async_commit();
-        if (it >= (uint32_t)kLag) {
-          cp_async_wait<kLag>();
-          warp_publish(&bar->full[(it - kLag) % S]);
-        }
+        cp_async_arrive_noinc(&bar->full[s]);
       }
     }
     producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
@@ -527,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
             ok = false;
             break;
           }
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
           const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
