@@ -1,38 +1,39 @@
-// bf16 SparseConv2D on the 5th-generation tensor cores (tcgen05 + TMEM).
+// bf16 SparseConv2D on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA.
 //
 // After the gather, each output tile is a dense contraction (SV-TAD page, Key
 // Design 2: y_k = sum_j W_j x[N[k,j]] is a GEMM with K = 9 * C_in whose A rows
 // are gathered through the neighbour table), so it runs as a warp-specialised,
-// persistent implicit GEMM:
+// persistent implicit GEMM with every operand moved by the TMA engine:
 //
-//   warps 4-7 (producers)  gather A: for K-block (tap j, 64 channels) each
-//                          128-token tile row is one 128-byte segment of a
-//                          neighbour's feature row, copied with 16-byte cp.async
-//                          into the 128B-swizzled K-major layout; -1 neighbours
-//                          are zero-filled by the copy itself.  Each thread then
-//                          arms cp.async.mbarrier.arrive, so a stage is published
-//                          when its copies land and the producers never stall on
-//                          their own loads (all pipeline stages fill at once).
-//                          One thread also issues the TMA load of the weight tile.
-//   warp 8 (MMA)           one thread issues tcgen05.mma (M=128, N=BN, K=16) into
-//                          a double-buffered fp32 accumulator in TMEM and
-//                          releases smem stages with tcgen05.commit.
-//   warps 0-3 (epilogue)   tcgen05.ld the accumulator (warp w owns TMEM lanes
-//                          32w..32w+31 = tile rows), add bias / GELU / residual,
-//                          convert to bf16 and store, overlapping the next
-//                          tile's main loop.
+//   warp 4 (producer)    per K-block (tap j, 64 channels): lane l issues one
+//                        tile::gather4 TMA load for tile rows 4l..4l+3, i.e. four
+//                        128-byte feature-row segments picked by the neighbour
+//                        indices; an index of -1 is an out-of-range row, which the
+//                        TMA unit fills with zeros (the padding of the page's
+//                        equation).  Lane 0 also loads the weight tile B.  All of
+//                        it lands in the 128B-swizzled layout tcgen05 reads and
+//                        completes on one mbarrier (complete_tx).  The next tile's
+//                        neighbour rows are prefetched into registers while the
+//                        current tile streams.
+//   warp 5 (MMA)         one thread issues tcgen05.mma (M=128, N=BN, K=16) into a
+//                        double-buffered fp32 accumulator in TMEM and releases smem
+//                        stages with tcgen05.commit.
+//   warps 0-3 (epilogue) tcgen05.ld the accumulator (warp w owns TMEM lanes
+//                        32w..32w+31 = tile rows), add bias / GELU / residual,
+//                        convert to bf16 and store, overlapping the next tile.
 //
-// The data gradient uses the same kernel: the gather goes through the mirrored
-// column N[k][8-j] of dY, and B = W_j^T is read straight from W[o][j][i] as an
+// The data gradient is the same kernel: the gather goes through the mirrored
+// column N[k][8-j] of dY and B = W_j^T is read straight from W[o][j][i] as an
 // MN-major operand (3-D TMA box over (i, j, o)), so no transposed copy of W is
-// made.  The dense adapter projections are the same kernel with one tap and the
-// identity "gather".
+// made.  The dense adapter projections are the same kernel with one tap and a
+// plain 2-D TMA box for A.
 //
 // The weight gradient dW^T[(j,i)][o] = sum_k X[N[k,j]][i] dY[k][o] is a GEMM with
-// K = tokens: A (gathered X) and B (dY, by TMA) are both MN-major tiles.  The
-// bias gradient comes out of the same MMAs: the A row after the last (j, i) row
-// is all ones, so its accumulator row is sum_k dY[k][o].  Token ranges are split
-// over CTAs into fp32 partials, reduced afterwards in a fixed order.
+// K = tokens: A (gathered X rows, MN-major) and B (dY by TMA, MN-major).  The bias
+// gradient comes out of the same MMAs: the A row after the last (j, i) row is
+// gathered from a constant [1, 0, ..., 0] row for every valid token, so its
+// accumulator row is sum_k dY[k][o].  Token ranges are split over CTAs into fp32
+// partials, reduced afterwards in a fixed order.
 //
 // No TMA multicast is used anywhere.
 #include <cuda.h>
@@ -48,12 +49,15 @@ namespace svc {
 constexpr int kBM = 128;                 // tile rows (tokens / dW rows) = TMEM lanes
 constexpr int kBK = 64;                  // bf16 elements per K-block (one 128-byte row)
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB per A stage
-constexpr int kThreads = 9 * 32;         // 4 epilogue + 4 producer + 1 MMA warp
+constexpr int kThreads = 6 * 32;         // 4 epilogue warps, 1 producer warp, 1 MMA warp
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
 constexpr int kMaxStages = 8;
+constexpr int kIdxPerLane = 4 * 9;       // conv: 4 tile rows x 9 taps per producer lane
+constexpr int kWgChunk = 8;              // weight gradient: K-blocks whose indices are prefetched together
 
 struct __align__(8) TcBarriers {
-  uint64_t full[kMaxStages];    // producers' cp.async data landed (one arrival per producer thread)
-  uint64_t bfull[kMaxStages];   // TMA weight tile landed (expect_tx)
+  uint64_t full[kMaxStages];    // A and B of the stage landed (arrive.expect_tx + TMA complete_tx)
   uint64_t empty[kMaxStages];   // MMA finished reading the stage (tcgen05.commit)
   uint64_t tfull[2];            // accumulator buffer ready for the epilogue
   uint64_t tempty[2];           // epilogue drained the accumulator buffer (one arrival per epilogue warp)
@@ -63,8 +67,8 @@ struct __align__(8) TcBarriers {
 };
 
 struct TcConvParams {
+  CUtensorMap tmap_a;  // gather: box {64, 1}; dense: box {64, 128}
   CUtensorMap tmap_b;
-  const __nv_bfloat16* A;
   const int32_t* nbr;
   const int32_t* row_lo;
   const int32_t* row_hi;
@@ -73,14 +77,15 @@ struct TcConvParams {
   __nv_bfloat16* out;
   int* status;
   unsigned long long timeout_ns;
-  int lda, a_rows, taps, mirror, Kc;
+  int a_rows, taps, Kc;
   int M, a_abs, nbr_abs, out_abs, N;
   int gelu, ldo, out_rows, stages;
 };
 
 struct TcWgradParams {
-  CUtensorMap tmap_dy;
-  const __nv_bfloat16* X;
+  CUtensorMap tmap_x;     // X [n][Cin], box {64, 1}
+  CUtensorMap tmap_ones;  // [1][64] constant row [1, 0, ..., 0], box {64, 1}
+  CUtensorMap tmap_dy;    // dY [n][Cout], box {64, 64}
   const int32_t* nbr;
   float* partial;
   int* status;
@@ -88,14 +93,19 @@ struct TcWgradParams {
   int n, Cin, Cout, splits, rows_pad, stages;
 };
 
+// The constant row behind the all-ones A row of the weight gradient (bf16 1.0, then zeros).
+__device__ __align__(128) uint16_t kOnesRow[64] = {0x3F80u};
+
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return (2 * bn) <= 32 ? 32 : (2 * bn) <= 64 ? 64 : (2 * bn) <= 128 ? 128 : (2 * bn) <= 256 ? 256 : 512;
 }
 
 __host__ __device__ constexpr size_t stage_bytes(int bn) { return (size_t)kABytes + (size_t)bn * kBK * 2; }
 
+constexpr size_t kIdxSmemBytes = sizeof(int32_t) * kBM * 9;
+
 static size_t smem_bytes(int bn, int stages) {
-  return 1024 /* alignment slack */ + stage_bytes(bn) * stages + sizeof(int32_t) * kBM * 9 + sizeof(TcBarriers);
+  return 1024 /* alignment slack */ + stage_bytes(bn) * stages + kIdxSmemBytes + sizeof(TcBarriers);
 }
 
 struct TileCarve {
@@ -114,14 +124,13 @@ __device__ __forceinline__ TileCarve carve(uint8_t* smem_raw, int stages) {
   c.a = s;
   c.b = s + (size_t)stages * kABytes;
   c.idx = reinterpret_cast<int32_t*>(c.b + (size_t)stages * BN * kBK * 2);
-  c.bar = reinterpret_cast<TcBarriers*>(c.idx + kBM * 9);
+  c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.idx) + kIdxSmemBytes);
   return c;
 }
 
 __device__ __forceinline__ void init_barriers(TcBarriers* b, int stages) {
   for (int s = 0; s < stages; ++s) {
-    mbar_init(&b->full[s], 128);
-    mbar_init(&b->bfull[s], 1);
+    mbar_init(&b->full[s], 1);
     mbar_init(&b->empty[s], 1);
   }
   for (int i = 0; i < 2; ++i) {
@@ -143,25 +152,52 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Producer exit: make sure no cp.async of this thread is still in flight and,
-// on abort, let lane 0 of producer warp 0 wait for the TMA loads it issued.
-__device__ __forceinline__ void producer_drain(TcBarriers* bar, uint32_t it, int stages, int pwarp, bool aborted,
-                                               int* err, uint64_t timeout_ns) {
-  cp_async_wait_all();
-  if (aborted && pwarp == 0 && (threadIdx.x & 31) == 0) {
+// Producer exit after an abort: wait (bounded, ignoring the abort flag) until
+// every TMA load still in flight has landed, so none writes after the CTA exits.
+__device__ __forceinline__ void producer_drain(TcBarriers* bar, uint32_t it, int stages, bool aborted, int* err,
+                                               uint64_t timeout_ns) {
+  if (aborted && (threadIdx.x & 31) == 0) {
     volatile int never = 0;
     const uint32_t lo = it >= (uint32_t)stages ? it - stages : 0u;
-    for (uint32_t q = lo; q < it; ++q) mbar_wait(&bar->bfull[q % stages], (q / stages) & 1u, &never, err, timeout_ns);
+    for (uint32_t q = lo; q < it; ++q) mbar_wait(&bar->full[q % stages], (q / stages) & 1u, &never, err, timeout_ns);
   }
   __syncwarp();
 }
 
-// A 16-byte row head holding bf16 1.0 followed by zeros: the source of the
-// all-ones A row that turns the weight-gradient GEMM's last row into db.
-__device__ __align__(16) uint32_t kOnesHead[4] = {0x3F80u, 0u, 0u, 0u};
+// Shared-memory descriptor geometry for the MMA issuer.
+// a_step / b_step: byte advance of the descriptors' start address per K=16 step.
+struct MmaCfg {
+  uint32_t idesc;
+  uint32_t a_lbo, a_sbo, a_step;
+  uint32_t b_lbo, b_sbo, b_step;
+};
+
+// One thread issues the MMAs of one tile (num_kb K-blocks) into accumulator d.
+__device__ __forceinline__ bool mma_tile(TcBarriers* bar, const TileCarve& sm, uint32_t b_bytes, int S, uint32_t& it,
+                                         int num_kb, uint32_t d, const MmaCfg& c, volatile int* abort_flag, int* err,
+                                         uint64_t timeout_ns) {
+  for (int kb = 0; kb < num_kb; ++kb, ++it) {
+    const int s = it % S;
+    const uint32_t ph = (it / S) & 1u;
+    if (!mbar_wait(&bar->full[s], ph, abort_flag, err, timeout_ns)) return false;
+    tc_fence_after();
+    const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
+    const uint32_t b0 = smem_u32(sm.b + (size_t)s * b_bytes);
+#pragma unroll
+    for (int k = 0; k < kBK / 16; ++k) {
+      const uint64_t ad = smem_desc_sw128(a0 + k * c.a_step, c.a_lbo, c.a_sbo);
+      const uint64_t bd = smem_desc_sw128(b0 + k * c.b_step, c.b_lbo, c.b_sbo);
+      tc_mma_bf16(d, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
+    }
+    tc_commit(&bar->empty[s]);
+  }
+  return true;
+}
 
 // ============================================================================ conv / dense GEMM
-template <int BN, bool B_MN>
+// MIRROR: gather through column 8-j (data gradient), which always pairs with an
+// MN-major weight operand.
+template <int BN, bool MIRROR>
 __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
   extern __shared__ uint8_t smem_raw[];
   const int S = p.stages;
@@ -171,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   int* err = p.status;
   constexpr uint32_t kBBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  constexpr bool B_MN = MIRROR;
 
   // rows handled by this launch (device-side bounds for the chunked adapter)
   int lo = 0, M = p.M;
@@ -192,9 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     init_barriers(bar, S);
+    prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -204,116 +242,119 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ producers
-    // Producer warp pw owns tile rows r = 4*pw + (lane >> 3) + 16*q (q = 0..7);
-    // lane & 7 picks the 16-byte chunk of the 128-byte row.  The warp loads the
-    // neighbour indices of exactly its own rows, so only __syncwarp is needed.
-    const int pw = warp - 4;
-    const int chunk = lane & 7;
-    const int rsub = pw * 4 + (lane >> 3);
-    uint32_t it = 0;
-    bool aborted = false;
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
     const int nbr_base = p.nbr_abs ? lo : 0;
     const int a_base = p.a_abs ? lo : 0;
+    uint32_t it = 0;
+    bool aborted = false;
+    // Neighbour rows of a tile: raw[i] = entry (lane + 32 i) of the tile's 128 x 9
+    // block of N (coalesced loads, all in flight together), then re-read through
+    // shared memory as cur[q * 9 + j] = N[m0 + 4*lane + q][j], validated and rebased.
+    int raw[kIdxPerLane];
+    int cur[kIdxPerLane];
+    auto load_raw = [&](int tile) {
+      const int m0 = (tile / n_tiles) * kBM;
+      const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
+      const int lim = (M - m0) * 9;  // entries of valid rows
+#pragma unroll
+      for (int i = 0; i < kIdxPerLane; ++i) {
+        const int e = lane + 32 * i;
+        raw[i] = e < lim ? __ldg(src + e) : -1;
+      }
+    };
+    auto publish_raw = [&]() {
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < kIdxPerLane; ++i) {
+        int v = raw[i];
+        if (v >= 0) {
+          v -= nbr_base;
+          if ((unsigned)v >= (unsigned)p.a_rows) {
+            atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+            v = -1;
+          }
+        }
+        sm.idx[lane + 32 * i] = v;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < kIdxPerLane; ++i) cur[i] = sm.idx[lane * kIdxPerLane + i];
+    };
+    if (gather && (int)blockIdx.x < num_tiles) {
+      load_raw(blockIdx.x);
+      publish_raw();
+    }
     for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
       const int m0 = (tile / n_tiles) * kBM;
       const int n0 = (tile % n_tiles) * BN;
-      if (gather) {
-        __syncwarp();
-        for (int e = lane; e < 32 * 9; e += 32) {
-          const int lr = e / 9, j = e - lr * 9;
-          const int r = pw * 4 + (lr & 3) + 16 * (lr >> 2);
-          const int row = m0 + r;
-          int v = -1;
-          if (row < M) {
-            v = p.nbr[(size_t)(nbr_base + row) * 9 + j];
-            if (v >= 0) {
-              v -= nbr_base;
-              if ((unsigned)v >= (unsigned)p.a_rows) {
-                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-                v = -1;
-              }
-            }
-          }
-          sm.idx[r * 9 + j] = v;
-        }
-        __syncwarp();
-      }
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+      const int next = tile + gridDim.x;
+      const bool prefetch = gather && next < num_tiles;
+      // one K-block: wait for the stage, arm it, load B and A
+      auto issue = [&](int j, int cb, int y0, int y1, int y2, int y3) -> bool {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
-        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
-          aborted = true;
-          break;
-        }
-        const int j = kb / kb_per_tap;
-        const int cb = kb - j * kb_per_tap;
+        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) return false;
         uint8_t* sb = sm.b + (size_t)s * kBBytes;
-        if (pw == 0 && lane == 0) {
-          mbar_arrive_expect_tx(&bar->bfull[s], kBBytes);
+        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar->full[s], (uint32_t)kABytes + kBBytes);
           if constexpr (!B_MN) {
-            tma_load_2d(smem_u32(sb), &p.tmap_b, &bar->bfull[s], j * p.Kc + cb * kBK, n0);
+            tma_load_2d(smem_u32(sb), &p.tmap_b, &bar->full[s], j * p.Kc + cb * kBK, n0);
           } else {
 #pragma unroll
             for (int q = 0; q < BN / 64; ++q)
-              tma_load_3d(smem_u32(sb + q * 8192), &p.tmap_b, &bar->bfull[s], n0 + q * 64, j, cb * kBK);
+              tma_load_3d(smem_u32(sb + q * 8192), &p.tmap_b, &bar->full[s], n0 + q * 64, j, cb * kBK);
           }
+          if (!gather) tma_load_2d(sa, &p.tmap_a, &bar->full[s], cb * kBK, a_base + m0);
         }
-        const int jj = p.mirror ? 8 - j : j;
-        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
+        __syncwarp();
+        if (gather) tma_gather4(sa + lane * 512, &p.tmap_a, &bar->full[s], cb * kBK, y0, y1, y2, y3);
+        ++it;
+        return true;
+      };
+      if (gather) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int r = rsub + 16 * q;
-          int src_row;
-          if (gather) {
-            src_row = sm.idx[r * 9 + jj];
-          } else {
-            const int ar = a_base + m0 + r;
-            src_row = (m0 + r < M && ar >= 0 && ar < p.a_rows) ? ar : -1;
+        for (int j = 0; j < 9; ++j) {
+          const int jj = MIRROR ? 8 - j : j;
+          for (int cb = 0; cb < kb_per_tap; ++cb) {
+            if (!issue(j, cb, cur[jj], cur[9 + jj], cur[18 + jj], cur[27 + jj])) {
+              aborted = true;
+              break;
+            }
+            if (prefetch && j == 0 && cb == 0) load_raw(next);  // overlaps this tile's stream
           }
-          const __nv_bfloat16* src =
-              p.A + (size_t)(src_row < 0 ? 0 : src_row) * p.lda + cb * kBK + chunk * 8;
-          cp_async_16(sa + r * 128 + ((chunk ^ (r & 7)) << 4), src, src_row >= 0 ? 16u : 0u);
+          if (aborted) break;
         }
-        cp_async_arrive_noinc(&bar->full[s]);
+        if (!aborted && prefetch) publish_raw();
+      } else {
+        for (int cb = 0; cb < kb_per_tap; ++cb)
+          if (!issue(0, cb, 0, 0, 0, 0)) {
+            aborted = true;
+            break;
+          }
       }
     }
-    producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
-  } else if (warp == 8) {
+    producer_drain(bar, it, S, aborted, err, p.timeout_ns);
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, B_MN ? 1 : 0);
+      MmaCfg c;
+      c.idesc = idesc_bf16_f32(kBM, BN, 0, B_MN ? 1 : 0);
+      c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // A: K-major, 128-byte rows
+      if (B_MN) {
+        c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // B: MN-major, 64-wide MN groups 8 KB apart
+      } else {
+        c.b_lbo = 16, c.b_sbo = 1024, c.b_step = 32;
+      }
       uint32_t it = 0, tc = 0;
       bool issued = false;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
         const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
         if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + ab * BN;
-        bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1u;
-          if (!mbar_wait(&bar->full[s], ph, abort_flag, err, p.timeout_ns) ||
-              !mbar_wait(&bar->bfull[s], ph, abort_flag, err, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
-          const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
-#pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024) : smem_desc_sw128(b0 + k * 32, 16, 1024);
-            tc_mma_bf16(d, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-          }
-          issued = true;
-          tc_commit(&bar->empty[s]);
-        }
-        if (!ok) break;
+        issued = true;
+        if (!mma_tile(bar, sm, kBBytes, S, it, num_kb, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       if (issued) {
@@ -387,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -413,9 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     init_barriers(bar, S);
+    prefetch_tmap(&p.tmap_x);
+    prefetch_tmap(&p.tmap_ones);
     prefetch_tmap(&p.tmap_dy);
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bar->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -438,64 +481,85 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
   };
 
-  if (warp >= 4 && warp < 8) {
-    const int pw = warp - 4;
-    const int chunk = lane & 7;
-    const int rsub = pw * 4 + (lane >> 3);  // token rows rsub + 16q, q = 0..3
+  if (warp == kProducerWarp) {
+    // Lane l fills 4 token rows (4*(l & 15) .. +3) of A-half (l >> 4); the half is
+    // 64 dW rows = one (tap, 64-channel block), the all-ones row, or padding.
+    const int h = lane >> 4;
+    const int kq = 4 * (lane & 15);
     uint32_t it = 0;
     bool aborted = false;
     for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
       int sp, m0, n0, kb0, kb1;
       decode(u, sp, m0, n0, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1u;
-        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
-          aborted = true;
-          break;
-        }
-        const int k0 = kb * kBK;
-        uint8_t* sb = sm.b + (size_t)s * kBBytes;
-        if (pw == 0 && lane == 0) {
-          mbar_arrive_expect_tx(&bar->bfull[s], kBBytes);
+      const int mh = m0 + 64 * h;
+      const int kind = mh < wrows ? 0 : (mh == wrows ? 1 : 2);  // 0 gather, 1 ones, 2 padding (not loaded)
+      const int jh = kind == 0 ? mh / p.Cin : 0;
+      const int i0 = kind == 0 ? mh - jh * p.Cin : 0;
+      // padding halves are not loaded: their accumulator rows are never read
+      const uint32_t a_bytes = (m0 <= wrows ? 8192u : 0u) + (m0 + 64 <= wrows ? 8192u : 0u);
+      int cur[kWgChunk][4], nxt[kWgChunk][4];
+      auto load_chunk = [&](int kbc, int (&dst)[kWgChunk][4]) {
 #pragma unroll
-          for (int q = 0; q < BN / 64; ++q) tma_load_2d(smem_u32(sb + q * 8192), &p.tmap_dy, &bar->bfull[s], n0 + q * 64, k0);
-        }
-        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int mh = m0 + 64 * h;  // first dW row of this 64-row half
+        for (int c = 0; c < kWgChunk; ++c)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int kk = rsub + 16 * q;
-            const int k = k0 + kk;
-            const uint32_t dst = sa + h * 8192 + kk * 128 + ((chunk ^ (kk & 7)) << 4);
-            if (mh < wrows) {
-              const int j = mh / p.Cin, i0 = mh - j * p.Cin;
-              int src_row = -1;
-              if (k < p.n) {
-                src_row = p.nbr[(size_t)k * 9 + j];
-                if (src_row >= p.n) {
-                  atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-                  src_row = -1;
-                }
-              }
-              const __nv_bfloat16* src = p.X + (size_t)(src_row < 0 ? 0 : src_row) * p.Cin + i0 + chunk * 8;
-              cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
-            } else {
-              // the all-ones row (db) sits at dW row 9*Cin; the rest is zero padding
-              const bool one = mh == wrows && chunk == 0 && k < p.n;
-              cp_async_16(dst, kOnesHead, one ? 16u : 0u);
+            const int k = (kbc + c) * kBK + kq + q;
+            int v = -1;
+            if (kbc + c < kb1 && k < p.n) v = kind == 0 ? __ldg(p.nbr + (size_t)k * 9 + jh) : 0;
+            dst[c][q] = v;
+          }
+      };
+      load_chunk(kb0, cur);
+      for (int kbc = kb0; kbc < kb1 && !aborted; kbc += kWgChunk) {
+        if (kbc + kWgChunk < kb1) load_chunk(kbc + kWgChunk, nxt);
+#pragma unroll
+        for (int c = 0; c < kWgChunk; ++c) {
+          const int kb = kbc + c;
+          if (kb >= kb1) break;
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* sb = sm.b + (size_t)s * kBBytes;
+          const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar->full[s], a_bytes + kBBytes);
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_2d(smem_u32(sb + q * 8192), &p.tmap_dy, &bar->full[s], n0 + q * 64, kb * kBK);
+          }
+          __syncwarp();
+          int y[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            y[q] = cur[c][q];
+            if (kind == 0 && y[q] >= p.n) {
+              atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+              y[q] = -1;
             }
           }
+          const uint32_t dst = sa + h * 8192 + kq * 128;
+          if (kind == 0)
+            tma_gather4(dst, &p.tmap_x, &bar->full[s], i0, y[0], y[1], y[2], y[3]);
+          else if (kind == 1)
+            tma_gather4(dst, &p.tmap_ones, &bar->full[s], 0, y[0], y[1], y[2], y[3]);
+          ++it;
         }
-        cp_async_arrive_noinc(&bar->full[s]);
+#pragma unroll
+        for (int c = 0; c < kWgChunk; ++c)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cur[c][q] = nxt[c][q];
       }
     }
-    producer_drain(bar, it, S, pw, aborted, err, p.timeout_ns);
-  } else if (warp == 8) {
+    producer_drain(bar, it, S, aborted, err, p.timeout_ns);
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 1, 1);
+      MmaCfg c;
+      c.idesc = idesc_bf16_f32(kBM, BN, 1, 1);
+      c.a_lbo = 8192, c.a_sbo = 1024, c.a_step = 2048;  // both MN-major: 64-wide groups 8 KB apart
+      c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;
       uint32_t it = 0, tc = 0;
       bool issued = false;
       for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
@@ -504,30 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
         if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + ab * BN;
-        bool ok = true;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1u;
-          if (!mbar_wait(&bar->full[s], ph, abort_flag, err, p.timeout_ns) ||
-              !mbar_wait(&bar->bfull[s], ph, abort_flag, err, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_smem();
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
-          const uint32_t b0 = smem_u32(sm.b + (size_t)s * kBBytes);
-#pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a0 + k * 2048, 8192, 1024);
-            const uint64_t bd = smem_desc_sw128(b0 + k * 2048, 8192, 1024);
-            tc_mma_bf16(d, ad, bd, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
-          }
-          issued = true;
-          tc_commit(&bar->empty[s]);
-        }
-        if (!ok) break;
+        issued = true;
+        if (!mma_tile(bar, sm, kBBytes, S, it, kb1 - kb0, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns))
+          break;
         tc_commit(&bar->tfull[ab]);
       }
       if (issued) {
@@ -572,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -610,7 +653,8 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims / strides innermost first (strides in bytes, rank-1 of them).
+// bf16 tensor map with 128-byte swizzle and zero fill outside the tensor;
+// dims / strides innermost first (strides in bytes, rank-1 of them).
 static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
                       const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
@@ -628,35 +672,44 @@ static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// rows x cols (bf16, row-major) with a box of box_rows x 64
+static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {64u, box_rows};
+  return make_tmap(m, base, 2, dims, strides, box);
+}
+
 static int pick_stages(int bn) {
   const size_t budget = 220 * 1024;
-  const size_t fixed = 1024 + sizeof(int32_t) * kBM * 9 + sizeof(TcBarriers);
+  const size_t fixed = 1024 + kIdxSmemBytes + sizeof(TcBarriers);
   int s = (int)((budget - fixed) / stage_bytes(bn));
   if (s > kMaxStages) s = kMaxStages;
   return s;
 }
 
-template <int BN, bool B_MN>
+template <int BN, bool MIRROR>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
   prm.stages = pick_stages(BN);
   const size_t smem = smem_bytes(BN, prm.stages);
   static int done[64];
-  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, B_MN>, smem, done);
+  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
-  tc_conv_kernel<BN, B_MN><<<grid, kThreads, smem, s>>>(prm);
+  tc_conv_kernel<BN, MIRROR><<<grid, kThreads, smem, s>>>(prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s) {
   TcConvParams prm;
   memset(&prm, 0, sizeof(prm));
-  // B operand tensor map
+  if (a.mirror != a.b_mn_major) return cudaErrorInvalidValue;  // the data gradient pairs both
+  if (a.nbr && a.taps != 9) return cudaErrorInvalidValue;
+  // A operand: gathered rows (box 64 x 1) or a dense 128-row box
+  if (!make_rows_tmap(&prm.tmap_a, a.A, (uint64_t)a.a_rows, (uint64_t)a.lda, a.nbr ? 1u : (uint32_t)kBM))
+    return cudaErrorInvalidValue;
   if (!a.b_mn_major) {
     // W viewed as [w_rows][w_cols] (rows = output channels, K contiguous)
-    const uint64_t dims[2] = {(uint64_t)w_cols, (uint64_t)w_rows};
-    const uint64_t strides[1] = {(uint64_t)w_cols * 2};
-    const uint32_t box[2] = {64u, (uint32_t)bn};
-    if (!make_tmap(&prm.tmap_b, Wt, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_rows_tmap(&prm.tmap_b, Wt, (uint64_t)w_rows, (uint64_t)w_cols, (uint32_t)bn)) return cudaErrorInvalidValue;
   } else {
     // W [Kc rows (o)][9][N cols (i)]: dims (i, j, o), box (64, 1, 64)
     const uint64_t dims[3] = {(uint64_t)a.N, 9u, (uint64_t)a.Kc};
@@ -664,7 +717,6 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
     const uint32_t box[3] = {64u, 1u, 64u};
     if (!make_tmap(&prm.tmap_b, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  prm.A = static_cast<const __nv_bfloat16*>(a.A);
   prm.nbr = a.nbr;
   prm.row_lo = a.row_lo;
   prm.row_hi = a.row_hi;
@@ -673,10 +725,8 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   prm.out = static_cast<__nv_bfloat16*>(a.out);
   prm.status = a.status ? a.status : device_error_word();
   prm.timeout_ns = kDefaultTimeoutNs;
-  prm.lda = a.lda;
   prm.a_rows = a.a_rows;
   prm.taps = a.taps;
-  prm.mirror = a.mirror;
   prm.Kc = a.Kc;
   prm.M = a.M;
   prm.a_abs = a.a_abs;
@@ -690,9 +740,9 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   if (tiles == 0) return cudaSuccess;
   int grid = sm_count();
   if (grid > tiles) grid = tiles;
-  if (bn == 256) return a.b_mn_major ? launch_conv_inst<256, true>(prm, grid, s) : launch_conv_inst<256, false>(prm, grid, s);
-  if (bn == 128) return a.b_mn_major ? launch_conv_inst<128, true>(prm, grid, s) : launch_conv_inst<128, false>(prm, grid, s);
-  if (bn == 64) return a.b_mn_major ? launch_conv_inst<64, true>(prm, grid, s) : launch_conv_inst<64, false>(prm, grid, s);
+  if (bn == 256) return a.mirror ? launch_conv_inst<256, true>(prm, grid, s) : launch_conv_inst<256, false>(prm, grid, s);
+  if (bn == 128) return a.mirror ? launch_conv_inst<128, true>(prm, grid, s) : launch_conv_inst<128, false>(prm, grid, s);
+  if (bn == 64) return a.mirror ? launch_conv_inst<64, true>(prm, grid, s) : launch_conv_inst<64, false>(prm, grid, s);
   return cudaErrorInvalidValue;
 }
 
@@ -722,17 +772,29 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
   return cudaGetLastError();
 }
 
+static const void* ones_row_address() {
+  static const void* addr[64];
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return nullptr;
+  if (!addr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kOnesRow) != cudaSuccess) return nullptr;
+    addr[d] = p;
+  }
+  return addr[d];
+}
+
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
   TcWgradParams prm;
   memset(&prm, 0, sizeof(prm));
   int splits, rows_pad, bn;
   tc_wgrad_plan(a.n, a.Cin, a.Cout, &splits, &rows_pad, &bn);
   if (splits != a.splits || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
-  const uint64_t dims[2] = {(uint64_t)a.Cout, (uint64_t)a.n};
-  const uint64_t strides[1] = {(uint64_t)a.Cout * 2};
-  const uint32_t box[2] = {64u, 64u};
-  if (!make_tmap(&prm.tmap_dy, a.dY, 2, dims, strides, box)) return cudaErrorInvalidValue;
-  prm.X = static_cast<const __nv_bfloat16*>(a.X);
+  const void* ones = ones_row_address();
+  if (!ones) return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, 1u)) return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_ones, ones, 1u, 64u, 1u)) return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_dy, a.dY, (uint64_t)a.n, (uint64_t)a.Cout, 64u)) return cudaErrorInvalidValue;
   prm.nbr = a.nbr;
   prm.partial = a.partial;
   prm.status = device_error_word();
