@@ -1,44 +1,48 @@
-// bf16 SparseConv2D on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA.
+// bf16 SparseConv2D on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
 // After the gather, each output tile is a dense contraction (SV-TAD page, Key
 // Design 2: y_k = sum_j W_j x[N[k,j]] is a GEMM with K = 9 * C_in whose A rows
-// are gathered through the neighbour table), so it runs as a warp-specialised,
-// persistent implicit GEMM with every operand moved by the TMA engine:
+// are gathered through the neighbour table).  The kernels below run it as a
+// warp-specialised, persistent implicit GEMM.
 //
-//   warp 4 (producer)    per K-block (tap j, 64 channels): lane l issues one
-//                        tile::gather4 TMA load for tile rows 4l..4l+3, i.e. four
-//                        128-byte feature-row segments picked by the neighbour
-//                        indices; an index of -1 is an out-of-range row, which the
-//                        TMA unit fills with zeros (the padding of the page's
-//                        equation).  Lane 0 also loads the weight tile B.  All of
-//                        it lands in the 128B-swizzled layout tcgen05 reads and
-//                        completes on one mbarrier (complete_tx).  The next tile's
-//                        neighbour rows are prefetched into registers while the
-//                        current tile streams.
-//   warp 5 (MMA)         one thread issues tcgen05.mma (M=128, N=BN, K=16) into a
-//                        double-buffered fp32 accumulator in TMEM and releases smem
-//                        stages with tcgen05.commit.
-//   warps 0-3 (epilogue) tcgen05.ld the accumulator (warp w owns TMEM lanes
-//                        32w..32w+31 = tile rows), add bias / GELU / residual,
-//                        convert to bf16 and store, overlapping the next tile.
+// Gathering each neighbour row from global memory once per tap moves 9x the
+// unique bytes through L2 in 128-byte pieces, and such row gathers are limited
+// by the number of requests an SM can keep in flight.  Instead, the rows a tile
+// needs are staged once: tokens are packed frame by frame (the page's packed
+// sequence), and within a frame in raster order a neighbour is at most W + 1
+// packed rows away, so the neighbours of 128 consecutive tokens lie in one
+// short contiguous "halo" range of rows.  That range is read with a few large
+// TMA boxes, and the A tile of every tap is assembled from it in shared memory.
+// When a tile's index range is too wide for the halo buffer (for example when
+// tokens are not in raster order), its A rows are read from global memory
+// directly: the result is the same, only slower.
+//
+// Warp roles (480 threads):
+//   warps 0-3    epilogue: tcgen05.ld the fp32 accumulator (warp w owns TMEM
+//                lanes 32w..32w+31 = tile rows), bias / GELU / residual, bf16 store.
+//   warps 4-11   A builders: copy each tile row's neighbour segment from the halo
+//                into the 128B-swizzled K-major A stage (zeros for -1 = padding).
+//   warp 12      index / halo loader: reads the tile's neighbour rows, finds the
+//                halo range, issues the halo TMA boxes (or, for the dense adapter
+//                projections, the A tile itself).
+//   warp 13      weight loader: TMA of the B tile (W_j, or W_j^T straight from
+//                W[o][j][i] as an MN-major operand for the data gradient).
+//   warp 14      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16) into
+//                a double-buffered TMEM accumulator; tcgen05.commit frees stages.
 //
 // The data gradient is the same kernel: the gather goes through the mirrored
-// column N[k][8-j] of dY and B = W_j^T is read straight from W[o][j][i] as an
-// MN-major operand (3-D TMA box over (i, j, o)), so no transposed copy of W is
-// made.  The dense adapter projections are the same kernel with one tap and a
-// plain 2-D TMA box for A.
-//
-// The weight gradient dW^T[(j,i)][o] = sum_k X[N[k,j]][i] dY[k][o] is a GEMM with
-// K = tokens: A (gathered X rows, MN-major) and B (dY by TMA, MN-major).  The bias
-// gradient comes out of the same MMAs: the A row after the last (j, i) row is
-// gathered from a constant [1, 0, ..., 0] row for every valid token, so its
-// accumulator row is sum_k dY[k][o].  Token ranges are split over CTAs into fp32
-// partials, reduced afterwards in a fixed order.
+// column N[k][8-j] of dY.  The weight gradient dW^T[(j,i)][o] = sum_k X[N[k,j]][i]
+// dY[k][o] is a GEMM with K = tokens, A (gathered X, MN-major, assembled from a
+// halo per 64-token block) and B (dY by TMA, MN-major).  The bias gradient comes
+// out of the same MMAs: the A row after the last (j, i) row is 1 for every valid
+// token, so its accumulator row is sum_k dY[k][o].  Token ranges are split over
+// CTAs into fp32 partials, reduced afterwards in a fixed order.
 //
 // No TMA multicast is used anywhere.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <climits>
 #include <cstring>
 
 #include "svconv_internal.h"
@@ -46,29 +50,44 @@
 
 namespace svc {
 
-constexpr int kBM = 128;                 // tile rows (tokens / dW rows) = TMEM lanes
-constexpr int kBK = 64;                  // bf16 elements per K-block (one 128-byte row)
-constexpr int kABytes = kBM * kBK * 2;   // 16 KB per A stage
-constexpr int kThreads = 6 * 32;         // 4 epilogue warps, 1 producer warp, 1 MMA warp
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kBM = 128;                // tile rows (tokens / dW rows) = TMEM lanes
+constexpr int kBK = 64;                 // bf16 elements per K-block (one 128-byte row)
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB per A stage
+constexpr int kEpiWarps = 4;
+constexpr int kProdWarps = 8;
+constexpr int kHaloWarp = kEpiWarps + kProdWarps;  // 12
+constexpr int kBWarp = kHaloWarp + 1;              // 13
+constexpr int kMmaWarp = kBWarp + 1;               // 14
+constexpr int kThreads = (kMmaWarp + 1) * 32;      // 480
 constexpr int kMaxStages = 8;
-constexpr int kIdxPerLane = 4 * 9;       // conv: 4 tile rows x 9 taps per producer lane
-constexpr int kWgChunk = 8;              // weight gradient: K-blocks whose indices are prefetched together
+constexpr int kHaloBox = 64;                       // rows per halo TMA box
+constexpr int kConvHaloRows = 192;                 // conv halo capacity (>= 128 + 2 * (W + 1) for W <= 31)
+constexpr int kWgHaloRows = 128;                   // weight-gradient halo capacity (64-token blocks)
+constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
+constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
 
 struct __align__(8) TcBarriers {
-  uint64_t full[kMaxStages];    // A and B of the stage landed (arrive.expect_tx + TMA complete_tx)
-  uint64_t empty[kMaxStages];   // MMA finished reading the stage (tcgen05.commit)
-  uint64_t tfull[2];            // accumulator buffer ready for the epilogue
-  uint64_t tempty[2];           // epilogue drained the accumulator buffer (one arrival per epilogue warp)
-  uint64_t done;                // final MMA drain before TMEM is released
+  uint64_t afull[kMaxStages], aempty[kMaxStages];  // A stages
+  uint64_t bfull[kMaxStages], bempty[kMaxStages];  // B stages
+  uint64_t ifull[2], iempty[2];                    // neighbour-row slots (and their halos, weight gradient)
+  uint64_t hfull[2], hempty[2];                    // conv halo buffers
+  uint64_t tfull[2], tempty[2];                    // TMEM accumulators
+  uint64_t done;                                   // final MMA drain before TMEM is released
   uint32_t tmem_base;
   int abort_flag;
 };
 
+struct HaloRange {
+  int lo;        // first staged row
+  int rows;      // staged rows (0: nothing valid)
+  int fallback;  // 1: read A rows from global memory
+  int pad;
+};
+
 struct TcConvParams {
-  CUtensorMap tmap_a;  // gather: box {64, 1}; dense: box {64, 128}
+  CUtensorMap tmap_a;  // gather: halo boxes {64, 64}; dense: A tile {64, 128}
   CUtensorMap tmap_b;
+  const __nv_bfloat16* A;
   const int32_t* nbr;
   const int32_t* row_lo;
   const int32_t* row_hi;
@@ -77,65 +96,86 @@ struct TcConvParams {
   __nv_bfloat16* out;
   int* status;
   unsigned long long timeout_ns;
-  int a_rows, taps, Kc;
+  int lda, a_rows, taps, Kc;
   int M, a_abs, nbr_abs, out_abs, N;
-  int gelu, ldo, out_rows, stages;
+  int gelu, ldo, out_rows, stages_a, stages_b;
 };
 
 struct TcWgradParams {
-  CUtensorMap tmap_x;     // X [n][Cin], box {64, 1}
-  CUtensorMap tmap_ones;  // [1][64] constant row [1, 0, ..., 0], box {64, 1}
-  CUtensorMap tmap_dy;    // dY [n][Cout], box {64, 64}
+  CUtensorMap tmap_x;   // X [n][Cin], halo boxes {64, 64}
+  CUtensorMap tmap_dy;  // dY [n][Cout], box {64, 64}
+  const __nv_bfloat16* X;
   const int32_t* nbr;
   float* partial;
   int* status;
   unsigned long long timeout_ns;
-  int n, Cin, Cout, splits, rows_pad, stages;
+  int n, Cin, Cout, splits, rows_pad, stages_a, stages_b;
 };
-
-// The constant row behind the all-ones A row of the weight gradient (bf16 1.0, then zeros).
-__device__ __align__(128) uint16_t kOnesRow[64] = {0x3F80u};
 
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return (2 * bn) <= 32 ? 32 : (2 * bn) <= 64 ? 64 : (2 * bn) <= 128 ? 128 : (2 * bn) <= 256 ? 256 : 512;
 }
 
-__host__ __device__ constexpr size_t stage_bytes(int bn) { return (size_t)kABytes + (size_t)bn * kBK * 2; }
-
-constexpr size_t kIdxSmemBytes = sizeof(int32_t) * kBM * 9;
-
-static size_t smem_bytes(int bn, int stages) {
-  return 1024 /* alignment slack */ + stage_bytes(bn) * stages + kIdxSmemBytes + sizeof(TcBarriers);
-}
-
-struct TileCarve {
-  uint8_t* a;
-  uint8_t* b;
-  int32_t* idx;
+// ---------------------------------------------------------------------------- shared memory layout
+struct Carve {
+  uint8_t* a;      // A ring
+  uint8_t* b;      // B ring
+  uint8_t* halo;   // conv: 2 halo buffers; weight gradient: 2 slots x 2 halos
+  int32_t* idx;    // 2 neighbour-row slots
+  HaloRange* rng;  // 2 ranges
   TcBarriers* bar;
 };
 
-template <int BN>
-__device__ __forceinline__ TileCarve carve(uint8_t* smem_raw, int stages) {
+struct Geometry {
+  size_t a_bytes, b_bytes, halo_bytes, idx_bytes;
+};
+
+__host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb) {
+  return {(size_t)sa * kABytes, (size_t)sb * bn * kBK * 2, (size_t)2 * kConvHaloRows * 128,
+          round_up((size_t)2 * kConvIdx * 4, 16)};
+}
+
+__host__ __device__ inline Geometry wgrad_geometry(int bn, int sa, int sb) {
+  return {(size_t)sa * kABytes, (size_t)sb * bn * kBK * 2, (size_t)4 * kWgHaloRows * 128,
+          round_up((size_t)2 * kWgIdx * 4, 16)};
+}
+
+__host__ __device__ inline size_t smem_total(const Geometry& g) {
+  return 1024 + g.a_bytes + g.b_bytes + g.halo_bytes + g.idx_bytes + 2 * sizeof(HaloRange) + sizeof(TcBarriers);
+}
+
+__device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
   const uint32_t base = smem_u32(smem_raw);
   const uint32_t pad = ((base + 1023u) & ~1023u) - base;
-  uint8_t* s = smem_raw + pad;
-  TileCarve c;
-  c.a = s;
-  c.b = s + (size_t)stages * kABytes;
-  c.idx = reinterpret_cast<int32_t*>(c.b + (size_t)stages * BN * kBK * 2);
-  c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.idx) + kIdxSmemBytes);
+  Carve c;
+  c.a = smem_raw + pad;
+  c.b = c.a + g.a_bytes;
+  c.halo = c.b + g.b_bytes;
+  c.idx = reinterpret_cast<int32_t*>(c.halo + g.halo_bytes);
+  c.rng = reinterpret_cast<HaloRange*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
+  c.bar = reinterpret_cast<TcBarriers*>(c.rng + 2);
   return c;
 }
 
-__device__ __forceinline__ void init_barriers(TcBarriers* b, int stages) {
-  for (int s = 0; s < stages; ++s) {
-    mbar_init(&b->full[s], 1);
-    mbar_init(&b->empty[s], 1);
+__device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uint32_t afull_count,
+                                              uint32_t ifull_count) {
+  for (int s = 0; s < sa; ++s) {
+    mbar_init(&b->afull[s], afull_count);
+    mbar_init(&b->aempty[s], 1);
+  }
+  for (int s = 0; s < sb; ++s) {
+    mbar_init(&b->bfull[s], 1);
+    mbar_init(&b->bempty[s], 1);
   }
   for (int i = 0; i < 2; ++i) {
+    mbar_init(&b->ifull[i], ifull_count);
+    mbar_init(&b->iempty[i], kProdWarps);
+    mbar_init(&b->hfull[i], 1);
+    mbar_init(&b->hempty[i], kProdWarps);
     mbar_init(&b->tfull[i], 1);
-    mbar_init(&b->tempty[i], 4);
+    mbar_init(&b->tempty[i], kEpiWarps);
   }
   mbar_init(&b->done, 1);
   b->abort_flag = 0;
@@ -152,62 +192,100 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Producer exit after an abort: wait (bounded, ignoring the abort flag) until
-// every TMA load still in flight has landed, so none writes after the CTA exits.
-__device__ __forceinline__ void producer_drain(TcBarriers* bar, uint32_t it, int stages, bool aborted, int* err,
-                                               uint64_t timeout_ns) {
-  if (aborted && (threadIdx.x & 31) == 0) {
+// Phase bookkeeping of a ring slot used for the it-th time.
+__device__ __forceinline__ uint32_t ring_parity(uint32_t it, int depth) { return (it / (uint32_t)depth) & 1u; }
+
+// After an abort: wait (bounded, ignoring the abort flag) for the last `count`
+// arms of a TMA-fed ring, so that no copy lands after the CTA exits.
+__device__ __forceinline__ void drain_ring(uint64_t* full, uint32_t issued, int depth, int* err, uint64_t timeout_ns) {
+  if ((threadIdx.x & 31) == 0) {
     volatile int never = 0;
-    const uint32_t lo = it >= (uint32_t)stages ? it - stages : 0u;
-    for (uint32_t q = lo; q < it; ++q) mbar_wait(&bar->full[q % stages], (q / stages) & 1u, &never, err, timeout_ns);
+    const uint32_t lo = issued >= (uint32_t)depth ? issued - depth : 0u;
+    for (uint32_t q = lo; q < issued; ++q) mbar_wait(&full[q % depth], ring_parity(q, depth), &never, err, timeout_ns);
   }
   __syncwarp();
 }
 
+// Writers of generic shared memory publish a stage to the async proxy (the MMA).
+__device__ __forceinline__ void warp_publish(uint64_t* bar) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+__device__ __forceinline__ int warp_min(int v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_max(int v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ldg_16(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
 // Shared-memory descriptor geometry for the MMA issuer.
-// a_step / b_step: byte advance of the descriptors' start address per K=16 step.
 struct MmaCfg {
   uint32_t idesc;
-  uint32_t a_lbo, a_sbo, a_step;
+  uint32_t a_lbo, a_sbo, a_step;  // a_step / b_step: start-address advance per K=16 step
   uint32_t b_lbo, b_sbo, b_step;
 };
 
 // One thread issues the MMAs of one tile (num_kb K-blocks) into accumulator d.
-__device__ __forceinline__ bool mma_tile(TcBarriers* bar, const TileCarve& sm, uint32_t b_bytes, int S, uint32_t& it,
-                                         int num_kb, uint32_t d, const MmaCfg& c, volatile int* abort_flag, int* err,
-                                         uint64_t timeout_ns) {
+__device__ __forceinline__ bool mma_tile(TcBarriers* bar, const Carve& sm, uint32_t b_stage_bytes, int SA, int SB,
+                                         uint32_t& it, int num_kb, uint32_t d, const MmaCfg& c,
+                                         volatile int* abort_flag, int* err, uint64_t timeout_ns) {
   for (int kb = 0; kb < num_kb; ++kb, ++it) {
-    const int s = it % S;
-    const uint32_t ph = (it / S) & 1u;
-    if (!mbar_wait(&bar->full[s], ph, abort_flag, err, timeout_ns)) return false;
+    const int sa = it % SA, sb = it % SB;
+    if (!mbar_wait(&bar->afull[sa], ring_parity(it, SA), abort_flag, err, timeout_ns)) return false;
+    if (!mbar_wait(&bar->bfull[sb], ring_parity(it, SB), abort_flag, err, timeout_ns)) return false;
     tc_fence_after();
-    const uint32_t a0 = smem_u32(sm.a + (size_t)s * kABytes);
-    const uint32_t b0 = smem_u32(sm.b + (size_t)s * b_bytes);
+    const uint32_t a0 = smem_u32(sm.a + (size_t)sa * kABytes);
+    const uint32_t b0 = smem_u32(sm.b + (size_t)sb * b_stage_bytes);
 #pragma unroll
     for (int k = 0; k < kBK / 16; ++k) {
       const uint64_t ad = smem_desc_sw128(a0 + k * c.a_step, c.a_lbo, c.a_sbo);
       const uint64_t bd = smem_desc_sw128(b0 + k * c.b_step, c.b_lbo, c.b_sbo);
       tc_mma_bf16(d, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
     }
-    tc_commit(&bar->empty[s]);
+    tc_commit(&bar->aempty[sa]);
+    tc_commit(&bar->bempty[sb]);
   }
   return true;
 }
 
+__device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err, uint64_t timeout_ns) {
+  if (issued) {
+    volatile int never = 0;
+    tc_commit(&bar->done);
+    mbar_wait(&bar->done, 0, &never, err, timeout_ns);
+  }
+}
+
 // ============================================================================ conv / dense GEMM
-// MIRROR: gather through column 8-j (data gradient), which always pairs with an
+// MIRROR: gather through column 8-j (data gradient); it always pairs with an
 // MN-major weight operand.
 template <int BN, bool MIRROR>
 __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const int S = p.stages;
-  TileCarve sm = carve<BN>(smem_raw, S);
+  const int SA = p.stages_a, SB = p.stages_b;
+  const Geometry geo = conv_geometry(BN, SA, SB);
+  const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
   constexpr uint32_t kBBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
-  constexpr bool B_MN = MIRROR;
+  constexpr uint32_t kHaloBufBytes = kConvHaloRows * 128;
 
   // rows handled by this launch (device-side bounds for the chunked adapter)
   int lo = 0, M = p.M;
@@ -224,11 +302,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int n_tiles = p.N / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int kb_per_tap = p.Kc / kBK;
-  const int num_kb = p.taps * kb_per_tap;
+  const int taps = p.taps;
+  const int num_kb = taps * kb_per_tap;
   const bool gather = p.nbr != nullptr;
+  const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, S);
+    init_barriers(bar, SA, SB, gather ? kProdWarps : 1, 1);
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -242,107 +322,182 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    const int nbr_base = p.nbr_abs ? lo : 0;
-    const int a_base = p.a_abs ? lo : 0;
-    uint32_t it = 0;
-    bool aborted = false;
-    // Neighbour rows of a tile: raw[i] = entry (lane + 32 i) of the tile's 128 x 9
-    // block of N (coalesced loads, all in flight together), then re-read through
-    // shared memory as cur[q * 9 + j] = N[m0 + 4*lane + q][j], validated and rebased.
-    int raw[kIdxPerLane];
-    int cur[kIdxPerLane];
-    auto load_raw = [&](int tile) {
-      const int m0 = (tile / n_tiles) * kBM;
-      const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
-      const int lim = (M - m0) * 9;  // entries of valid rows
-#pragma unroll
-      for (int i = 0; i < kIdxPerLane; ++i) {
-        const int e = lane + 32 * i;
-        raw[i] = e < lim ? __ldg(src + e) : -1;
-      }
-    };
-    auto publish_raw = [&]() {
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < kIdxPerLane; ++i) {
-        int v = raw[i];
-        if (v >= 0) {
-          v -= nbr_base;
-          if ((unsigned)v >= (unsigned)p.a_rows) {
-            atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-            v = -1;
-          }
+  if (warp == kHaloWarp) {
+    // ------------------------------------------------------------ index / halo (or dense A) loader
+    if (gather) {
+      uint32_t ti = 0, hi = 0;
+      bool aborted = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
+        const int m0 = (tile / n_tiles) * kBM;
+        const int slot = ti & 1;
+        if (!warp_wait(&bar->iempty[slot], ring_parity(ti, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
         }
-        sm.idx[lane + 32 * i] = v;
-      }
-      __syncwarp();
+        // the tile's 128 x 9 neighbour entries: coalesced, all loads in flight together
+        const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
+        const int lim = min(M - m0, kBM) * 9;
+        int v[kConvIdx / 32];
 #pragma unroll
-      for (int i = 0; i < kIdxPerLane; ++i) cur[i] = sm.idx[lane * kIdxPerLane + i];
-    };
-    if (gather && (int)blockIdx.x < num_tiles) {
-      load_raw(blockIdx.x);
-      publish_raw();
-    }
-    for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
-      const int m0 = (tile / n_tiles) * kBM;
-      const int n0 = (tile % n_tiles) * BN;
-      const int next = tile + gridDim.x;
-      const bool prefetch = gather && next < num_tiles;
-      // one K-block: wait for the stage, arm it, load B and A
-      auto issue = [&](int j, int cb, int y0, int y1, int y2, int y3) -> bool {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1u;
-        if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) return false;
-        uint8_t* sb = sm.b + (size_t)s * kBBytes;
-        const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bar->full[s], (uint32_t)kABytes + kBBytes);
-          if constexpr (!B_MN) {
-            tma_load_2d(smem_u32(sb), &p.tmap_b, &bar->full[s], j * p.Kc + cb * kBK, n0);
-          } else {
-#pragma unroll
-            for (int q = 0; q < BN / 64; ++q)
-              tma_load_3d(smem_u32(sb + q * 8192), &p.tmap_b, &bar->full[s], n0 + q * 64, j, cb * kBK);
-          }
-          if (!gather) tma_load_2d(sa, &p.tmap_a, &bar->full[s], cb * kBK, a_base + m0);
+        for (int i = 0; i < kConvIdx / 32; ++i) {
+          const int e = lane + 32 * i;
+          v[i] = e < lim ? __ldg(src + e) : -1;
         }
-        __syncwarp();
-        if (gather) tma_gather4(sa + lane * 512, &p.tmap_a, &bar->full[s], cb * kBK, y0, y1, y2, y3);
-        ++it;
-        return true;
-      };
-      if (gather) {
+        int vmin = INT_MAX, vmax = -1;
+        int32_t* sidx = sm.idx + slot * kConvIdx;
 #pragma unroll
-        for (int j = 0; j < 9; ++j) {
-          const int jj = MIRROR ? 8 - j : j;
-          for (int cb = 0; cb < kb_per_tap; ++cb) {
-            if (!issue(j, cb, cur[jj], cur[9 + jj], cur[18 + jj], cur[27 + jj])) {
-              aborted = true;
-              break;
+        for (int i = 0; i < kConvIdx / 32; ++i) {
+          int x = v[i];
+          if (x >= 0) {
+            x -= nbr_base;
+            if ((unsigned)x >= (unsigned)p.a_rows) {
+              atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+              x = -1;
             }
-            if (prefetch && j == 0 && cb == 0) load_raw(next);  // overlaps this tile's stream
           }
-          if (aborted) break;
+          if (x >= 0) {
+            vmin = min(vmin, x);
+            vmax = max(vmax, x);
+          }
+          sidx[lane + 32 * i] = x;
         }
-        if (!aborted && prefetch) publish_raw();
-      } else {
-        for (int cb = 0; cb < kb_per_tap; ++cb)
-          if (!issue(0, cb, 0, 0, 0, 0)) {
+        vmin = warp_min(vmin);
+        vmax = warp_max(vmax);
+        const int rows = vmax >= 0 ? vmax - vmin + 1 : 0;
+        const bool fallback = rows == 0 || rows > kConvHaloRows;
+        if (lane == 0) sm.rng[slot] = HaloRange{vmin, rows, fallback ? 1 : 0, 0};
+        warp_arrive(&bar->ifull[slot]);  // release: the entries and the range are visible
+        if (fallback) continue;
+        const int nbox = (rows + kHaloBox - 1) / kHaloBox;
+        for (int cb = 0; cb < kb_per_tap; ++cb, ++hi) {
+          const int hb = hi & 1;
+          if (!warp_wait(&bar->hempty[hb], ring_parity(hi, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
             aborted = true;
             break;
           }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar->hfull[hb], (uint32_t)nbox * kHaloBox * 128);
+            const uint32_t dst = smem_u32(sm.halo + hb * kHaloBufBytes);
+            for (int q = 0; q < nbox; ++q)
+              tma_load_2d(dst + q * kHaloBox * 128, &p.tmap_a, &bar->hfull[hb], cb * kBK, vmin + q * kHaloBox);
+          }
+          __syncwarp();
+        }
+      }
+      if (aborted) drain_ring(bar->hfull, hi, 2, err, p.timeout_ns);
+    } else {
+      const int a_base = p.a_abs ? lo : 0;
+      uint32_t it = 0;
+      bool aborted = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
+        const int m0 = (tile / n_tiles) * kBM;
+        for (int cb = 0; cb < kb_per_tap; ++cb, ++it) {
+          const int sa = it % SA;
+          if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
+            aborted = true;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar->afull[sa], (uint32_t)kABytes);
+            tma_load_2d(smem_u32(sm.a + (size_t)sa * kABytes), &p.tmap_a, &bar->afull[sa], cb * kBK, a_base + m0);
+          }
+          __syncwarp();
+        }
+      }
+      if (aborted) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
+    }
+  } else if (warp == kBWarp) {
+    // ------------------------------------------------------------ weight loader
+    uint32_t it = 0;
+    bool aborted = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
+      const int n0 = (tile % n_tiles) * BN;
+      for (int cb = 0; cb < kb_per_tap && !aborted; ++cb)
+        for (int j = 0; j < taps; ++j, ++it) {
+          const int sb = it % SB;
+          if (!warp_wait(&bar->bempty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
+            aborted = true;
+            break;
+          }
+          if (lane == 0) {
+            const uint32_t dst = smem_u32(sm.b + (size_t)sb * kBBytes);
+            mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
+            if constexpr (!MIRROR) {
+              tma_load_2d(dst, &p.tmap_b, &bar->bfull[sb], j * p.Kc + cb * kBK, n0);
+            } else {
+#pragma unroll
+              for (int q = 0; q < BN / 64; ++q)
+                tma_load_3d(dst + q * 8192, &p.tmap_b, &bar->bfull[sb], n0 + q * 64, j, cb * kBK);
+            }
+          }
+          __syncwarp();
+        }
+    }
+    if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+  } else if (warp >= kEpiWarps && warp < kHaloWarp) {
+    // ------------------------------------------------------------ A builders
+    if (gather) {
+      const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
+      const int chunk = pt & 7;                     // 16-byte chunk of a 128-byte row
+      const int rsub = pt >> 3;                     // rows rsub + 32 q, q = 0..3
+      uint32_t ti = 0, hi = 0, it = 0;
+      bool aborted = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
+        const int slot = ti & 1;
+        if (!warp_wait(&bar->ifull[slot], ring_parity(ti, 2), abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const HaloRange rg = sm.rng[slot];
+        const int32_t* sidx = sm.idx + slot * kConvIdx;
+        for (int cb = 0; cb < kb_per_tap && !aborted; ++cb) {
+          const int hb = hi & 1;
+          if (!rg.fallback &&
+              !warp_wait(&bar->hfull[hb], ring_parity(hi, 2), abort_flag, err, p.timeout_ns)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t halo = smem_u32(sm.halo + hb * kHaloBufBytes);
+          for (int j = 0; j < 9; ++j, ++it) {
+            const int jj = MIRROR ? 8 - j : j;
+            const int sa = it % SA;
+            if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
+              aborted = true;
+              break;
+            }
+            const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int r = rsub + 32 * q;
+              const int idx = sidx[r * 9 + jj];
+              uint4 val = make_uint4(0u, 0u, 0u, 0u);
+              if (idx >= 0) {
+                if (!rg.fallback) {
+                  const int h = idx - rg.lo;
+                  val = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
+                } else {
+                  val = ldg_16(p.A + (size_t)idx * p.lda + cb * kBK + chunk * 8);
+                }
+              }
+              st_shared_v4(a_st + r * 128 + ((chunk ^ (r & 7)) << 4), val);
+            }
+            warp_publish(&bar->afull[sa]);
+          }
+          if (!rg.fallback && !aborted) {
+            warp_arrive(&bar->hempty[hb]);
+            ++hi;
+          }
+        }
+        if (!aborted) warp_arrive(&bar->iempty[slot]);
       }
     }
-    producer_drain(bar, it, S, aborted, err, p.timeout_ns);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       MmaCfg c;
-      c.idesc = idesc_bf16_f32(kBM, BN, 0, B_MN ? 1 : 0);
+      c.idesc = idesc_bf16_f32(kBM, BN, 0, MIRROR ? 1 : 0);
       c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // A: K-major, 128-byte rows
-      if (B_MN) {
+      if (MIRROR) {
         c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // B: MN-major, 64-wide MN groups 8 KB apart
       } else {
         c.b_lbo = 16, c.b_sbo = 1024, c.b_step = 32;
@@ -350,18 +505,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       uint32_t it = 0, tc = 0;
       bool issued = false;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
-        const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
-        if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        const uint32_t ab = tc & 1u;
+        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, sm, kBBytes, S, it, num_kb, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns)) break;
+        if (!mma_tile(bar, sm, kBBytes, SA, SB, it, num_kb, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns))
+          break;
         tc_commit(&bar->tfull[ab]);
       }
-      if (issued) {
-        volatile int never = 0;
-        tc_commit(&bar->done);
-        mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
-      }
+      mma_drain(bar, issued, err, p.timeout_ns);
     }
     __syncwarp();
   } else {
@@ -369,8 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     uint32_t tc = 0;
     const int out_base = p.out_abs ? lo : 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
-      const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
-      if (!warp_wait(&bar->tfull[ab], aph, abort_flag, err, p.timeout_ns)) break;
+      const uint32_t ab = tc & 1u;
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, 2), abort_flag, err, p.timeout_ns)) break;
       tc_fence_after();
       const int m0 = (tile / n_tiles) * kBM;
       const int n0 = (tile % n_tiles) * BN;
@@ -421,8 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->tempty[ab]);
+      warp_arrive(&bar->tempty[ab]);
     }
   }
 
@@ -438,13 +589,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_constant__ TcWgradParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const int S = p.stages;
-  TileCarve sm = carve<BN>(smem_raw, S);
+  const int SA = p.stages_a, SB = p.stages_b;
+  const Geometry geo = wgrad_geometry(BN, SA, SB);
+  const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
   constexpr uint32_t kBBytes = BN * kBK * 2;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
 
   const int m_tiles = p.rows_pad / kBM;
   const int n_tiles = p.Cout / BN;
@@ -453,9 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   const int wrows = 9 * p.Cin;             // real dW rows; row wrows is db
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, S);
+    init_barriers(bar, SA, SB, kProdWarps, 1);
     prefetch_tmap(&p.tmap_x);
-    prefetch_tmap(&p.tmap_ones);
     prefetch_tmap(&p.tmap_dy);
   }
   if (warp == kMmaWarp) {
@@ -469,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   volatile int* abort_flag = &bar->abort_flag;
 
   // unit -> (split, m-tile, n-tile); units of one split run side by side so the
-  // tiles of dY and the gathered X rows they share are hot in L2.
+  // tiles of dY and the X rows they share are hot in L2.
   auto decode = [&](int u, int& sp, int& m0, int& n0, int& kb0, int& kb1) {
     const int nt = u % n_tiles;
     const int rest = u / n_tiles;
@@ -480,80 +632,163 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     kb0 = (int)((long long)kbt * sp / p.splits);
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
   };
+  // the two 64-row halves of an m-tile: kind 0 = a (tap, 64-channel block) of X,
+  // kind 1 = the all-ones row (db), kind 2 = padding (never loaded: its
+  // accumulator rows are not read)
+  auto half_info = [&](int m0, int h, int& kind, int& tap, int& cblk) {
+    const int mh = m0 + 64 * h;
+    kind = mh < wrows ? 0 : (mh == wrows ? 1 : 2);
+    tap = kind == 0 ? mh / p.Cin : 0;
+    cblk = kind == 0 ? (mh - tap * p.Cin) / kBK : 0;
+  };
 
-  if (warp == kProducerWarp) {
-    // Lane l fills 4 token rows (4*(l & 15) .. +3) of A-half (l >> 4); the half is
-    // 64 dW rows = one (tap, 64-channel block), the all-ones row, or padding.
-    const int h = lane >> 4;
-    const int kq = 4 * (lane & 15);
+  if (warp == kHaloWarp) {
+    // per 64-token block: neighbour entries, their range, and one halo per
+    // distinct channel block of the tile's gathered halves, all on ifull[slot]
+    uint32_t q = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+      int sp, m0, n0, kb0, kb1;
+      decode(u, sp, m0, n0, kb0, kb1);
+      int kind0, tap0, cb0, kind1, tap1, cb1;
+      half_info(m0, 0, kind0, tap0, cb0);
+      half_info(m0, 1, kind1, tap1, cb1);
+      const bool second_halo = kind1 == 0 && !(kind0 == 0 && cb1 == cb0);
+      for (int kb = kb0; kb < kb1; ++kb, ++q) {
+        const int slot = q & 1;
+        if (!warp_wait(&bar->iempty[slot], ring_parity(q, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const int k0 = kb * kBK;
+        const int lim = min(p.n - k0, kBK) * 9;
+        const int32_t* src = p.nbr + (size_t)k0 * 9;
+        int v[kWgIdx / 32];
+#pragma unroll
+        for (int i = 0; i < kWgIdx / 32; ++i) {
+          const int e = lane + 32 * i;
+          v[i] = e < lim ? __ldg(src + e) : -1;
+        }
+        int vmin = INT_MAX, vmax = -1;
+        int32_t* sidx = sm.idx + slot * kWgIdx;
+#pragma unroll
+        for (int i = 0; i < kWgIdx / 32; ++i) {
+          int x = v[i];
+          if (x >= p.n) {
+            atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+            x = -1;
+          }
+          if (x >= 0) {
+            vmin = min(vmin, x);
+            vmax = max(vmax, x);
+          }
+          sidx[lane + 32 * i] = x < 0 ? -1 : x;
+        }
+        vmin = warp_min(vmin);
+        vmax = warp_max(vmax);
+        const int rows = vmax >= 0 ? vmax - vmin + 1 : 0;
+        const bool fallback = rows == 0 || rows > kWgHaloRows;
+        const int nbox = fallback ? 0 : (rows + kHaloBox - 1) / kHaloBox;
+        const int nhalo = fallback ? 0 : (kind0 == 0 ? 1 : 0) + (second_halo ? 1 : 0);
+        if (lane == 0) sm.rng[slot] = HaloRange{vmin, rows, fallback ? 1 : 0, 0};
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar->ifull[slot], (uint32_t)(nbox * nhalo) * kHaloBox * 128);
+          const uint32_t dst = smem_u32(sm.halo + (size_t)slot * 2 * kHaloBufBytes);
+          for (int hh = 0; hh < 2; ++hh) {
+            if (nbox == 0) break;
+            if (hh == 0 && kind0 != 0) continue;
+            if (hh == 1 && !second_halo) continue;
+            const int cb = hh == 0 ? cb0 : cb1;
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(dst + hh * kHaloBufBytes + b * kHaloBox * 128, &p.tmap_x, &bar->ifull[slot], cb * kBK,
+                          vmin + b * kHaloBox);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (aborted) drain_ring(bar->ifull, q, 2, err, p.timeout_ns);
+  } else if (warp == kBWarp) {
     uint32_t it = 0;
     bool aborted = false;
     for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
       int sp, m0, n0, kb0, kb1;
       decode(u, sp, m0, n0, kb0, kb1);
-      const int mh = m0 + 64 * h;
-      const int kind = mh < wrows ? 0 : (mh == wrows ? 1 : 2);  // 0 gather, 1 ones, 2 padding (not loaded)
-      const int jh = kind == 0 ? mh / p.Cin : 0;
-      const int i0 = kind == 0 ? mh - jh * p.Cin : 0;
-      // padding halves are not loaded: their accumulator rows are never read
-      const uint32_t a_bytes = (m0 <= wrows ? 8192u : 0u) + (m0 + 64 <= wrows ? 8192u : 0u);
-      int cur[kWgChunk][4], nxt[kWgChunk][4];
-      auto load_chunk = [&](int kbc, int (&dst)[kWgChunk][4]) {
-#pragma unroll
-        for (int c = 0; c < kWgChunk; ++c)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int k = (kbc + c) * kBK + kq + q;
-            int v = -1;
-            if (kbc + c < kb1 && k < p.n) v = kind == 0 ? __ldg(p.nbr + (size_t)k * 9 + jh) : 0;
-            dst[c][q] = v;
-          }
-      };
-      load_chunk(kb0, cur);
-      for (int kbc = kb0; kbc < kb1 && !aborted; kbc += kWgChunk) {
-        if (kbc + kWgChunk < kb1) load_chunk(kbc + kWgChunk, nxt);
-#pragma unroll
-        for (int c = 0; c < kWgChunk; ++c) {
-          const int kb = kbc + c;
-          if (kb >= kb1) break;
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1u;
-          if (!warp_wait(&bar->empty[s], ph ^ 1u, abort_flag, err, p.timeout_ns)) {
-            aborted = true;
-            break;
-          }
-          uint8_t* sb = sm.b + (size_t)s * kBBytes;
-          const uint32_t sa = smem_u32(sm.a + (size_t)s * kABytes);
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&bar->full[s], a_bytes + kBBytes);
-#pragma unroll
-            for (int q = 0; q < BN / 64; ++q)
-              tma_load_2d(smem_u32(sb + q * 8192), &p.tmap_dy, &bar->full[s], n0 + q * 64, kb * kBK);
-          }
-          __syncwarp();
-          int y[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            y[q] = cur[c][q];
-            if (kind == 0 && y[q] >= p.n) {
-              atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-              y[q] = -1;
-            }
-          }
-          const uint32_t dst = sa + h * 8192 + kq * 128;
-          if (kind == 0)
-            tma_gather4(dst, &p.tmap_x, &bar->full[s], i0, y[0], y[1], y[2], y[3]);
-          else if (kind == 1)
-            tma_gather4(dst, &p.tmap_ones, &bar->full[s], 0, y[0], y[1], y[2], y[3]);
-          ++it;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int sb = it % SB;
+        if (!warp_wait(&bar->bempty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
         }
+        if (lane == 0) {
+          const uint32_t dst = smem_u32(sm.b + (size_t)sb * kBBytes);
+          mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
 #pragma unroll
-        for (int c = 0; c < kWgChunk; ++c)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) cur[c][q] = nxt[c][q];
+          for (int q = 0; q < BN / 64; ++q)
+            tma_load_2d(dst + q * 8192, &p.tmap_dy, &bar->bfull[sb], n0 + q * 64, kb * kBK);
+        }
+        __syncwarp();
       }
     }
-    producer_drain(bar, it, S, aborted, err, p.timeout_ns);
+    if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+  } else if (warp >= kEpiWarps && warp < kHaloWarp) {
+    const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
+    const int chunk = pt & 7;
+    const int ksub = pt >> 3;  // token rows ksub and ksub + 32 of each half
+    uint32_t q = 0, it = 0;
+    bool aborted = false;
+    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+      int sp, m0, n0, kb0, kb1;
+      decode(u, sp, m0, n0, kb0, kb1);
+      int kind[2], tap[2], cblk[2];
+      half_info(m0, 0, kind[0], tap[0], cblk[0]);
+      half_info(m0, 1, kind[1], tap[1], cblk[1]);
+      const int hsel1 = (kind[0] == 0 && cblk[1] == cblk[0]) ? 0 : 1;  // halo buffer used by half 1
+      for (int kb = kb0; kb < kb1; ++kb, ++q, ++it) {
+        const int slot = q & 1;
+        if (!warp_wait(&bar->ifull[slot], ring_parity(q, 2), abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const int sa = it % SA;
+        if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        const HaloRange rg = sm.rng[slot];
+        const int32_t* sidx = sm.idx + slot * kWgIdx;
+        const uint32_t halo = smem_u32(sm.halo + (size_t)slot * 2 * kHaloBufBytes);
+        const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
+        const int k0 = kb * kBK;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (kind[h] == 2) continue;
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int kk = ksub + 32 * rr;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (kind[h] == 0) {
+              const int idx = sidx[kk * 9 + tap[h]];
+              if (idx >= 0) {
+                if (!rg.fallback) {
+                  const int hr = idx - rg.lo;
+                  const uint32_t hbase = halo + (h == 0 ? 0u : (uint32_t)hsel1 * kHaloBufBytes);
+                  val = ld_shared_16(hbase + hr * 128 + ((chunk ^ (hr & 7)) << 4));
+                } else {
+                  val = ldg_16(p.X + (size_t)idx * p.Cin + cblk[h] * kBK + chunk * 8);
+                }
+              }
+            } else if (chunk == 0 && k0 + kk < p.n) {
+              val.x = 0x3F80u;  // bf16 1.0 in element 0
+            }
+            st_shared_v4(a_st + h * 8192 + kk * 128 + ((chunk ^ (kk & 7)) << 4), val);
+          }
+        }
+        warp_publish(&bar->afull[sa]);
+        warp_arrive(&bar->iempty[slot]);
+      }
+    }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       MmaCfg c;
@@ -565,19 +800,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
         int sp, m0, n0, kb0, kb1;
         decode(u, sp, m0, n0, kb0, kb1);
-        const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
-        if (!mbar_wait(&bar->tempty[ab], aph ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        const uint32_t ab = tc & 1u;
+        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, sm, kBBytes, S, it, kb1 - kb0, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns))
+        if (!mma_tile(bar, sm, kBBytes, SA, SB, it, kb1 - kb0, tmem_base + ab * BN, c, abort_flag, err,
+                      p.timeout_ns))
           break;
         tc_commit(&bar->tfull[ab]);
       }
-      if (issued) {
-        volatile int never = 0;
-        tc_commit(&bar->done);
-        mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
-      }
+      mma_drain(bar, issued, err, p.timeout_ns);
     }
     __syncwarp();
   } else {
@@ -585,9 +817,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
       int sp, m0, n0, kb0, kb1;
       decode(u, sp, m0, n0, kb0, kb1);
-      const uint32_t ab = tc & 1u, aph = (tc >> 1) & 1u;
+      const uint32_t ab = tc & 1u;
       const bool empty_range = kb1 <= kb0;  // no MMA ran for this unit: its partial is zero
-      if (!warp_wait(&bar->tfull[ab], aph, abort_flag, err, p.timeout_ns)) break;
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, 2), abort_flag, err, p.timeout_ns)) break;
       tc_fence_after();
       const int row = m0 + warp * 32 + lane;
       float* dst = p.partial + ((size_t)sp * p.rows_pad + row) * p.Cout + n0;
@@ -608,8 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->tempty[ab]);
+      warp_arrive(&bar->tempty[ab]);
     }
   }
 
@@ -680,18 +911,30 @@ static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint
   return make_tmap(m, base, 2, dims, strides, box);
 }
 
-static int pick_stages(int bn) {
+// Stage counts: up to 4 A stages (built in shared memory, short latency) and as
+// many B stages (TMA from L2) as fit in about 220 KB of shared memory.
+static void pick_stages(bool wgrad, int bn, int* sa, int* sb) {
   const size_t budget = 220 * 1024;
-  const size_t fixed = 1024 + kIdxSmemBytes + sizeof(TcBarriers);
-  int s = (int)((budget - fixed) / stage_bytes(bn));
-  if (s > kMaxStages) s = kMaxStages;
-  return s;
+  for (int a = 4; a >= 2; --a) {
+    int b_best = 0;
+    for (int b = 2; b <= kMaxStages; ++b) {
+      const Geometry g = wgrad ? wgrad_geometry(bn, a, b) : conv_geometry(bn, a, b);
+      if (smem_total(g) <= budget) b_best = b;
+    }
+    if (b_best >= 3 || (a == 2 && b_best >= 2)) {
+      *sa = a;
+      *sb = b_best;
+      return;
+    }
+  }
+  *sa = 2;
+  *sb = 2;
 }
 
 template <int BN, bool MIRROR>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
-  prm.stages = pick_stages(BN);
-  const size_t smem = smem_bytes(BN, prm.stages);
+  pick_stages(false, BN, &prm.stages_a, &prm.stages_b);
+  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
@@ -704,8 +947,8 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   memset(&prm, 0, sizeof(prm));
   if (a.mirror != a.b_mn_major) return cudaErrorInvalidValue;  // the data gradient pairs both
   if (a.nbr && a.taps != 9) return cudaErrorInvalidValue;
-  // A operand: gathered rows (box 64 x 1) or a dense 128-row box
-  if (!make_rows_tmap(&prm.tmap_a, a.A, (uint64_t)a.a_rows, (uint64_t)a.lda, a.nbr ? 1u : (uint32_t)kBM))
+  // A operand: halo boxes of 64 rows (gather) or the 128-row tile itself (dense)
+  if (!make_rows_tmap(&prm.tmap_a, a.A, (uint64_t)a.a_rows, (uint64_t)a.lda, a.nbr ? (uint32_t)kHaloBox : (uint32_t)kBM))
     return cudaErrorInvalidValue;
   if (!a.b_mn_major) {
     // W viewed as [w_rows][w_cols] (rows = output channels, K contiguous)
@@ -717,6 +960,7 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
     const uint32_t box[3] = {64u, 1u, 64u};
     if (!make_tmap(&prm.tmap_b, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
+  prm.A = static_cast<const __nv_bfloat16*>(a.A);
   prm.nbr = a.nbr;
   prm.row_lo = a.row_lo;
   prm.row_hi = a.row_hi;
@@ -725,6 +969,7 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   prm.out = static_cast<__nv_bfloat16*>(a.out);
   prm.status = a.status ? a.status : device_error_word();
   prm.timeout_ns = kDefaultTimeoutNs;
+  prm.lda = a.lda;
   prm.a_rows = a.a_rows;
   prm.taps = a.taps;
   prm.Kc = a.Kc;
@@ -763,25 +1008,13 @@ void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn
 
 template <int BN>
 static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t s) {
-  prm.stages = pick_stages(BN);
-  const size_t smem = smem_bytes(BN, prm.stages);
+  pick_stages(true, BN, &prm.stages_a, &prm.stages_b);
+  const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_a, prm.stages_b));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
   if (e != cudaSuccess) return e;
   tc_wgrad_kernel<BN><<<grid, kThreads, smem, s>>>(prm);
   return cudaGetLastError();
-}
-
-static const void* ones_row_address() {
-  static const void* addr[64];
-  int d = 0;
-  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return nullptr;
-  if (!addr[d]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, kOnesRow) != cudaSuccess) return nullptr;
-    addr[d] = p;
-  }
-  return addr[d];
 }
 
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
@@ -790,11 +1023,10 @@ cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
   int splits, rows_pad, bn;
   tc_wgrad_plan(a.n, a.Cin, a.Cout, &splits, &rows_pad, &bn);
   if (splits != a.splits || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
-  const void* ones = ones_row_address();
-  if (!ones) return cudaErrorInvalidValue;
-  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, 1u)) return cudaErrorInvalidValue;
-  if (!make_rows_tmap(&prm.tmap_ones, ones, 1u, 64u, 1u)) return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kHaloBox))
+    return cudaErrorInvalidValue;
   if (!make_rows_tmap(&prm.tmap_dy, a.dY, (uint64_t)a.n, (uint64_t)a.Cout, 64u)) return cudaErrorInvalidValue;
+  prm.X = static_cast<const __nv_bfloat16*>(a.X);
   prm.nbr = a.nbr;
   prm.partial = a.partial;
   prm.status = device_error_word();
