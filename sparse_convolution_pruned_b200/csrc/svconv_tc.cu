@@ -436,9 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders
-    // K-blocks are built two at a time (one proxy fence per pair: the fence waits
-    // for the thread's stores to drain, so it is amortised), all loads of a pair
-    // issued before its stores.
     if (gather) {
       const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
       const int chunk = pt & 7;                     // 16-byte chunk of a 128-byte row
@@ -453,77 +450,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         }
         const HaloRange rg = sm.rng[slot];
         const int32_t* sidx = sm.idx + slot * kConvIdx;
-        const uint32_t hi0 = hi;  // halo of channel block cb is number hi0 + cb
-        for (int kb = 0; kb < num_kb && !aborted; kb += 2) {
-          const int ng = num_kb - kb < 2 ? num_kb - kb : 2;
-          int idx[2][4];
-          uint4 val[2][4];
-          uint32_t dst[2];
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g >= ng) break;
-            const int k = kb + g;
-            const int cb = k / 9, j = k - cb * 9;
+        for (int cb = 0; cb < kb_per_tap && !aborted; ++cb) {
+          const int hb = hi & 1;
+          if (!rg.fallback &&
+              !warp_wait(&bar->hfull[hb], ring_parity(hi, 2), abort_flag, err, p.timeout_ns)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t halo = smem_u32(sm.halo + hb * kHaloBufBytes);
+          for (int j = 0; j < 9; ++j, ++it) {
             const int jj = MIRROR ? 8 - j : j;
-            if (j == 0 && !rg.fallback &&
-                !warp_wait(&bar->hfull[(hi0 + cb) & 1], ring_parity(hi0 + cb, 2), abort_flag, err, p.timeout_ns)) {
+            const int sa = it % SA;
+            if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
               aborted = true;
               break;
             }
-            const int sa = (it + g) % SA;
-            if (!warp_wait(&bar->aempty[sa], ring_parity(it + g, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
-              aborted = true;
-              break;
-            }
-            dst[g] = smem_u32(sm.a + (size_t)sa * kABytes);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) idx[g][q] = sidx[(rsub + 32 * q) * 9 + jj];
-          }
-          if (aborted) break;
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g >= ng) break;
-            const int cb = (kb + g) / 9;
-            const uint32_t halo = smem_u32(sm.halo + ((hi0 + cb) & 1) * kHaloBufBytes);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int x = idx[g][q];
-              val[g][q] = make_uint4(0u, 0u, 0u, 0u);
-              if (x >= 0) {
-                if (!rg.fallback) {
-                  const int h = x - rg.lo;
-                  val[g][q] = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
-                } else {
-                  val[g][q] = ldg_16(p.A + (size_t)x * p.lda + cb * kBK + chunk * 8);
-                }
-              }
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g >= ng) break;
+            const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int r = rsub + 32 * q;
-              st_shared_v4(dst[g] + r * 128 + ((chunk ^ (r & 7)) << 4), val[g][q]);
+              const int idx = sidx[r * 9 + jj];
+              uint4 val = make_uint4(0u, 0u, 0u, 0u);
+              if (idx >= 0) {
+                if (!rg.fallback) {
+                  const int h = idx - rg.lo;
+                  val = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
+                } else {
+                  val = ldg_16(p.A + (size_t)idx * p.lda + cb * kBK + chunk * 8);
+                }
+              }
+              st_shared_v4(a_st + r * 128 + ((chunk ^ (r & 7)) << 4), val);
             }
+            warp_publish(&bar->afull[sa]);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (g >= ng) break;
-            const int k = kb + g;
-            const int cb = k / 9;
-            if (lane == 0) {
-              mbar_arrive(&bar->afull[(it + g) % SA]);
-              // the halo of channel block cb is done after its tap 8
-              if (!rg.fallback && k - cb * 9 == 8) mbar_arrive(&bar->hempty[(hi0 + cb) & 1]);
-            }
+          if (!rg.fallback && !aborted) {
+            warp_arrive(&bar->hempty[hb]);
+            ++hi;
           }
-          it += ng;
         }
-        if (!rg.fallback) hi = hi0 + kb_per_tap;
         if (!aborted) warp_arrive(&bar->iempty[slot]);
       }
     }
