@@ -128,6 +128,28 @@ SVCONV_API int svconv_bwd_weight(int dtype, const void* dY, const void* X, const
 SVCONV_API size_t svconv_bwd_weight_workspace_size(int dtype, int n, int Cin, int Cout);
 
 /*
+ * Allocation-free weight / bias gradient.  The paper has no counterpart: this is a
+ * convenience for callers that cannot allocate device memory at call time (a
+ * service with a fixed memory budget that must not call cudaMalloc after start-up,
+ * a plugin that cannot reach its host framework's allocator, a callback where an
+ * allocation would synchronise the device).  It computes exactly what
+ * svconv_bwd_weight computes, same arguments minus the workspace: the split
+ * partials live in a fixed device array of SVCONV_NOALLOC_SCRATCH_BYTES inside the
+ * library, which every GPU that loads the library holds until the process exits.
+ *   - The first call on a device looks up that array's address; make it before
+ *     any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race.  Serialise them.
+ *   - If the usual number of token splits does not fit, fewer are used (a different
+ *     summation order, same tolerance); if one split's partials
+ *     ((9*Cin+1 rounded up to 128) * Cout floats for bf16) exceed the array, it
+ *     returns SVCONV_ERR_SIZE.
+ *   - It calls no cudaMalloc / cudaFree and no allocating library routine.
+ */
+#define SVCONV_NOALLOC_SCRATCH_BYTES (16u << 20)
+SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin,
+                                         int Cout, float* dW, float* db, void* stream);
+
+/*
  * Chunked bottleneck adapter forward (Key Design 2, "chunked execution" that
  * keeps memory flat in the number of frames; the adapter is the "lightweight
  * bottleneck adapter" with "down-projected" features of the Overall Architecture

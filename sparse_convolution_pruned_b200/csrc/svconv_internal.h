@@ -83,6 +83,7 @@ struct TcWgradArgs {
 };
 void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn);
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s);
+cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s);
 
 // failure-detection self test
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s);

@@ -1044,6 +1044,36 @@ cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
   return launch_wgrad_inst<64>(prm, grid, s);
 }
 
+// Same kernel with a caller-chosen number of token splits (1 <= splits <= token
+// blocks); used by the allocation-free entry point, whose scratch is fixed.
+cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s) {
+  TcWgradParams prm;
+  memset(&prm, 0, sizeof(prm));
+  int plan_splits, rows_pad, bn;
+  tc_wgrad_plan(a.n, a.Cin, a.Cout, &plan_splits, &rows_pad, &bn);
+  const int kbt = (a.n + kBK - 1) / kBK;
+  if (a.splits < 1 || a.splits > kbt || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kHaloBox))
+    return cudaErrorInvalidValue;
+  if (!make_rows_tmap(&prm.tmap_dy, a.dY, (uint64_t)a.n, (uint64_t)a.Cout, 64u)) return cudaErrorInvalidValue;
+  prm.X = static_cast<const __nv_bfloat16*>(a.X);
+  prm.nbr = a.nbr;
+  prm.partial = a.partial;
+  prm.status = device_error_word();
+  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.n = a.n;
+  prm.Cin = a.Cin;
+  prm.Cout = a.Cout;
+  prm.splits = a.splits;
+  prm.rows_pad = rows_pad;
+  const int units = (rows_pad / kBM) * (a.Cout / bn) * a.splits;
+  int grid = sm_count();
+  if (grid > units) grid = units;
+  if (bn == 256) return launch_wgrad_inst<256>(prm, grid, s);
+  if (bn == 128) return launch_wgrad_inst<128>(prm, grid, s);
+  return launch_wgrad_inst<64>(prm, grid, s);
+}
+
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s) {
   timeout_selftest_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
   return cudaGetLastError();

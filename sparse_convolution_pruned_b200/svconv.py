@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.svconv_fwd.argtypes = [I, P, P, I, I, I, P, P, P, P]
         L.svconv_bwd_data.argtypes = [I, P, P, I, I, I, P, P, P]
         L.svconv_bwd_weight.argtypes = [I, P, P, P, I, I, I, P, P, P, Z, P]
+        L.svconv_bwd_weight_noalloc.argtypes = [I, P, P, P, I, I, I, P, P, P]
+        L.svconv_bwd_weight_noalloc.restype = I
         L.svconv_bwd_weight_workspace_size.argtypes = [I, I, I, I]
         L.svconv_bwd_weight_workspace_size.restype = Z
         L.svconv_adapter_fwd.argtypes = [P, P, P, I, I, I, I, P, P, P, P, I, I, P, Z, P, P]
@@ -188,6 +190,24 @@ def svconv_bwd_weight(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tensor, *, d
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _stream(X, stream))
     _check("svconv_bwd_weight", rc)
+    return dW, db
+
+
+def svconv_bwd_weight_noalloc(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tensor, *,
+                              dW: Optional[torch.Tensor] = None, db: Optional[torch.Tensor] = None,
+                              want_db: bool = True, stream=None):
+    """As svconv_bwd_weight, with the split partials in the library's fixed device array
+    (no workspace; concurrent calls race, see include/svconv.h)."""
+    _cuda(dY, X, nbr, dW, db)
+    n, Cout = dY.shape
+    Cin = X.shape[1]
+    if dW is None:
+        dW = torch.empty((Cout, 9, Cin), dtype=torch.float32, device=X.device)
+    if db is None and want_db:
+        db = torch.empty((Cout,), dtype=torch.float32, device=X.device)
+    rc = lib().svconv_bwd_weight_noalloc(_dtype_code(X), _ptr(dY), _ptr(X), _ptr(nbr), n, Cin, Cout, _ptr(dW),
+                                         _ptr(db), _stream(X, stream))
+    _check("svconv_bwd_weight_noalloc", rc)
     return dW, db
 
 
