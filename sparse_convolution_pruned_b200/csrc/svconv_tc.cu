@@ -240,25 +240,60 @@ struct MmaCfg {
   uint32_t b_lbo, b_sbo, b_step;
 };
 
+// Issuer state: descriptors of stage 0 and the per-stage / per-K=16 advances of their
+// start-address field (16-byte units), plus ring positions and phases.  The issuing
+// thread is on the critical path of the tensor pipe (an MMA of 128x256x16 takes
+// ~130 cycles), so its loop avoids divisions and rebuilding descriptors: stage
+// indices advance by increment and descriptors by 32-bit adds (the start-address
+// field is 14 bits of a 16-byte-granular shared address, so an add never carries
+// out of it).
+struct MmaIssuer {
+  uint64_t a_desc0, b_desc0;
+  uint32_t a_stage16, b_stage16, a_k16, b_k16;
+  uint32_t idesc;
+  int SA, SB;
+  int sa, sb;
+  uint32_t pa, pb;
+};
+
+__device__ __forceinline__ MmaIssuer make_issuer(const Carve& sm, uint32_t b_stage_bytes, int SA, int SB,
+                                                 const MmaCfg& c) {
+  MmaIssuer m;
+  m.a_desc0 = smem_desc_sw128(smem_u32(sm.a), c.a_lbo, c.a_sbo);
+  m.b_desc0 = smem_desc_sw128(smem_u32(sm.b), c.b_lbo, c.b_sbo);
+  m.a_stage16 = (uint32_t)kABytes >> 4;
+  m.b_stage16 = b_stage_bytes >> 4;
+  m.a_k16 = c.a_step >> 4;
+  m.b_k16 = c.b_step >> 4;
+  m.idesc = c.idesc;
+  m.SA = SA;
+  m.SB = SB;
+  m.sa = m.sb = 0;
+  m.pa = m.pb = 0;
+  return m;
+}
+
 // One thread issues the MMAs of one tile (num_kb K-blocks) into accumulator d.
-__device__ __forceinline__ bool mma_tile(TcBarriers* bar, const Carve& sm, uint32_t b_stage_bytes, int SA, int SB,
-                                         uint32_t& it, int num_kb, uint32_t d, const MmaCfg& c,
+__device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                          volatile int* abort_flag, int* err, uint64_t timeout_ns) {
-  for (int kb = 0; kb < num_kb; ++kb, ++it) {
-    const int sa = it % SA, sb = it % SB;
-    if (!mbar_wait(&bar->afull[sa], ring_parity(it, SA), abort_flag, err, timeout_ns)) return false;
-    if (!mbar_wait(&bar->bfull[sb], ring_parity(it, SB), abort_flag, err, timeout_ns)) return false;
-    tc_fence_after();
-    const uint32_t a0 = smem_u32(sm.a + (size_t)sa * kABytes);
-    const uint32_t b0 = smem_u32(sm.b + (size_t)sb * b_stage_bytes);
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!mbar_wait(&bar->afull[m.sa], m.pa, abort_flag, err, timeout_ns)) return false;
+    if (!mbar_wait(&bar->bfull[m.sb], m.pb, abort_flag, err, timeout_ns)) return false;
+    const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
+    const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sb * m.b_stage16);
 #pragma unroll
-    for (int k = 0; k < kBK / 16; ++k) {
-      const uint64_t ad = smem_desc_sw128(a0 + k * c.a_step, c.a_lbo, c.a_sbo);
-      const uint64_t bd = smem_desc_sw128(b0 + k * c.b_step, c.b_lbo, c.b_sbo);
-      tc_mma_bf16(d, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
+    for (int k = 0; k < kBK / 16; ++k)
+      tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
+    tc_commit(&bar->aempty[m.sa]);
+    tc_commit(&bar->bempty[m.sb]);
+    if (++m.sa == m.SA) {
+      m.sa = 0;
+      m.pa ^= 1u;
     }
-    tc_commit(&bar->aempty[sa]);
-    tc_commit(&bar->bempty[sb]);
+    if (++m.sb == m.SB) {
+      m.sb = 0;
+      m.pb ^= 1u;
+    }
   }
   return true;
 }
@@ -502,15 +537,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       } else {
         c.b_lbo = 16, c.b_sbo = 1024, c.b_step = 32;
       }
-      uint32_t it = 0, tc = 0;
+      MmaIssuer mi = make_issuer(sm, kBBytes, SA, SB, c);
+      uint32_t tc = 0;
       bool issued = false;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
         const uint32_t ab = tc & 1u;
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, sm, kBBytes, SA, SB, it, num_kb, tmem_base + ab * BN, c, abort_flag, err, p.timeout_ns))
-          break;
+        if (!mma_tile(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
@@ -795,7 +830,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       c.idesc = idesc_bf16_f32(kBM, BN, 1, 1);
       c.a_lbo = 8192, c.a_sbo = 1024, c.a_step = 2048;  // both MN-major: 64-wide groups 8 KB apart
       c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;
-      uint32_t it = 0, tc = 0;
+      MmaIssuer mi = make_issuer(sm, kBBytes, SA, SB, c);
+      uint32_t tc = 0;
       bool issued = false;
       for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
         int sp, m0, n0, kb0, kb1;
@@ -804,9 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, sm, kBBytes, SA, SB, it, kb1 - kb0, tmem_base + ab * BN, c, abort_flag, err,
-                      p.timeout_ns))
-          break;
+        if (!mma_tile(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
