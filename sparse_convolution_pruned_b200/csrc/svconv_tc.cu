@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, SA, SB, gather ? kProdWarps : 1, 1);
+    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 1);  // one builder group per A stage
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -471,10 +471,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders
+    // Two groups of four warps build alternate K-blocks (group g takes the K-blocks
+    // with counter parity g, i.e. A stages g and g+2), so one group's proxy fence,
+    // which waits for its shared-memory stores to drain, overlaps the other
+    // group's copying.  Each thread copies 8 rows' 16-byte chunks, all loads first.
     if (gather) {
       const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
-      const int chunk = pt & 7;                     // 16-byte chunk of a 128-byte row
-      const int rsub = pt >> 3;                     // rows rsub + 32 q, q = 0..3
+      const int grp = pt >> 7;                      // builder group 0 or 1
+      const int gt = pt & 127;
+      const int chunk = gt & 7;                     // 16-byte chunk of a 128-byte row
+      const int rsub = gt >> 3;                     // rows rsub + 16 q, q = 0..7
       uint32_t ti = 0, hi = 0, it = 0;
       bool aborted = false;
       for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
@@ -494,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
           }
           const uint32_t halo = smem_u32(sm.halo + hb * kHaloBufBytes);
           for (int j = 0; j < 9; ++j, ++it) {
+            if ((int)(it & 1u) != grp) continue;
             const int jj = MIRROR ? 8 - j : j;
             const int sa = it % SA;
             if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
@@ -501,20 +508,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               break;
             }
             const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
+            int idx[8];
+            uint4 val[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int r = rsub + 32 * q;
-              const int idx = sidx[r * 9 + jj];
-              uint4 val = make_uint4(0u, 0u, 0u, 0u);
-              if (idx >= 0) {
+            for (int q = 0; q < 8; ++q) idx[q] = sidx[(rsub + 16 * q) * 9 + jj];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              val[q] = make_uint4(0u, 0u, 0u, 0u);
+              if (idx[q] >= 0) {
                 if (!rg.fallback) {
-                  const int h = idx - rg.lo;
-                  val = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
+                  const int h = idx[q] - rg.lo;
+                  val[q] = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
                 } else {
-                  val = ldg_16(p.A + (size_t)idx * p.lda + cb * kBK + chunk * 8);
+                  val[q] = ldg_16(p.A + (size_t)idx[q] * p.lda + cb * kBK + chunk * 8);
                 }
               }
-              st_shared_v4(a_st + r * 128 + ((chunk ^ (r & 7)) << 4), val);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int r = rsub + 16 * q;
+              st_shared_v4(a_st + r * 128 + ((chunk ^ (r & 7)) << 4), val[q]);
             }
             warp_publish(&bar->afull[sa]);
           }
@@ -950,6 +963,7 @@ static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint
 static void pick_stages(bool wgrad, int bn, int* sa, int* sb) {
   const size_t budget = 220 * 1024;
   for (int a = 4; a >= 2; --a) {
+    if (!wgrad && (a & 1)) continue;  // conv: two builder groups alternate A stages
     int b_best = 0;
     for (int b = 2; b <= kMaxStages; ++b) {
       const Geometry g = wgrad ? wgrad_geometry(bn, a, b) : conv_geometry(bn, a, b);
