@@ -65,6 +65,8 @@ constexpr int kConvHaloRows = 192;                 // conv halo capacity (>= 128
 constexpr int kWgHaloRows = 128;                   // weight-gradient halo capacity (64-token blocks)
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
+constexpr int kTmemAStages = 4;                    // gather conv: A stages held in tensor memory
+constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
 struct __align__(8) TcBarriers {
   uint64_t afull[kMaxStages], aempty[kMaxStages];  // A stages
@@ -132,9 +134,20 @@ struct Geometry {
 
 __host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb) {
-  return {(size_t)sa * kABytes, (size_t)sb * bn * kBK * 2, (size_t)2 * kConvHaloRows * 128,
-          round_up((size_t)2 * kConvIdx * 4, 16)};
+// a_in_tmem: the gathered A stages live in tensor memory, so no shared A ring.
+__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem) {
+  return {a_in_tmem ? (size_t)0 : (size_t)sa * kABytes, (size_t)sb * bn * kBK * 2,
+          (size_t)2 * kConvHaloRows * 128, round_up((size_t)2 * kConvIdx * 4, 16)};
+}
+
+// Tensor-memory plan of the conv kernel: accumulator buffers first, then the A stages.
+__host__ __device__ constexpr int conv_acc_buffers(int bn, bool a_in_tmem) { return (a_in_tmem && bn == 256) ? 1 : 2; }
+__host__ __device__ constexpr uint32_t pow2_cols(uint32_t c) {
+  return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
+}
+__host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem) {
+  return pow2_cols((uint32_t)(conv_acc_buffers(bn, a_in_tmem) * bn) +
+                   (a_in_tmem ? (uint32_t)(kTmemAStages * kTmemAStageCols) : 0u));
 }
 
 __host__ __device__ inline Geometry wgrad_geometry(int bn, int sa, int sb) {
@@ -248,6 +261,7 @@ struct MmaCfg {
 // field is 14 bits of a 16-byte-granular shared address, so an add never carries
 // out of it).
 struct MmaIssuer {
+  uint32_t a_tmem0;  // A in tensor memory: column address of A stage 0
   uint64_t a_desc0, b_desc0;
   uint32_t a_stage16, b_stage16, a_k16, b_k16;
   uint32_t idesc;
@@ -259,6 +273,7 @@ struct MmaIssuer {
 __device__ __forceinline__ MmaIssuer make_issuer(const Carve& sm, uint32_t b_stage_bytes, int SA, int SB,
                                                  const MmaCfg& c) {
   MmaIssuer m;
+  m.a_tmem0 = 0;
   m.a_desc0 = smem_desc_sw128(smem_u32(sm.a), c.a_lbo, c.a_sbo);
   m.b_desc0 = smem_desc_sw128(smem_u32(sm.b), c.b_lbo, c.b_sbo);
   m.a_stage16 = (uint32_t)kABytes >> 4;
@@ -274,16 +289,26 @@ __device__ __forceinline__ MmaIssuer make_issuer(const Carve& sm, uint32_t b_sta
 }
 
 // One thread issues the MMAs of one tile (num_kb K-blocks) into accumulator d.
+// A_TMEM: A stages in tensor memory (written by the builder warps with tcgen05.st).
+template <bool A_TMEM>
 __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                          volatile int* abort_flag, int* err, uint64_t timeout_ns) {
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!mbar_wait(&bar->afull[m.sa], m.pa, abort_flag, err, timeout_ns)) return false;
     if (!mbar_wait(&bar->bfull[m.sb], m.pb, abort_flag, err, timeout_ns)) return false;
-    const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
     const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sb * m.b_stage16);
+    if constexpr (A_TMEM) {
+      tc_fence_after();  // the A stage was written to tensor memory by other threads
+      const uint32_t at = m.a_tmem0 + (uint32_t)m.sa * kTmemAStageCols;
 #pragma unroll
-    for (int k = 0; k < kBK / 16; ++k)
-      tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
+      for (int k = 0; k < kBK / 16; ++k)
+        tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
+    } else {
+      const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k)
+        tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
+    }
     tc_commit(&bar->aempty[m.sa]);
     tc_commit(&bar->bempty[m.sb]);
     if (++m.sa == m.SA) {
@@ -312,14 +337,17 @@ __device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err
 template <int BN, bool MIRROR>
 __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
   extern __shared__ uint8_t smem_raw[];
+  const bool gather = p.nbr != nullptr;  // gathered A lives in tensor memory
   const int SA = p.stages_a, SB = p.stages_b;
-  const Geometry geo = conv_geometry(BN, SA, SB);
+  const Geometry geo = conv_geometry(BN, SA, SB, gather);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
   constexpr uint32_t kBBytes = BN * kBK * 2;
-  constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  const uint32_t tmem_cols = conv_tmem_cols(BN, gather);
+  const int n_acc = conv_acc_buffers(BN, gather);
+  const uint32_t a_tmem_col = (uint32_t)(n_acc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kConvHaloRows * 128;
 
   // rows handled by this launch (device-side bounds for the chunked adapter)
@@ -339,7 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int kb_per_tap = p.Kc / kBK;
   const int taps = p.taps;
   const int num_kb = taps * kb_per_tap;
-  const bool gather = p.nbr != nullptr;
   const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
@@ -348,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     prefetch_tmap(&p.tmap_b);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&bar->tmem_base, kTmemCols);
+    tmem_alloc(&bar->tmem_base, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -472,15 +499,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders
     // Two groups of four warps build alternate K-blocks (group g takes the K-blocks
-    // with counter parity g, i.e. A stages g and g+2), so one group's proxy fence,
-    // which waits for its shared-memory stores to drain, overlaps the other
-    // group's copying.  Each thread copies 8 rows' 16-byte chunks, all loads first.
+    // with counter parity g, i.e. A stages g and g+2).  Each thread owns one tile row:
+    // warp w may only touch TMEM lanes 32*(w%4) .. +31, so thread (w, lane) copies
+    // row 32*(w%4) + lane.  It reads the row's neighbour segment from the halo in
+    // shared memory (or global memory on the fallback path) and writes it straight
+    // into the tensor-memory A stage with tcgen05.st: no shared-memory stores, no
+    // proxy fence, and the MMA reads only B from shared memory.
     if (gather) {
-      const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
-      const int grp = pt >> 7;                      // builder group 0 or 1
-      const int gt = pt & 127;
-      const int chunk = gt & 7;                     // 16-byte chunk of a 128-byte row
-      const int rsub = gt >> 3;                     // rows rsub + 16 q, q = 0..7
+      const int grp = (warp - kEpiWarps) >> 2;  // builder group 0 or 1
+      const int quarter = warp & 3;             // TMEM lane quarter of this warp
+      const int r = quarter * 32 + lane;        // the tile row this thread writes
+      const uint32_t a_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + a_tmem_col;
       uint32_t ti = 0, hi = 0, it = 0;
       bool aborted = false;
       for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
@@ -507,29 +536,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               aborted = true;
               break;
             }
-            const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
-            int idx[8];
-            uint4 val[8];
+            tc_fence_after();  // the MMAs that read this stage are complete
+            const int idx = sidx[r * 9 + jj];
+            uint32_t v[32];
+            if (idx >= 0 && !rg.fallback) {
+              const int h = idx - rg.lo;
+              const uint32_t row = halo + h * 128;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) idx[q] = sidx[(rsub + 16 * q) * 9 + jj];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              val[q] = make_uint4(0u, 0u, 0u, 0u);
-              if (idx[q] >= 0) {
-                if (!rg.fallback) {
-                  const int h = idx[q] - rg.lo;
-                  val[q] = ld_shared_16(halo + h * 128 + ((chunk ^ (h & 7)) << 4));
-                } else {
-                  val[q] = ldg_16(p.A + (size_t)idx[q] * p.lda + cb * kBK + chunk * 8);
-                }
+              for (int c = 0; c < 8; ++c) {
+                const uint4 q = ld_shared_16(row + ((c ^ (h & 7)) << 4));
+                v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
               }
-            }
+            } else if (idx >= 0) {
+              const __nv_bfloat16* src = p.A + (size_t)idx * p.lda + cb * kBK;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int r = rsub + 16 * q;
-              st_shared_v4(a_st + r * 128 + ((chunk ^ (r & 7)) << 4), val[q]);
+              for (int c = 0; c < 8; ++c) {
+                const uint4 q = ldg_16(src + c * 8);
+                v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) v[c] = 0u;
             }
-            warp_publish(&bar->afull[sa]);
+            tmem_st_32x32b_x32(a_lane + (uint32_t)sa * kTmemAStageCols, v);
+            tmem_st_wait();
+            tc_fence_before();
+            warp_arrive(&bar->afull[sa]);
           }
           if (!rg.fallback && !aborted) {
             warp_arrive(&bar->hempty[hb]);
@@ -544,21 +576,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     if (lane == 0) {
       MmaCfg c;
       c.idesc = idesc_bf16_f32(kBM, BN, 0, MIRROR ? 1 : 0);
-      c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // A: K-major, 128-byte rows
+      c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // smem A (dense): K-major, 128-byte rows
       if (MIRROR) {
         c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // B: MN-major, 64-wide MN groups 8 KB apart
       } else {
         c.b_lbo = 16, c.b_sbo = 1024, c.b_step = 32;
       }
       MmaIssuer mi = make_issuer(sm, kBBytes, SA, SB, c);
+      mi.a_tmem0 = tmem_base + a_tmem_col;
       uint32_t tc = 0;
       bool issued = false;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
-        const uint32_t ab = tc & 1u;
-        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        const uint32_t ab = tc % (uint32_t)n_acc;
+        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, n_acc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
+        const bool ok = gather ? mma_tile<true>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)
+                               : mma_tile<false>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        if (!ok) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
@@ -569,8 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     uint32_t tc = 0;
     const int out_base = p.out_abs ? lo : 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
-      const uint32_t ab = tc & 1u;
-      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, 2), abort_flag, err, p.timeout_ns)) break;
+      const uint32_t ab = tc % (uint32_t)n_acc;
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, n_acc), abort_flag, err, p.timeout_ns)) break;
       tc_fence_after();
       const int m0 = (tile / n_tiles) * kBM;
       const int n0 = (tile % n_tiles) * BN;
@@ -629,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, tmem_cols);
   }
 }
 
@@ -853,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
+        if (!mma_tile<false>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
@@ -966,7 +1001,7 @@ static void pick_stages(bool wgrad, int bn, int* sa, int* sb) {
     if (!wgrad && (a & 1)) continue;  // conv: two builder groups alternate A stages
     int b_best = 0;
     for (int b = 2; b <= kMaxStages; ++b) {
-      const Geometry g = wgrad ? wgrad_geometry(bn, a, b) : conv_geometry(bn, a, b);
+      const Geometry g = wgrad ? wgrad_geometry(bn, a, b) : conv_geometry(bn, a, b, false);
       if (smem_total(g) <= budget) b_best = b;
     }
     if (b_best >= 3 || (a == 2 && b_best >= 2)) {
@@ -981,8 +1016,17 @@ static void pick_stages(bool wgrad, int bn, int* sa, int* sb) {
 
 template <int BN, bool MIRROR>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
-  pick_stages(false, BN, &prm.stages_a, &prm.stages_b);
-  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b));
+  const bool a_in_tmem = prm.nbr != nullptr;
+  if (a_in_tmem) {
+    // A stages in tensor memory: the whole shared-memory budget goes to B stages
+    prm.stages_a = kTmemAStages;
+    prm.stages_b = 2;
+    for (int b = 2; b <= kMaxStages; ++b)
+      if (smem_total(conv_geometry(BN, 0, b, true)) <= 220 * 1024) prm.stages_b = b;
+  } else {
+    pick_stages(false, BN, &prm.stages_a, &prm.stages_b);
+  }
+  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b, a_in_tmem));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
