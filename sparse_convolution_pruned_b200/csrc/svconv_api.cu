@@ -216,7 +216,7 @@ int svconv_bwd_weight(int dtype, const void* dY, const void* X, const int32_t* n
     cudaError_t e = launch_f32_wgrad_partials(static_cast<const float*>(dY), static_cast<const float*>(X), nbr, n,
                                               Cin, Cout, partial, splits, rows, s);
     if (e != cudaSuccess) return SVCONV_ERR_CUDA;
-    return cuda_rc(launch_wgrad_reduce(partial, splits, rows, Cin, Cout, dW, db, s));
+    return cuda_rc(launch_wgrad_reduce(partial, splits, rows, Cin, Cout, 0, dW, db, s));
   }
   if (!aligned16(dY) || !aligned16(X)) return SVCONV_ERR_ALIGN;
   TcWgradArgs a{};
@@ -231,7 +231,7 @@ int svconv_bwd_weight(int dtype, const void* dY, const void* X, const int32_t* n
   tc_wgrad_plan(n, Cin, Cout, &a.splits, &a.rows_pad, &bn);
   cudaError_t e = launch_tc_wgrad(a, s);
   if (e != cudaSuccess) return SVCONV_ERR_CUDA;
-  return cuda_rc(launch_wgrad_reduce(partial, a.splits, a.rows_pad, Cin, Cout, dW, db, s));
+  return cuda_rc(launch_wgrad_reduce(partial, a.splits, a.rows_pad, Cin, Cout, 1, dW, db, s));
 }
 
 size_t svconv_adapter_workspace_size(int R, int max_chunk_rows) {

@@ -113,12 +113,14 @@ __global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __r
   }
 }
 
-// One thread per (dW row m, output channel o); 32 x 32 tiles so that both the
-// partial reads (along o) and the transposed dW writes (along m) are coalesced.
-// The split sums are issued 8 loads at a time so they overlap.
+// One thread per (dW row m = j * Cin + i, output channel o); 32 x 32 tiles so that
+// both the partial reads (along o) and the transposed dW writes (along m) are
+// coalesced.  The split sums are issued 8 loads at a time so they overlap.
+// grouped = 0: partial row m (db at 9 Cin); grouped = 1 (tensor-core layout, Cin a
+// multiple of 64): partial row ((i / 64) * 10 + j) * 64 + i % 64, db at 9 * 64.
 __global__ void __launch_bounds__(1024) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
-                                                            int rows_pad, int Cin, int Cout, float* __restrict__ dW,
-                                                            float* __restrict__ db) {
+                                                            int rows_pad, int Cin, int Cout, int grouped,
+                                                            float* __restrict__ dW, float* __restrict__ db) {
   __shared__ float tile[32][33];
   const int rows = 9 * Cin + 1;
   const int m0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
@@ -127,8 +129,13 @@ __global__ void __launch_bounds__(1024) wgrad_reduce_kernel(const float* __restr
     const int m = m0 + ty, o = o0 + tx;
     Dot2 s;
     if (m < rows && o < Cout) {
+      int pm = m;
+      if (grouped) {
+        const int j = m / Cin, i = m - j * Cin;
+        pm = m == 9 * Cin ? 9 * 64 : ((i >> 6) * 10 + j) * 64 + (i & 63);
+      }
       const size_t stride = (size_t)rows_pad * Cout;
-      const float* src = partial + (size_t)m * Cout + o;
+      const float* src = partial + (size_t)pm * Cout + o;
       for (int sp0 = 0; sp0 < splits; sp0 += 8) {
         float v[8];
 #pragma unroll
@@ -187,11 +194,11 @@ cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int
   return cudaGetLastError();
 }
 
-cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, float* dW,
-                                float* db, cudaStream_t s) {
+cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, int grouped,
+                                float* dW, float* db, cudaStream_t s) {
   const int rows = 9 * Cin + 1;
   dim3 grid((rows + 31) / 32, (Cout + 31) / 32);
-  wgrad_reduce_kernel<<<grid, dim3(32, 32), 0, s>>>(partial, splits, rows_pad, Cin, Cout, dW, db);
+  wgrad_reduce_kernel<<<grid, dim3(32, 32), 0, s>>>(partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
   return cudaGetLastError();
 }
 

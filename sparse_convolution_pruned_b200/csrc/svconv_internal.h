@@ -38,9 +38,10 @@ cudaError_t launch_f32_conv(bool mirror_bwd, const float* src, const int32_t* nb
 size_t f32_wgrad_splits(int n);
 cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int32_t* nbr, int n, int Cin, int Cout,
                                       float* partial, int splits, int rows_pad, cudaStream_t s);
-// partial [splits][rows_pad][Cout] with row m = j*Cin + i (m = 9*Cin holds db)
-cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, float* dW,
-                                float* db, cudaStream_t s);
+// partial [splits][rows_pad][Cout]; grouped = 0: row m = j*Cin + i (m = 9*Cin holds db);
+// grouped = 1 (tensor-core layout): row ((i/64)*10 + j)*64 + i%64, db in row 576
+cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, int grouped,
+                                float* dW, float* db, cudaStream_t s);
 
 // ---------------------------------------------------------------- tcgen05 bf16 path
 struct TcConvArgs {
@@ -78,7 +79,7 @@ struct TcWgradArgs {
   const void* X;      // bf16 [n][Cin]
   const int32_t* nbr; // [n][9]
   int n, Cin, Cout;
-  float* partial;     // [splits][rows_pad][Cout]
+  float* partial;     // [splits][rows_pad][Cout], grouped row layout (see launch_wgrad_reduce)
   int splits, rows_pad;
 };
 void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn);

@@ -112,6 +112,6 @@ extern "C" int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
     e = launch_tc_wgrad_with_splits(a, s);
   }
   if (e != cudaSuccess) return SVCONV_ERR_CUDA;
-  e = launch_wgrad_reduce(partial, splits, rows_pad, Cin, Cout, dW, db, s);
+  e = launch_wgrad_reduce(partial, splits, rows_pad, Cin, Cout, dtype == SVCONV_BF16 ? 1 : 0, dW, db, s);
   return e == cudaSuccess ? SVCONV_OK : SVCONV_ERR_CUDA;
 }

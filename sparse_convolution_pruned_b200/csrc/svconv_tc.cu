@@ -62,16 +62,20 @@ constexpr int kThreads = (kMmaWarp + 1) * 32;      // 480
 constexpr int kMaxStages = 8;
 constexpr int kHaloBox = 64;                       // rows per halo TMA box
 constexpr int kConvHaloRows = 192;                 // conv halo capacity (>= 128 + 2 * (W + 1) for W <= 31)
-constexpr int kWgHaloRows = 128;                   // weight-gradient halo capacity (64-token blocks)
+constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
+constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
+constexpr int kWgSlots = 4;                        // weight gradient: index + halo slots in flight
+constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
 constexpr int kTmemAStages = 4;                    // gather conv: A stages held in tensor memory
 constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
-struct __align__(8) TcBarriers {
+struct __align__(16) TcBarriers {
+  uint32_t zero16[4];                              // 16 zero bytes (row source for missing neighbours)
   uint64_t afull[kMaxStages], aempty[kMaxStages];  // A stages
   uint64_t bfull[kMaxStages], bempty[kMaxStages];  // B stages
-  uint64_t ifull[2], iempty[2];                    // neighbour-row slots (and their halos, weight gradient)
+  uint64_t ifull[kMaxStages], iempty[kMaxStages];  // neighbour-row slots (and their halos, weight gradient)
   uint64_t hfull[2], hempty[2];                    // conv halo buffers
   uint64_t tfull[2], tempty[2];                    // TMEM accumulators
   uint64_t done;                                   // final MMA drain before TMEM is released
@@ -150,9 +154,14 @@ __host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem) {
                    (a_in_tmem ? (uint32_t)(kTmemAStages * kTmemAStageCols) : 0u));
 }
 
-__host__ __device__ inline Geometry wgrad_geometry(int bn, int sa, int sb) {
-  return {(size_t)sa * kABytes, (size_t)sb * bn * kBK * 2, (size_t)4 * kWgHaloRows * 128,
-          round_up((size_t)2 * kWgIdx * 4, 16)};
+// Weight gradient: A lives in tensor memory; kWgSlots slots of (index entries, halo).
+__host__ __device__ inline Geometry wgrad_geometry(int bn, int sb) {
+  return {(size_t)0, (size_t)sb * bn * kBK * 2, (size_t)kWgSlots * kWgHaloRows * 128,
+          round_up((size_t)kWgSlots * kWgIdx * 4, 16)};
+}
+__host__ __device__ constexpr int wgrad_acc_buffers(int bn) { return bn == 256 ? 1 : 2; }
+__host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
+  return pow2_cols((uint32_t)(wgrad_acc_buffers(bn) * bn + kTmemAStages * kTmemAStageCols));
 }
 
 __host__ __device__ inline size_t smem_total(const Geometry& g) {
@@ -172,8 +181,14 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
   return c;
 }
 
-__device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uint32_t afull_count,
-                                              uint32_t ifull_count) {
+// nslots neighbour-row slots with the given arrival counts; everything else fixed.
+__device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uint32_t afull_count, int nslots,
+                                              uint32_t ifull_count, uint32_t iempty_count) {
+  for (int i = 0; i < 4; ++i) b->zero16[i] = 0u;
+  for (int i = 0; i < nslots; ++i) {
+    mbar_init(&b->ifull[i], ifull_count);
+    mbar_init(&b->iempty[i], iempty_count);
+  }
   for (int s = 0; s < sa; ++s) {
     mbar_init(&b->afull[s], afull_count);
     mbar_init(&b->aempty[s], 1);
@@ -183,8 +198,6 @@ __device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uin
     mbar_init(&b->bempty[s], 1);
   }
   for (int i = 0; i < 2; ++i) {
-    mbar_init(&b->ifull[i], ifull_count);
-    mbar_init(&b->iempty[i], kProdWarps);
     mbar_init(&b->hfull[i], 1);
     mbar_init(&b->hempty[i], kProdWarps);
     mbar_init(&b->tfull[i], 1);
@@ -370,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 1);  // one builder group per A stage
+    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 1, kProdWarps);  // one builder group per A stage
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -669,27 +682,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
 }
 
 // ============================================================================ weight gradient
+// dW^T[(j,i)][o] = sum_k X[N[k,j]][i] dY[k][o] (SV-TAD page, Key Design 2: the
+// weight gradient is the transposed contraction over kept tokens), db[o] = sum_k dY[k][o].
+//
+// M (accumulator rows) runs over (64-channel block cb, tap j, channel c): each
+// block cb owns 10 half-tiles of 64 rows, taps 0..8 then one extra half that holds
+// the all-ones row for db (block 0) or padding (other blocks), so a 128-row tile
+// covers two taps of ONE channel block and needs a single halo.  Partial row of
+// (j, i): ((i / 64) * 10 + j) * 64 + i % 64; db is row 9 * 64.
+//
+// K runs over tokens in blocks of 64.  The halo of a block is the fixed window
+// of X rows k0 - 32 .. k0 + 95 (a neighbour is at most W + 1 packed rows away), so
+// its TMA is issued together with the block's index entries, without waiting for
+// them; an entry outside the window (W > 31, or tokens out of raster order) is
+// read from global memory instead.  A lives in tensor memory: the builders read
+// 8 x 8 (token x channel) pieces of the halo with ldmatrix.trans, which yields
+// exactly the (channel lane, token-pair column) order of tcgen05.st.16x128b, so A
+// is transposed and gathered on the way in, with no shared-memory stores.  B is
+// dY by TMA (MN-major).
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_constant__ TcWgradParams p) {
   extern __shared__ uint8_t smem_raw[];
-  const int SA = p.stages_a, SB = p.stages_b;
-  const Geometry geo = wgrad_geometry(BN, SA, SB);
+  const int SB = p.stages_b;
+  const Geometry geo = wgrad_geometry(BN, SB);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
   constexpr uint32_t kBBytes = BN * kBK * 2;
-  constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  constexpr int kAcc = wgrad_acc_buffers(BN);
+  constexpr uint32_t kTmemCols = wgrad_tmem_cols(BN);
+  constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
 
   const int m_tiles = p.rows_pad / kBM;
   const int n_tiles = p.Cout / BN;
   const int num_units = m_tiles * n_tiles * p.splits;
   const int kbt = (p.n + kBK - 1) / kBK;  // token blocks in total
-  const int wrows = 9 * p.Cin;             // real dW rows; row wrows is db
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, SA, SB, kProdWarps, 1);
+    // ifull: 32 cp.async arrivals of the loader lanes + its expect_tx arrival
+    init_barriers(bar, kTmemAStages, SB, kProdWarps / 2, kWgSlots, 33, kProdWarps / 2);
     prefetch_tmap(&p.tmap_x);
     prefetch_tmap(&p.tmap_dy);
   }
@@ -705,101 +738,60 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 
   // unit -> (split, m-tile, n-tile); units of one split run side by side so the
   // tiles of dY and the X rows they share are hot in L2.
-  auto decode = [&](int u, int& sp, int& m0, int& n0, int& kb0, int& kb1) {
+  auto decode = [&](int u, int& sp, int& mt, int& n0, int& kb0, int& kb1) {
     const int nt = u % n_tiles;
     const int rest = u / n_tiles;
-    const int mt = rest % m_tiles;
+    mt = rest % m_tiles;
     sp = rest / m_tiles;
-    m0 = mt * kBM;
     n0 = nt * BN;
     kb0 = (int)((long long)kbt * sp / p.splits);
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
   };
-  // the two 64-row halves of an m-tile: kind 0 = a (tap, 64-channel block) of X,
-  // kind 1 = the all-ones row (db), kind 2 = padding (never loaded: its
-  // accumulator rows are not read)
-  auto half_info = [&](int m0, int h, int& kind, int& tap, int& cblk) {
-    const int mh = m0 + 64 * h;
-    kind = mh < wrows ? 0 : (mh == wrows ? 1 : 2);
-    tap = kind == 0 ? mh / p.Cin : 0;
-    cblk = kind == 0 ? (mh - tap * p.Cin) / kBK : 0;
-  };
 
   if (warp == kHaloWarp) {
-    // per 64-token block: neighbour entries, their range, and one halo per
-    // distinct channel block of the tile's gathered halves, all on ifull[slot]
+    // ------------------------------------------------------------ index entries + halo window, per token block
     uint32_t q = 0;
     bool aborted = false;
     for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      int sp, m0, n0, kb0, kb1;
-      decode(u, sp, m0, n0, kb0, kb1);
-      int kind0, tap0, cb0, kind1, tap1, cb1;
-      half_info(m0, 0, kind0, tap0, cb0);
-      half_info(m0, 1, kind1, tap1, cb1);
-      const bool second_halo = kind1 == 0 && !(kind0 == 0 && cb1 == cb0);
+      int sp, mt, n0, kb0, kb1;
+      decode(u, sp, mt, n0, kb0, kb1);
+      const int cb = mt / kWgTiles;
       for (int kb = kb0; kb < kb1; ++kb, ++q) {
-        const int slot = q & 1;
-        if (!warp_wait(&bar->iempty[slot], ring_parity(q, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
+        const int slot = (int)(q % kWgSlots);
+        if (!warp_wait(&bar->iempty[slot], ring_parity(q, kWgSlots) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
         const int k0 = kb * kBK;
         const int lim = min(p.n - k0, kBK) * 9;
         const int32_t* src = p.nbr + (size_t)k0 * 9;
-        int v[kWgIdx / 32];
+        const uint32_t dst = smem_u32(sm.idx + slot * kWgIdx);
 #pragma unroll
         for (int i = 0; i < kWgIdx / 32; ++i) {
           const int e = lane + 32 * i;
-          v[i] = e < lim ? __ldg(src + e) : -1;
+          cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
         }
-        int vmin = INT_MAX, vmax = -1;
-        int32_t* sidx = sm.idx + slot * kWgIdx;
-#pragma unroll
-        for (int i = 0; i < kWgIdx / 32; ++i) {
-          int x = v[i];
-          if (x >= p.n) {
-            atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-            x = -1;
-          }
-          if (x >= 0) {
-            vmin = min(vmin, x);
-            vmax = max(vmax, x);
-          }
-          sidx[lane + 32 * i] = x < 0 ? -1 : x;
-        }
-        vmin = warp_min(vmin);
-        vmax = warp_max(vmax);
-        const int rows = vmax >= 0 ? vmax - vmin + 1 : 0;
-        const bool fallback = rows == 0 || rows > kWgHaloRows;
-        const int nbox = fallback ? 0 : (rows + kHaloBox - 1) / kHaloBox;
-        const int nhalo = fallback ? 0 : (kind0 == 0 ? 1 : 0) + (second_halo ? 1 : 0);
-        if (lane == 0) sm.rng[slot] = HaloRange{vmin, rows, fallback ? 1 : 0, 0};
-        __syncwarp();
+        cp_async_arrive_noinc(&bar->ifull[slot]);
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bar->ifull[slot], (uint32_t)(nbox * nhalo) * kHaloBox * 128);
-          const uint32_t dst = smem_u32(sm.halo + (size_t)slot * 2 * kHaloBufBytes);
-          for (int hh = 0; hh < 2; ++hh) {
-            if (nbox == 0) break;
-            if (hh == 0 && kind0 != 0) continue;
-            if (hh == 1 && !second_halo) continue;
-            const int cb = hh == 0 ? cb0 : cb1;
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(dst + hh * kHaloBufBytes + b * kHaloBox * 128, &p.tmap_x, &bar->ifull[slot], cb * kBK,
-                          vmin + b * kHaloBox);
-          }
+          mbar_arrive_expect_tx(&bar->ifull[slot], kHaloBufBytes);
+          const uint32_t hb = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
+#pragma unroll
+          for (int b = 0; b < kWgHaloRows / kHaloBox; ++b)
+            tma_load_2d(hb + b * kHaloBox * 128, &p.tmap_x, &bar->ifull[slot], cb * kBK, k0 - kWgPad + b * kHaloBox);
         }
         __syncwarp();
       }
     }
-    if (aborted) drain_ring(bar->ifull, q, 2, err, p.timeout_ns);
+    if (aborted) drain_ring(bar->ifull, q, kWgSlots, err, p.timeout_ns);
   } else if (warp == kBWarp) {
+    // ------------------------------------------------------------ dY tiles
     uint32_t it = 0;
     bool aborted = false;
     for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      int sp, m0, n0, kb0, kb1;
-      decode(u, sp, m0, n0, kb0, kb1);
+      int sp, mt, n0, kb0, kb1;
+      decode(u, sp, mt, n0, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        const int sb = it % SB;
+        const int sb = (int)(it % (uint32_t)SB);
         if (!warp_wait(&bar->bempty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
@@ -816,94 +808,146 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     }
     if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
-    const int pt = threadIdx.x - kEpiWarps * 32;  // 0..255
-    const int chunk = pt & 7;
-    const int ksub = pt >> 3;  // token rows ksub and ksub + 32 of each half
-    uint32_t q = 0, it = 0;
+    // ------------------------------------------------------------ A builders (tensor memory)
+    // Two groups of four warps take alternate token blocks.  Warp w writes TMEM lanes
+    // 32 (w % 4) .. + 31: half (w % 4) / 2 of the tile, channels 32 (w % 2) .. + 31 of
+    // that half's tap, as two 16-lane pieces of 16 channels x 64 tokens.  For one
+    // piece, ldmatrix k4 (k4 = 0..3) covers tokens 16 k4 .. + 15: lane i supplies the
+    // halo row of token 16 k4 + 8 (i / 16) + i % 8, channels +8 ((i / 8) % 2); its four
+    // registers are then registers 4 k4 .. 4 k4 + 3 of the 16x128b.x8 store.
+    const int grp = (warp - kEpiWarps) >> 2;
+    const int quarter = warp & 3;
+    const int half = quarter >> 1;
+    const int cq = (quarter & 1) * 32;
+    const uint32_t zero_addr = smem_u32(bar->zero16);
+    const uint16_t* X16 = reinterpret_cast<const uint16_t*>(p.X);
+    uint32_t q = 0;
     bool aborted = false;
     for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      int sp, m0, n0, kb0, kb1;
-      decode(u, sp, m0, n0, kb0, kb1);
-      int kind[2], tap[2], cblk[2];
-      half_info(m0, 0, kind[0], tap[0], cblk[0]);
-      half_info(m0, 1, kind[1], tap[1], cblk[1]);
-      const int hsel1 = (kind[0] == 0 && cblk[1] == cblk[0]) ? 0 : 1;  // halo buffer used by half 1
-      for (int kb = kb0; kb < kb1; ++kb, ++q, ++it) {
-        const int slot = q & 1;
-        if (!warp_wait(&bar->ifull[slot], ring_parity(q, 2), abort_flag, err, p.timeout_ns)) {
+      int sp, mt, n0, kb0, kb1;
+      decode(u, sp, mt, n0, kb0, kb1);
+      const int cb = mt / kWgTiles;
+      const int j = 2 * (mt % kWgTiles) + half;        // tap of this warp's half (9: the extra half)
+      const int kind = j < 9 ? 0 : (cb == 0 ? 1 : 2);  // gathered X, ones row, padding
+      for (int kb = kb0; kb < kb1; ++kb, ++q) {
+        if ((int)(q & 1u) != grp) continue;
+        const int slot = (int)(q % kWgSlots);
+        const int sa = (int)(q % kTmemAStages);
+        if (!warp_wait(&bar->ifull[slot], ring_parity(q, kWgSlots), abort_flag, err, p.timeout_ns) ||
+            !warp_wait(&bar->aempty[sa], ring_parity(q, kTmemAStages) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
-        const int sa = it % SA;
-        if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
-          aborted = true;
-          break;
-        }
-        const HaloRange rg = sm.rng[slot];
-        const int32_t* sidx = sm.idx + slot * kWgIdx;
-        const uint32_t halo = smem_u32(sm.halo + (size_t)slot * 2 * kHaloBufBytes);
-        const uint32_t a_st = smem_u32(sm.a + (size_t)sa * kABytes);
+        tc_fence_after();  // the MMAs that read this A stage are complete
         const int k0 = kb * kBK;
+        const uint32_t a_col = tmem_base + kACol + (uint32_t)sa * kTmemAStageCols;
+        if (kind == 0) {
+          const int32_t* sidx = sm.idx + slot * kWgIdx;
+          const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
+          const int hlo = k0 - kWgPad;
+          const int mi = lane >> 3;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (kind[h] == 2) continue;
+          for (int sub = 0; sub < 2; ++sub) {
+            const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
+            uint32_t R[16];
+            bool far = false;
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int kk = ksub + 32 * rr;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (kind[h] == 0) {
-              const int idx = sidx[kk * 9 + tap[h]];
-              if (idx >= 0) {
-                if (!rg.fallback) {
-                  const int hr = idx - rg.lo;
-                  const uint32_t hbase = halo + (h == 0 ? 0u : (uint32_t)hsel1 * kHaloBufBytes);
-                  val = ld_shared_16(hbase + hr * 128 + ((chunk ^ (hr & 7)) << 4));
-                } else {
-                  val = ldg_16(p.X + (size_t)idx * p.Cin + cblk[h] * kBK + chunk * 8);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
+              int x = k0 + tk < p.n ? sidx[tk * 9 + j] : -1;
+              if (x >= p.n) {
+                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+                x = -1;
+              }
+              const int h = x - hlo;
+              const int chunk = (c16 >> 3) + (mi & 1);
+              uint32_t addr = zero_addr;
+              if (x >= 0) {
+                if ((unsigned)h < (unsigned)kWgHaloRows)
+                  addr = halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4);
+                else
+                  far = true;
+              }
+              ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
+            }
+            if (__any_sync(0xffffffffu, far)) {
+              // entries outside the halo window read as zero above: fetch them from global memory
+#pragma unroll
+              for (int r = 0; r < 16; ++r) {
+                const int k4 = r >> 2, m = r & 3;
+                const int ch = cb * kBK + c16 + 8 * (m & 1) + (lane >> 2);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int tk = 16 * k4 + 8 * (m >> 1) + 2 * (lane & 3) + e;
+                  const int x = k0 + tk < p.n ? sidx[tk * 9 + j] : -1;
+                  if (x >= 0 && x < p.n && (unsigned)(x - hlo) >= (unsigned)kWgHaloRows) {
+                    const uint32_t v = __ldg(X16 + (size_t)x * p.Cin + ch);
+                    R[r] = e == 0 ? ((R[r] & 0xFFFF0000u) | v) : ((R[r] & 0x0000FFFFu) | (v << 16));
+                  }
                 }
               }
-            } else if (chunk == 0 && k0 + kk < p.n) {
-              val.x = 0x3F80u;  // bf16 1.0 in element 0
             }
-            st_shared_v4(a_st + h * 8192 + kk * 128 + ((chunk ^ (kk & 7)) << 4), val);
+            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+          }
+        } else if (kind == 1) {
+          // row 0 of the extra half is 1 for every valid token: its accumulator row is db
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            uint32_t R[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) R[r] = 0u;
+            if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int tk = k0 + 8 * k + 2 * lane;
+                R[2 * k] = (tk < p.n ? 0x3F80u : 0u) | (tk + 1 < p.n ? 0x3F800000u : 0u);
+              }
+            }
+            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
           }
         }
-        warp_publish(&bar->afull[sa]);
+        // (padding halves are not written: their accumulator rows are never read)
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(&bar->afull[sa]);
         warp_arrive(&bar->iempty[slot]);
       }
     }
   } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       MmaCfg c;
-      c.idesc = idesc_bf16_f32(kBM, BN, 1, 1);
-      c.a_lbo = 8192, c.a_sbo = 1024, c.a_step = 2048;  // both MN-major: 64-wide groups 8 KB apart
-      c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;
-      MmaIssuer mi = make_issuer(sm, kBBytes, SA, SB, c);
+      c.idesc = idesc_bf16_f32(kBM, BN, 0, 1);  // A from tensor memory, B (dY) MN-major
+      c.a_lbo = 0, c.a_sbo = 0, c.a_step = 0;
+      c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // 64-wide N groups 8 KB apart, 16 K rows per step
+      MmaIssuer mi = make_issuer(sm, kBBytes, kTmemAStages, SB, c);
+      mi.a_tmem0 = tmem_base + kACol;
       uint32_t tc = 0;
       bool issued = false;
       for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
-        int sp, m0, n0, kb0, kb1;
-        decode(u, sp, m0, n0, kb0, kb1);
-        const uint32_t ab = tc & 1u;
-        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
+        int sp, mt, n0, kb0, kb1;
+        decode(u, sp, mt, n0, kb0, kb1);
+        const uint32_t ab = tc % (uint32_t)kAcc;
+        if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, kAcc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile<false>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
+        if (!mma_tile<true>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
     }
     __syncwarp();
   } else {
+    // ------------------------------------------------------------ epilogue: fp32 partial rows
     uint32_t tc = 0;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
-      int sp, m0, n0, kb0, kb1;
-      decode(u, sp, m0, n0, kb0, kb1);
-      const uint32_t ab = tc & 1u;
+      int sp, mt, n0, kb0, kb1;
+      decode(u, sp, mt, n0, kb0, kb1);
+      const uint32_t ab = tc % (uint32_t)kAcc;
       const bool empty_range = kb1 <= kb0;  // no MMA ran for this unit: its partial is zero
-      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, 2), abort_flag, err, p.timeout_ns)) break;
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, kAcc), abort_flag, err, p.timeout_ns)) break;
       tc_fence_after();
-      const int row = m0 + warp * 32 + lane;
+      const int row = mt * kBM + warp * 32 + lane;
       float* dst = p.partial + ((size_t)sp * p.rows_pad + row) * p.Cout + n0;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -993,15 +1037,14 @@ static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint
   return make_tmap(m, base, 2, dims, strides, box);
 }
 
-// Stage counts: up to 4 A stages (built in shared memory, short latency) and as
-// many B stages (TMA from L2) as fit in about 220 KB of shared memory.
-static void pick_stages(bool wgrad, int bn, int* sa, int* sb) {
+// Stage counts for the dense path: up to 4 A stages (short latency) and as many
+// B stages (TMA from L2) as fit in about 220 KB of shared memory.
+static void pick_stages(int bn, int* sa, int* sb) {
   const size_t budget = 220 * 1024;
-  for (int a = 4; a >= 2; --a) {
-    if (!wgrad && (a & 1)) continue;  // conv: two builder groups alternate A stages
+  for (int a = 4; a >= 2; a -= 2) {  // two builder groups alternate A stages: keep it even
     int b_best = 0;
     for (int b = 2; b <= kMaxStages; ++b) {
-      const Geometry g = wgrad ? wgrad_geometry(bn, a, b) : conv_geometry(bn, a, b, false);
+      const Geometry g = conv_geometry(bn, a, b, false);
       if (smem_total(g) <= budget) b_best = b;
     }
     if (b_best >= 3 || (a == 2 && b_best >= 2)) {
@@ -1024,7 +1067,7 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
     for (int b = 2; b <= kMaxStages; ++b)
       if (smem_total(conv_geometry(BN, 0, b, true)) <= 220 * 1024) prm.stages_b = b;
   } else {
-    pick_stages(false, BN, &prm.stages_a, &prm.stages_b);
+    pick_stages(BN, &prm.stages_a, &prm.stages_b);
   }
   const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b, a_in_tmem));
   static int done[64];
@@ -1087,7 +1130,7 @@ static int wgrad_bn(int Cout) { return Cout % 256 == 0 ? 256 : Cout % 128 == 0 ?
 
 void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn) {
   const int b = wgrad_bn(Cout);
-  const int rp = ((9 * Cin + 1 + kBM - 1) / kBM) * kBM;
+  const int rp = (Cin / kBK) * kWgTiles * kBM;  // 10 half-tiles of 64 rows per 64-channel block
   const int base_units = (rp / kBM) * (Cout / b);
   const int kbt = (n + kBK - 1) / kBK;
   int sp = sm_count() / base_units;
@@ -1100,8 +1143,11 @@ void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn
 
 template <int BN>
 static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t s) {
-  pick_stages(true, BN, &prm.stages_a, &prm.stages_b);
-  const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_a, prm.stages_b));
+  prm.stages_a = kTmemAStages;
+  prm.stages_b = 2;
+  for (int b = 2; b <= kMaxStages; ++b)
+    if (smem_total(wgrad_geometry(BN, b)) <= 220 * 1024) prm.stages_b = b;
+  const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_b));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
   if (e != cudaSuccess) return e;

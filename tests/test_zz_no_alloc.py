@@ -85,7 +85,7 @@ def test_noalloc_matches_workspace_entry_point_twice(sv, make, dtype):
 
 
 def test_noalloc_rejects_channels_beyond_the_scratch(sv):
-    # one split of C_in = C_out = 1024 needs (9*1024+1 -> 9344 rows) * 1024 floats = 36.5 MiB > 16 MiB
+    # one split of C_in = C_out = 1024 needs 16 x 640 = 10240 partial rows x 1024 floats = 40 MiB > 16 MiB
     X = torch.zeros((64, 1024), dtype=torch.bfloat16, device="cuda")
     nbr = torch.full((64, 9), -1, dtype=torch.int32, device="cuda")
     dW = torch.empty((1024, 9, 1024), device="cuda")
