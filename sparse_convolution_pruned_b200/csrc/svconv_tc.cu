@@ -11,20 +11,21 @@
 // needs are staged once: tokens are packed frame by frame (the page's packed
 // sequence), and within a frame in raster order a neighbour is at most W + 1
 // packed rows away, so the neighbours of 128 consecutive tokens lie in one
-// short contiguous "halo" range of rows.  That range is read with a few large
-// TMA boxes, and the A tile of every tap is assembled from it in shared memory.
-// When a tile's index range is too wide for the halo buffer (for example when
-// tokens are not in raster order), its A rows are read from global memory
-// directly: the result is the same, only slower.
+// short contiguous "halo" range of rows.  The kernels stage the fixed window of
+// rows m0 - 32 .. m0 + 127 + 32 around a tile (valid for W <= 31) with a few
+// large TMA boxes, issued together with the tile's index entries since the
+// window does not depend on them, and assemble the A tile of every tap from it.
+// A neighbour outside the window (wider grids, tokens not in raster order) is
+// read from global memory instead: the result is the same, only slower.
 //
 // Warp roles (480 threads):
 //   warps 0-3    epilogue: tcgen05.ld the fp32 accumulator (warp w owns TMEM
 //                lanes 32w..32w+31 = tile rows), bias / GELU / residual, bf16 store.
 //   warps 4-11   A builders: copy each tile row's neighbour segment from the halo
 //                into the 128B-swizzled K-major A stage (zeros for -1 = padding).
-//   warp 12      index / halo loader: reads the tile's neighbour rows, finds the
-//                halo range, issues the halo TMA boxes (or, for the dense adapter
-//                projections, the A tile itself).
+//   warp 12      index / halo loader: cp.async of the tile's neighbour entries and
+//                the halo window's TMA boxes (or, for the dense adapter
+//                projections, TMA of the A tile itself).
 //   warp 13      weight loader: TMA of the B tile (W_j, or W_j^T straight from
 //                W[o][j][i] as an MN-major operand for the data gradient).
 //   warp 14      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16) into
@@ -61,7 +62,8 @@ constexpr int kMmaWarp = kBWarp + 1;               // 14
 constexpr int kThreads = (kMmaWarp + 1) * 32;      // 480
 constexpr int kMaxStages = 8;
 constexpr int kHaloBox = 64;                       // rows per halo TMA box
-constexpr int kConvHaloRows = 192;                 // conv halo capacity (>= 128 + 2 * (W + 1) for W <= 31)
+constexpr int kConvPad = 32;                       // conv halo margin: W + 1 <= 32 stays inside
+constexpr int kConvHaloRows = kBM + 2 * kConvPad;  // conv halo window (A rows m0 - 32 .. m0 + 159)
 constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
 constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
 constexpr int kWgSlots = 4;                        // weight gradient: index + halo slots in flight
@@ -81,13 +83,6 @@ struct __align__(16) TcBarriers {
   uint64_t done;                                   // final MMA drain before TMEM is released
   uint32_t tmem_base;
   int abort_flag;
-};
-
-struct HaloRange {
-  int lo;        // first staged row
-  int rows;      // staged rows (0: nothing valid)
-  int fallback;  // 1: read A rows from global memory
-  int pad;
 };
 
 struct TcConvParams {
@@ -128,7 +123,6 @@ struct Carve {
   uint8_t* b;      // B ring
   uint8_t* halo;   // conv: 2 halo buffers; weight gradient: 2 slots x 2 halos
   int32_t* idx;    // 2 neighbour-row slots
-  HaloRange* rng;  // 2 ranges
   TcBarriers* bar;
 };
 
@@ -165,7 +159,7 @@ __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
 }
 
 __host__ __device__ inline size_t smem_total(const Geometry& g) {
-  return 1024 + g.a_bytes + g.b_bytes + g.halo_bytes + g.idx_bytes + 2 * sizeof(HaloRange) + sizeof(TcBarriers);
+  return 1024 + g.a_bytes + g.b_bytes + g.halo_bytes + g.idx_bytes + sizeof(TcBarriers);
 }
 
 __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
@@ -176,8 +170,7 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
   c.b = c.a + g.a_bytes;
   c.halo = c.b + g.b_bytes;
   c.idx = reinterpret_cast<int32_t*>(c.halo + g.halo_bytes);
-  c.rng = reinterpret_cast<HaloRange*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
-  c.bar = reinterpret_cast<TcBarriers*>(c.rng + 2);
+  c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
   return c;
 }
 
@@ -383,7 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
-    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 1, kProdWarps);  // one builder group per A stage
+    // afull: one builder group per A stage; ifull: the 32 cp.async arrivals of the loader lanes
+    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 32, kProdWarps);
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -400,7 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   if (warp == kHaloWarp) {
     // ------------------------------------------------------------ index / halo (or dense A) loader
     if (gather) {
-      uint32_t ti = 0, hi = 0;
+      // The tile's 128 x 9 neighbour entries arrive by cp.async on ifull[slot]; the
+      // halo window (A rows m0 - 32 .. m0 + 159) needs none of them, so its TMA boxes
+      // are issued right away and both loads are in flight together.
+      uint32_t ti = 0, hi = 0, ni = 0;  // ni: index loads issued
       bool aborted = false;
       for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
         const int m0 = (tile / n_tiles) * kBM;
@@ -409,41 +406,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
           aborted = true;
           break;
         }
-        // the tile's 128 x 9 neighbour entries: coalesced, all loads in flight together
         const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
         const int lim = min(M - m0, kBM) * 9;
-        int v[kConvIdx / 32];
+        const uint32_t dst = smem_u32(sm.idx + slot * kConvIdx);
 #pragma unroll
         for (int i = 0; i < kConvIdx / 32; ++i) {
           const int e = lane + 32 * i;
-          v[i] = e < lim ? __ldg(src + e) : -1;
+          cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
         }
-        int vmin = INT_MAX, vmax = -1;
-        int32_t* sidx = sm.idx + slot * kConvIdx;
-#pragma unroll
-        for (int i = 0; i < kConvIdx / 32; ++i) {
-          int x = v[i];
-          if (x >= 0) {
-            x -= nbr_base;
-            if ((unsigned)x >= (unsigned)p.a_rows) {
-              atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-              x = -1;
-            }
-          }
-          if (x >= 0) {
-            vmin = min(vmin, x);
-            vmax = max(vmax, x);
-          }
-          sidx[lane + 32 * i] = x;
-        }
-        vmin = warp_min(vmin);
-        vmax = warp_max(vmax);
-        const int rows = vmax >= 0 ? vmax - vmin + 1 : 0;
-        const bool fallback = rows == 0 || rows > kConvHaloRows;
-        if (lane == 0) sm.rng[slot] = HaloRange{vmin, rows, fallback ? 1 : 0, 0};
-        warp_arrive(&bar->ifull[slot]);  // release: the entries and the range are visible
-        if (fallback) continue;
-        const int nbox = (rows + kHaloBox - 1) / kHaloBox;
+        cp_async_arrive_noinc(&bar->ifull[slot]);
+        ++ni;
         for (int cb = 0; cb < kb_per_tap; ++cb, ++hi) {
           const int hb = hi & 1;
           if (!warp_wait(&bar->hempty[hb], ring_parity(hi, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
@@ -451,15 +423,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             break;
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&bar->hfull[hb], (uint32_t)nbox * kHaloBox * 128);
-            const uint32_t dst = smem_u32(sm.halo + hb * kHaloBufBytes);
-            for (int q = 0; q < nbox; ++q)
-              tma_load_2d(dst + q * kHaloBox * 128, &p.tmap_a, &bar->hfull[hb], cb * kBK, vmin + q * kHaloBox);
+            mbar_arrive_expect_tx(&bar->hfull[hb], kHaloBufBytes);
+            const uint32_t hdst = smem_u32(sm.halo + hb * kHaloBufBytes);
+#pragma unroll
+            for (int q = 0; q < kConvHaloRows / kHaloBox; ++q)
+              tma_load_2d(hdst + q * kHaloBox * 128, &p.tmap_a, &bar->hfull[hb], cb * kBK,
+                          m0 - kConvPad + q * kHaloBox);
           }
           __syncwarp();
         }
       }
-      if (aborted) drain_ring(bar->hfull, hi, 2, err, p.timeout_ns);
+      if (aborted) {
+        drain_ring(bar->ifull, ni, 2, err, p.timeout_ns);
+        drain_ring(bar->hfull, hi, 2, err, p.timeout_ns);
+      }
     } else {
       const int a_base = p.a_abs ? lo : 0;
       uint32_t it = 0;
@@ -515,7 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     // with counter parity g, i.e. A stages g and g+2).  Each thread owns one tile row:
     // warp w may only touch TMEM lanes 32*(w%4) .. +31, so thread (w, lane) copies
     // row 32*(w%4) + lane.  It reads the row's neighbour segment from the halo in
-    // shared memory (or global memory on the fallback path) and writes it straight
+    // shared memory (or, for a neighbour outside the halo window, from global
+    // memory) and writes it straight
     // into the tensor-memory A stage with tcgen05.st: no shared-memory stores, no
     // proxy fence, and the MMA reads only B from shared memory.
     if (gather) {
@@ -531,12 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
           aborted = true;
           break;
         }
-        const HaloRange rg = sm.rng[slot];
+        const int m0 = (tile / n_tiles) * kBM;
+        const bool row_ok = m0 + r < M;
+        const int hlo = m0 - kConvPad;  // A row of halo row 0
         const int32_t* sidx = sm.idx + slot * kConvIdx;
         for (int cb = 0; cb < kb_per_tap && !aborted; ++cb) {
           const int hb = hi & 1;
-          if (!rg.fallback &&
-              !warp_wait(&bar->hfull[hb], ring_parity(hi, 2), abort_flag, err, p.timeout_ns)) {
+          if (!warp_wait(&bar->hfull[hb], ring_parity(hi, 2), abort_flag, err, p.timeout_ns)) {
             aborted = true;
             break;
           }
@@ -550,10 +529,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               break;
             }
             tc_fence_after();  // the MMAs that read this stage are complete
-            const int idx = sidx[r * 9 + jj];
+            int idx = row_ok ? sidx[r * 9 + jj] : -1;
+            if (idx >= 0) {
+              idx -= nbr_base;
+              if ((unsigned)idx >= (unsigned)p.a_rows) {
+                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+                idx = -1;
+              }
+            }
+            const int h = idx - hlo;
             uint32_t v[32];
-            if (idx >= 0 && !rg.fallback) {
-              const int h = idx - rg.lo;
+            if (idx >= 0 && (unsigned)h < (unsigned)kConvHaloRows) {
               const uint32_t row = halo + h * 128;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
@@ -576,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             tc_fence_before();
             warp_arrive(&bar->afull[sa]);
           }
-          if (!rg.fallback && !aborted) {
+          if (!aborted) {
             warp_arrive(&bar->hempty[hb]);
             ++hi;
           }

@@ -172,6 +172,10 @@ BF16_FULL_CASES = [
                                                      dtype="bf16")),
     ("C320x64_allkept", lambda: wl.custom_conv(seed=33, T=2, H=12, W=12, keep_frac=1.0, Cin=320, Cout=64,
                                                dtype="bf16")),
+    # W + 1 = 81 packed rows: vertical neighbours fall outside the kernels' staged
+    # halo windows and are read from global memory
+    ("wide_grid_5x80_C64", lambda: wl.custom_conv(seed=34, T=6, H=5, W=80, keep_frac=0.6, Cin=64, Cout=64,
+                                                  dtype="bf16")),
 ]
 
 
