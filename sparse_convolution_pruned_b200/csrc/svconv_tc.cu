@@ -337,6 +337,59 @@ __device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err
   }
 }
 
+// Epilogue of one output tile row: the fp32 accumulator row at TMEM address acc (this
+// warp's lane quarter, column 0 of the tile) + bias, GELU, residual -> bf16 row orow,
+// columns n0 .. n0 + BN - 1.  Two 32-column loads are in flight per wait.
+template <int BN>
+__device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t acc, bool valid, size_t orow, int n0) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    uint32_t v[2][32];
+    tmem_ld_32x32b_x32(acc + c0, v[0]);
+    tmem_ld_32x32b_x32(acc + c0 + 32, v[1]);
+    tmem_ld_wait();
+    if (!valid) continue;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int c = c0 + 32 * hh;
+      float f[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[hh][q]);
+      if (p.bias) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c + q);
+      }
+      if (p.gelu) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) f[q] = 0.5f * f[q] * (1.0f + erff(f[q] * 0.70710678118654752f));
+      }
+      if (p.residual) {
+        const uint4* rp = reinterpret_cast<const uint4*>(p.residual + orow * p.ldo + n0 + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 u = rp[q];
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 x2 = __bfloat1622float2(h[e]);
+            f[q * 8 + 2 * e] += x2.x;
+            f[q * 8 + 2 * e + 1] += x2.y;
+          }
+        }
+      }
+      uint4* op = reinterpret_cast<uint4*>(p.out + orow * p.ldo + n0 + c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[q * 8 + 2 * e], f[q * 8 + 2 * e + 1]);
+        op[q] = u;
+      }
+    }
+  }
+}
+
 // ============================================================================ conv / dense GEMM
 // MIRROR: gather through column 8-j (data gradient); it always pairs with an
 // MN-major weight operand.
@@ -611,49 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       const int row = m0 + warp * 32 + lane;
       const int orow_i = out_base + row;
       const bool valid = row < M && orow_i >= 0 && orow_i < p.out_rows;
-      const size_t orow = (size_t)orow_i;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
-        tmem_ld_wait();
-        if (valid) {
-          float f[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
-          if (p.bias) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c0 + q);
-          }
-          if (p.gelu) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) f[q] = 0.5f * f[q] * (1.0f + erff(f[q] * 0.70710678118654752f));
-          }
-          if (p.residual) {
-            const uint4* rp = reinterpret_cast<const uint4*>(p.residual + orow * p.ldo + n0 + c0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 u = rp[q];
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float2 x2 = __bfloat1622float2(h[e]);
-                f[q * 8 + 2 * e] += x2.x;
-                f[q * 8 + 2 * e + 1] += x2.y;
-              }
-            }
-          }
-          uint4* op = reinterpret_cast<uint4*>(p.out + orow * p.ldo + n0 + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 u;
-            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[q * 8 + 2 * e], f[q * 8 + 2 * e + 1]);
-            op[q] = u;
-          }
-        }
-      }
+      epilogue_rows<BN>(p, tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN, valid, (size_t)orow_i, n0);
       tc_fence_before();
       warp_arrive(&bar->tempty[ab]);
     }
@@ -664,6 +675,262 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ============================================================================ small-channel conv
+// C = 64 on the gathered side and 64 output columns (the small-channel adapter
+// conv and its data gradient).  Here an MMA is short (128x64x16) and the per-stage
+// handshakes of the general kernel (an mbarrier wait on A and on B before every 4
+// MMAs) cost more than the MMAs themselves.  So this kernel keeps all of W (9 taps x
+// 64 x 64 bf16 = 72 KB) resident in shared memory, holds all 9 gathered A taps of a
+// tile in tensor memory at once (9 x 32 columns next to two 64-column accumulators),
+// and synchronises the MMA issuer with the builders twice per tile (one barrier per
+// builder group: taps 0-4 and 5-8) instead of twice per tap.  The first two tiles'
+// index entries, halo windows and W are requested before the CTA's setup barrier.
+constexpr int kSmallTaps0 = 5;                    // builder group 0: taps 0..4, group 1: 5..8
+constexpr uint32_t kSmallACol = 128;              // A taps after the two accumulators
+constexpr uint32_t kSmallTmemCols = 512;          // 128 + 9 * 32 = 416 columns used
+constexpr uint32_t kSmallWBytes = 9 * 64 * 64 * 2;
+
+struct __align__(16) SmallBars {
+  uint64_t wfull;
+  uint64_t lfull[2], lempty[2];  // index entries + halo window of a tile
+  uint64_t afull[2], aempty[2];  // per builder group
+  uint64_t tfull[2], tempty[2];  // accumulators
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__host__ __device__ constexpr size_t small_smem_bytes() {
+  return 1024 + kSmallWBytes + 2 * (size_t)kConvHaloRows * 128 + 2 * (size_t)kConvIdx * 4 + sizeof(SmallBars);
+}
+
+template <bool MIRROR>
+__global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid_constant__ TcConvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  constexpr uint32_t kHaloBufBytes = kConvHaloRows * 128;
+  const uint32_t sbase = smem_u32(smem_raw);
+  uint8_t* sw = smem_raw + (((sbase + 1023u) & ~1023u) - sbase);
+  uint8_t* shalo = sw + kSmallWBytes;
+  int32_t* sidx = reinterpret_cast<int32_t*>(shalo + 2 * kHaloBufBytes);
+  SmallBars* bar = reinterpret_cast<SmallBars*>(reinterpret_cast<uint8_t*>(sidx) + 2 * kConvIdx * 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* err = p.status;
+  const int M = p.M;
+  const int num_tiles = (M + kBM - 1) / kBM;
+
+  // index entries (cp.async, one arrival per lane) and the halo window (TMA) of a tile
+  auto issue_tile = [&](int tile, int slot) {
+    const int m0 = tile * kBM;
+    const int32_t* src = p.nbr + (size_t)m0 * 9;
+    const int lim = min(M - m0, kBM) * 9;
+    const uint32_t dst = smem_u32(sidx + slot * kConvIdx);
+#pragma unroll
+    for (int i = 0; i < kConvIdx / 32; ++i) {
+      const int e = lane + 32 * i;
+      cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
+    }
+    cp_async_arrive_noinc(&bar->lfull[slot]);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar->lfull[slot], kHaloBufBytes);
+      const uint32_t hdst = smem_u32(shalo + slot * kHaloBufBytes);
+#pragma unroll
+      for (int q = 0; q < kConvHaloRows / kHaloBox; ++q)
+        tma_load_2d(hdst + q * kHaloBox * 128, &p.tmap_a, &bar->lfull[slot], 0, m0 - kConvPad + q * kHaloBox);
+    }
+    __syncwarp();
+  };
+
+  // ---- setup: the loaders initialise their own barriers and start their first copies
+  uint32_t issued = 0;
+  if (warp == kHaloWarp) {
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bar->lfull[i], 33);  // 32 cp.async arrivals + the expect_tx arrival
+        mbar_init(&bar->lempty[i], kProdWarps);
+      }
+      fence_barrier_init();
+      fence_proxy_async_smem();
+      prefetch_tmap(&p.tmap_a);
+    }
+    __syncwarp();
+    for (int t = blockIdx.x; t < num_tiles && issued < 2; t += gridDim.x) issue_tile(t, (int)issued++);
+  } else if (warp == kBWarp) {
+    if (lane == 0) {
+      mbar_init(&bar->wfull, 1);
+      fence_barrier_init();
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bar->wfull, kSmallWBytes);
+      const uint32_t dst = smem_u32(sw);
+      for (int j = 0; j < 9; ++j) {
+        if constexpr (!MIRROR) {
+          tma_load_2d(dst + j * 8192, &p.tmap_b, &bar->wfull, j * 64, 0);  // W_j [o][i], K-major
+        } else {
+          tma_load_3d(dst + j * 8192, &p.tmap_b, &bar->wfull, 0, j, 0);   // W_j^T: [o] rows of i, MN-major
+        }
+      }
+    }
+    __syncwarp();
+  } else if (threadIdx.x == 0) {
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bar->afull[g], kProdWarps / 2);
+      mbar_init(&bar->aempty[g], 1);
+      mbar_init(&bar->tfull[g], 1);
+      mbar_init(&bar->tempty[g], kEpiWarps);
+    }
+    mbar_init(&bar->done, 1);
+    bar->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bar->tmem_base, kSmallTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bar->tmem_base;
+  volatile int* abort_flag = &bar->abort_flag;
+
+  if (warp == kHaloWarp) {
+    // ------------------------------------------------------------ index / halo loader (tiles 2, 3, ...)
+    bool aborted = false;
+    uint32_t ti = issued;
+    for (int tile = blockIdx.x + (int)issued * gridDim.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      const int slot = ti & 1;
+      if (!warp_wait(&bar->lempty[slot], ring_parity(ti, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
+        aborted = true;
+        break;
+      }
+      issue_tile(tile, slot);
+      ++issued;
+    }
+    if (aborted) drain_ring(bar->lfull, issued, 2, err, p.timeout_ns);
+  } else if (warp == kBWarp) {
+    // W stays resident; make sure its copy has landed before the CTA can exit
+    if (lane == 0) {
+      volatile int never = 0;
+      mbar_wait(&bar->wfull, 0, &never, err, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= kEpiWarps && warp < kHaloWarp) {
+    // ------------------------------------------------------------ A builders
+    // Thread (w, lane) owns tile row 32 (w % 4) + lane; group 0 writes taps 0-4 and
+    // group 1 taps 5-8 of that row into their tensor-memory columns.
+    const int grp = (warp - kEpiWarps) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int j0 = grp ? kSmallTaps0 : 0, j1 = grp ? 9 : kSmallTaps0;
+    const uint32_t a_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + kSmallACol;
+    uint32_t ti = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      const int slot = ti & 1;
+      if (!warp_wait(&bar->lfull[slot], ring_parity(ti, 2), abort_flag, err, p.timeout_ns) ||
+          !warp_wait(&bar->aempty[grp], (ti & 1u) ^ 1u, abort_flag, err, p.timeout_ns))
+        break;
+      tc_fence_after();  // the previous tile's MMAs have finished reading these columns
+      const int m0 = tile * kBM;
+      const bool row_ok = m0 + r < M;
+      const int hlo = m0 - kConvPad;
+      const uint32_t halo = smem_u32(shalo + slot * kHaloBufBytes);
+      const int32_t* si = sidx + slot * kConvIdx;
+      for (int j = j0; j < j1; ++j) {
+        const int jj = MIRROR ? 8 - j : j;
+        int idx = row_ok ? si[r * 9 + jj] : -1;
+        if (idx >= 0 && (unsigned)idx >= (unsigned)p.a_rows) {
+          atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+          idx = -1;
+        }
+        const int h = idx - hlo;
+        uint32_t v[32];
+        if (idx >= 0 && (unsigned)h < (unsigned)kConvHaloRows) {
+          const uint32_t row = halo + h * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 q = ld_shared_16(row + ((c ^ (h & 7)) << 4));
+            v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+          }
+        } else if (idx >= 0) {
+          const __nv_bfloat16* src = p.A + (size_t)idx * p.lda;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 q = ldg_16(src + c * 8);
+            v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = 0u;
+        }
+        tmem_st_32x32b_x32(a_lane + (uint32_t)j * kTmemAStageCols, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      warp_arrive(&bar->afull[grp]);
+      warp_arrive(&bar->lempty[slot]);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer: 36 MMAs per tile, 2 waits
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, 64, 0, MIRROR ? 1 : 0);
+      const uint64_t b0 = MIRROR ? smem_desc_sw128(smem_u32(sw), 8192, 1024) : smem_desc_sw128(smem_u32(sw), 16, 1024);
+      const uint32_t k16 = MIRROR ? (2048u >> 4) : (32u >> 4);  // start-address step per K=16
+      bool issued_any = false;
+      if (mbar_wait(&bar->wfull, 0, abort_flag, err, p.timeout_ns)) {
+        uint32_t tc = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+          const uint32_t ab = tc & 1u;
+          if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, 2) ^ 1u, abort_flag, err, p.timeout_ns)) break;
+          const uint32_t d = tmem_base + ab * 64;
+          bool ok = true;
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (!mbar_wait(&bar->afull[g], tc & 1u, abort_flag, err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issued_any = true;
+            const int j0 = g ? kSmallTaps0 : 0, j1 = g ? 9 : kSmallTaps0;
+            for (int j = j0; j < j1; ++j) {
+              const uint64_t bd = b0 + (uint64_t)((uint32_t)j * (8192u >> 4));
+              const uint32_t at = tmem_base + kSmallACol + (uint32_t)j * kTmemAStageCols;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * k16), idesc, (j | k) != 0 ? 1u : 0u);
+            }
+            tc_commit(&bar->aempty[g]);
+          }
+          if (!ok) break;
+          tc_commit(&bar->tfull[ab]);
+        }
+      }
+      if (issued_any) {
+        volatile int never = 0;
+        tc_commit(&bar->done);
+        mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    uint32_t tc = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+      const uint32_t ab = tc & 1u;
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, 2), abort_flag, err, p.timeout_ns)) break;
+      tc_fence_after();
+      const int row = tile * kBM + warp * 32 + lane;
+      epilogue_rows<64>(p, tmem_base + ((uint32_t)(warp * 32) << 16) + ab * 64, row < M, (size_t)row, 0);
+      tc_fence_before();
+      warp_arrive(&bar->tempty[ab]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kSmallTmemCols);
   }
 }
 
@@ -1063,6 +1330,16 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
   return cudaGetLastError();
 }
 
+template <bool MIRROR>
+static cudaError_t launch_small_inst(const TcConvParams& prm, int grid, cudaStream_t s) {
+  const size_t smem = small_smem_bytes();
+  static int done[64];
+  cudaError_t e = ensure_smem_attr(tc_conv_small_kernel<MIRROR>, smem, done);
+  if (e != cudaSuccess) return e;
+  tc_conv_small_kernel<MIRROR><<<grid, kThreads, smem, s>>>(prm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s) {
   TcConvParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -1106,6 +1383,9 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   if (tiles == 0) return cudaSuccess;
   int grid = sm_count();
   if (grid > tiles) grid = tiles;
+  // 64 gathered channels and 64 output columns, whole-table rows: W-resident small-channel kernel
+  if (a.nbr && a.Kc == 64 && a.N == 64 && bn == 64 && !a.row_lo && !a.a_abs && !a.nbr_abs && !a.out_abs)
+    return a.mirror ? launch_small_inst<true>(prm, grid, s) : launch_small_inst<false>(prm, grid, s);
   if (bn == 256) return a.mirror ? launch_conv_inst<256, true>(prm, grid, s) : launch_conv_inst<256, false>(prm, grid, s);
   if (bn == 128) return a.mirror ? launch_conv_inst<128, true>(prm, grid, s) : launch_conv_inst<128, false>(prm, grid, s);
   if (bn == 64) return a.mirror ? launch_conv_inst<64, true>(prm, grid, s) : launch_conv_inst<64, false>(prm, grid, s);
