@@ -57,21 +57,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to suspend_ns until the phase
+// completes instead of returning at once: a waiting warp then issues no shared-memory
+// traffic of its own while it waits.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false if the CTA
-// is aborting (another thread timed out) or this wait ran past timeout_ns.
+// is aborting (another thread timed out) or this wait ran past timeout_ns.  Between
+// checks of the abort flag and the clock the thread sleeps in try_wait (up to 20 us).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* err_word, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) {
-        *abort_flag = 1;
-        atomicOr(err_word, SVCONV_STATUS_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      atomicOr(err_word, SVCONV_STATUS_TIMEOUT);
+      return false;
     }
   }
 }
@@ -105,6 +119,11 @@ __device__ __forceinline__ uint4 ld_shared_16(uint32_t src) {
   return v;
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t dst, uint4 v) { st_shared_16(dst, v.x, v.y, v.z, v.w); }
+__device__ __forceinline__ int ld_shared_s32(uint32_t src) {
+  int v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(src) : "memory");
+  return v;
+}
 
 // Four 8x8 b16 matrices, transposed on the way in: thread i supplies the address of
 // row (i & 7) of matrix i >> 3 (16 bytes); register m of thread t receives column t / 4

@@ -66,7 +66,9 @@ constexpr int kConvPad = 32;                       // conv halo margin: W + 1 <=
 constexpr int kConvHaloRows = kBM + 2 * kConvPad;  // conv halo window (A rows m0 - 32 .. m0 + 159)
 constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
 constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
-constexpr int kWgSlots = 4;                        // weight gradient: index + halo slots in flight
+__host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: index + halo slots in flight
+  return bn == 256 ? 4 : 8;                                // (covers ~2 us of load latency at small C)
+}
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
@@ -148,10 +150,10 @@ __host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem) {
                    (a_in_tmem ? (uint32_t)(kTmemAStages * kTmemAStageCols) : 0u));
 }
 
-// Weight gradient: A lives in tensor memory; kWgSlots slots of (index entries, halo).
+// Weight gradient: A lives in tensor memory; wgrad_slots(bn) slots of (index entries, halo).
 __host__ __device__ inline Geometry wgrad_geometry(int bn, int sb) {
-  return {(size_t)0, (size_t)sb * bn * kBK * 2, (size_t)kWgSlots * kWgHaloRows * 128,
-          round_up((size_t)kWgSlots * kWgIdx * 4, 16)};
+  return {(size_t)0, (size_t)sb * bn * kBK * 2, (size_t)wgrad_slots(bn) * kWgHaloRows * 128,
+          round_up((size_t)wgrad_slots(bn) * kWgIdx * 4, 16)};
 }
 __host__ __device__ constexpr int wgrad_acc_buffers(int bn) { return bn == 256 ? 1 : 2; }
 __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         const int m0 = (tile / n_tiles) * kBM;
         const bool row_ok = m0 + r < M;
         const int hlo = m0 - kConvPad;  // A row of halo row 0
-        const int32_t* sidx = sm.idx + slot * kConvIdx;
+        const uint32_t sidx_s = smem_u32(sm.idx + slot * kConvIdx);
         for (int cb = 0; cb < kb_per_tap && !aborted; ++cb) {
           const int hb = hi & 1;
           if (!warp_wait(&bar->hfull[hb], ring_parity(hi, 2), abort_flag, err, p.timeout_ns)) {
@@ -582,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               break;
             }
             tc_fence_after();  // the MMAs that read this stage are complete
-            int idx = row_ok ? sidx[r * 9 + jj] : -1;
+            int idx = row_ok ? ld_shared_s32(sidx_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
             if (idx >= 0) {
               idx -= nbr_base;
               if ((unsigned)idx >= (unsigned)p.a_rows) {
@@ -835,10 +837,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
       const bool row_ok = m0 + r < M;
       const int hlo = m0 - kConvPad;
       const uint32_t halo = smem_u32(shalo + slot * kHaloBufBytes);
-      const int32_t* si = sidx + slot * kConvIdx;
+      const uint32_t si_s = smem_u32(sidx + slot * kConvIdx);
       for (int j = j0; j < j1; ++j) {
         const int jj = MIRROR ? 8 - j : j;
-        int idx = row_ok ? si[r * 9 + jj] : -1;
+        int idx = row_ok ? ld_shared_s32(si_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
         if (idx >= 0 && (unsigned)idx >= (unsigned)p.a_rows) {
           atomicOr(err, SVCONV_STATUS_BAD_INDEX);
           idx = -1;
@@ -967,6 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   constexpr uint32_t kTmemCols = wgrad_tmem_cols(BN);
   constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
+  constexpr int kSlots = wgrad_slots(BN);
 
   const int m_tiles = p.rows_pad / kBM;
   const int n_tiles = p.Cout / BN;
@@ -975,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     // ifull: 32 cp.async arrivals of the loader lanes + its expect_tx arrival
-    init_barriers(bar, kTmemAStages, SB, kProdWarps / 2, kWgSlots, 33, kProdWarps / 2);
+    init_barriers(bar, kTmemAStages, SB, kProdWarps / 2, kSlots, 33, kProdWarps / 2);
     prefetch_tmap(&p.tmap_x);
     prefetch_tmap(&p.tmap_dy);
   }
@@ -1010,8 +1013,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       decode(u, sp, mt, n0, kb0, kb1);
       const int cb = mt / kWgTiles;
       for (int kb = kb0; kb < kb1; ++kb, ++q) {
-        const int slot = (int)(q % kWgSlots);
-        if (!warp_wait(&bar->iempty[slot], ring_parity(q, kWgSlots) ^ 1u, abort_flag, err, p.timeout_ns)) {
+        const int slot = (int)(q % kSlots);
+        if (!warp_wait(&bar->iempty[slot], ring_parity(q, kSlots) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
@@ -1035,7 +1038,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         __syncwarp();
       }
     }
-    if (aborted) drain_ring(bar->ifull, q, kWgSlots, err, p.timeout_ns);
+    if (aborted) drain_ring(bar->ifull, q, kSlots, err, p.timeout_ns);
   } else if (warp == kBWarp) {
     // ------------------------------------------------------------ dY tiles
     uint32_t it = 0;
@@ -1084,9 +1087,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       const int kind = j < 9 ? 0 : (cb == 0 ? 1 : 2);  // gathered X, ones row, padding
       for (int kb = kb0; kb < kb1; ++kb, ++q) {
         if ((int)(q & 1u) != grp) continue;
-        const int slot = (int)(q % kWgSlots);
+        const int slot = (int)(q % kSlots);
         const int sa = (int)(q % kTmemAStages);
-        if (!warp_wait(&bar->ifull[slot], ring_parity(q, kWgSlots), abort_flag, err, p.timeout_ns) ||
+        if (!warp_wait(&bar->ifull[slot], ring_parity(q, kSlots), abort_flag, err, p.timeout_ns) ||
             !warp_wait(&bar->aempty[sa], ring_parity(q, kTmemAStages) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
@@ -1095,7 +1098,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         const int k0 = kb * kBK;
         const uint32_t a_col = tmem_base + kACol + (uint32_t)sa * kTmemAStageCols;
         if (kind == 0) {
-          const int32_t* sidx = sm.idx + slot * kWgIdx;
+          const uint32_t sidx_s = smem_u32(sm.idx + slot * kWgIdx);
           const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
           const int hlo = k0 - kWgPad;
           const int mi = lane >> 3;
@@ -1107,7 +1110,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
-              int x = k0 + tk < p.n ? sidx[tk * 9 + j] : -1;
+              int x = k0 + tk < p.n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
               if (x >= p.n) {
                 atomicOr(err, SVCONV_STATUS_BAD_INDEX);
                 x = -1;
@@ -1132,7 +1135,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                   const int tk = 16 * k4 + 8 * (m >> 1) + 2 * (lane & 3) + e;
-                  const int x = k0 + tk < p.n ? sidx[tk * 9 + j] : -1;
+                  const int x = k0 + tk < p.n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
                   if (x >= 0 && x < p.n && (unsigned)(x - hlo) >= (unsigned)kWgHaloRows) {
                     const uint32_t v = __ldg(X16 + (size_t)x * p.Cin + ch);
                     R[r] = e == 0 ? ((R[r] & 0xFFFF0000u) | v) : ((R[r] & 0x0000FFFFu) | (v << 16));
