@@ -75,13 +75,13 @@ def roofline_entry(name, work, ms, peaks):
             "frac": achieved / peaks["hbm_gbs"]}
 
 
-def kernel_traffic(kernel_key):
+def kernel_traffic(workload_key, kernel_key):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    ent = d.get(kernel_key)
+    ent = d.get(f"{workload_key}/{kernel_key}")
     if not ent:
         return None
     src = os.path.join(ROOT, ent["source"])
@@ -418,7 +418,7 @@ def run_b200(args):
         roof = dict(kern[top])
         roof.pop("ms")
         roof["kernel"] = top
-        roof["traffic"] = kernel_traffic(top)
+        roof["traffic"] = kernel_traffic(args.workload, top)
         roof["peak_source"] = peaks["source"]
         tokens = n * world
         line = {
