@@ -206,6 +206,8 @@ def run_reference(args):
     import oracle
     oracle.build()
     w = make_inputs(0)
+    if WORKLOAD == "adapter":
+        return run_reference_adapter(args, w)
     # each step: the first frames of the workload, about 4e9 multiply-adds (a few seconds)
     frames = oracle_frames(w, 4e9)
     for _ in range(args.warmup):
@@ -221,12 +223,44 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n_kept": w.n, "sample": f"first {frames} of {w.T} frames per step"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
                          "sample": f"index+fwd+bwd_data+bwd_weight on the first {frames} frames "
-                                   f"({int(w.frame_off[frames])} tokens) per step"},
+                                   f"({int(w.frame_off[frames])} tokens) per step; 1 core used of "
+                                   f"{os.cpu_count()}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+    return 0
+
+
+def run_reference_adapter(args, w):
+    """Oracle index build + adapter forward on the first 8 frames of the long video per step."""
+    import oracle
+    frames = 8
+    r1 = int(w.frame_off[frames])
+
+    def one():
+        t0 = time.perf_counter()
+        sub_n, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W,
+                                         want_map=False)
+        oracle.adapter_fwd(w.X[:r1], sub_n, 0, r1, w.Wd, w.Wc, w.Wu)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        one()
+    tot = sum(one() for _ in range(args.steps))
+    value = r1 * args.steps / tot
+    sample = (f"index build + adapter forward on the first {frames} of {w.T} frames ({r1} tokens) per step; "
+              f"single-threaded C, fp64; 1 core used of {os.cpu_count()}")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n_kept": w.n, "sample": f"first {frames} of {w.T} frames per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
     return 0
 
 
@@ -293,10 +327,11 @@ def run_b200(args):
         if world > 1:
             dist.all_reduce(grads)
 
-    def timed_loop(fn, steps, warmup):
+    def timed_loop(fn, steps, warmup, flush_l2=True):
         with torch.cuda.stream(stream):
             for _ in range(warmup):
-                flush.zero_()
+                if flush_l2:
+                    flush.zero_()
                 fn()
             torch.cuda.synchronize()
             if world > 1:
@@ -304,7 +339,8 @@ def run_b200(args):
             torch.cuda.synchronize()
             evs = []
             for _ in range(steps):
-                flush.zero_()
+                if flush_l2:
+                    flush.zero_()
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
@@ -321,11 +357,13 @@ def run_b200(args):
         total_ms = timed_loop(one_step, args.steps, args.warmup)
     clocks = clk.summary()
     fwd_ms = timed_loop(g_fwd.replay, args.steps, args.warmup)
+    # the same step with the workload left in L2 between steps (reported beside the flushed number)
+    hot_ms = timed_loop(one_step, args.steps, args.warmup, flush_l2=False)
 
-    t = torch.tensor([total_ms, fwd_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([total_ms, fwd_ms, hot_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms = float(t[0]), float(t[1])
+    total_ms, fwd_ms, hot_ms = float(t[0]), float(t[1]), float(t[2])
 
     # per-kernel durations (events between the library calls on the launching stream)
     names = ["build_index", "fwd", "bwd_data", "bwd_weight"]
@@ -404,9 +442,10 @@ def run_b200(args):
             d, r = cpu_oracle_step(w, frames)
             dt += d
             toks += r
-        cpu = {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+        cpu = {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
                "sample": f"index+fwd+bwd_data+bwd_weight on the first {frames} of {w.T} frames "
-                         f"({int(w.frame_off[frames])} tokens), {reps} time(s); single-threaded C, fp64"}
+                         f"({int(w.frame_off[frames])} tokens), {reps} time(s); single-threaded C, fp64; "
+                         f"1 core used of {os.cpu_count()}"}
 
     if rank == 0:
         peaks = load_peaks()
@@ -433,6 +472,8 @@ def run_b200(args):
                        "graph": "step replayed from a CUDA graph", "parallelism": f"dp{world}"},
             "fwd": {"value": tokens * args.steps / (fwd_ms * 1e-3), "unit": UNIT,
                     "ms_per_step": fwd_ms / args.steps, "step": "build_index+fwd"},
+            "l2_hot": {"value": tokens * args.steps / (hot_ms * 1e-3), "unit": UNIT,
+                       "ms_per_step": hot_ms / args.steps, "note": "same step, no L2 flush between steps"},
             "roofline": roof,
             "kernels": kern,
             "e2e": {"value": tokens * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
@@ -448,6 +489,189 @@ def run_b200(args):
     return 0
 
 
+def host_cpu():
+    """CPU model and logical core count of this host (for the CPU-baseline record)."""
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
+# ----------------------------------------------------------------------------- adapter workload (a5)
+def run_adapter(args):
+    """Long-video bottleneck adapter: one step = index build + chunked adapter forward.
+
+    X (n x 1024 bf16, 579 MB at the full size) is read and written in place each step,
+    far larger than L2, so no flush is needed between steps.
+    """
+    import torch
+    import torch.distributed as dist
+
+    from sparse_convolution_pruned_b200 import svconv as sv
+
+    rank, local, world = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    w = make_inputs(rank)
+    n, T, D, R = w.n, w.T, w.D, w.R
+    chunk_T = 512
+    offs = w.frame_off.astype(np.int64)
+    max_rows = int(max(offs[min(t + chunk_T, T)] - offs[t] for t in range(0, T, chunk_T)))
+
+    h_coords = torch.from_numpy(w.coords).pin_memory()
+    h_off = torch.from_numpy(w.frame_off).pin_memory()
+    h_X = torch.from_numpy(w.X).to(torch.bfloat16).pin_memory()
+    torch.cuda.reset_peak_memory_stats(dev)
+    coords = h_coords.to(dev)
+    off = h_off.to(dev)
+    X = h_X.to(dev)
+    Wd = torch.from_numpy(w.Wd).to(torch.bfloat16).to(dev)
+    Wc = torch.from_numpy(w.Wc).to(torch.bfloat16).to(dev)
+    Wu = torch.from_numpy(w.Wu).to(torch.bfloat16).to(dev)
+    nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty((max(16, sv.svconv_adapter_workspace_size(R, max_rows)),), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def index():
+        sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
+
+    def adapter():
+        sv.svconv_adapter_fwd(X, nbr, off, T, Wd, Wc, Wu, chunk_T=chunk_T, max_chunk_rows=max_rows,
+                              workspace=ws, status=status)
+
+    n_chunks = (T + chunk_T - 1) // chunk_T
+    launches_per_step = 1 + 3 * n_chunks  # index; per chunk: down GEMM, conv, up GEMM
+
+    def timed(fn, steps, warmup):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                fn()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            evs = []
+            for _ in range(steps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                evs.append((a, b))
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    def step():
+        index()
+        adapter()
+
+    with torch.cuda.stream(stream):
+        step()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            step()
+        g_ad = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_ad, stream=stream, capture_error_mode="relaxed"):
+            adapter()
+    torch.cuda.synchronize()
+    peak = torch.cuda.max_memory_allocated(dev)
+
+    with ClockSampler(local) as clk:
+        total_ms = timed(g.replay, args.steps, args.warmup)
+    clocks = clk.summary()
+    ad_ms = timed(g_ad.replay, args.steps, args.warmup) / args.steps
+    idx_ms = timed(index, args.steps, args.warmup) / args.steps
+
+    # end to end: the video's coordinates and features in from pinned host memory, the
+    # updated features back out
+    h_out = torch.empty_like(h_X).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (h_coords, h_off, h_X))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e():
+        coords.copy_(h_coords, non_blocking=True)
+        off.copy_(h_off, non_blocking=True)
+        X.copy_(h_X, non_blocking=True)
+        step()
+        h_out.copy_(X, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_ms = timed(e2e, e2e_steps, 3)
+    t = torch.tensor([total_ms, e2e_ms, ad_ms, idx_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, ad_ms, idx_ms = (float(v) for v in t)
+    torch.cuda.synchronize()
+    st = int(status.item())
+    err = sv.svconv_read_error_word()
+    if st or err:
+        raise SystemExit(f"device status {st} / library error word {err}: results invalid")
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        # whole frames are independent: the oracle runs the first `frames` frames
+        frames = 8
+        r1 = int(w.frame_off[frames])
+        t0 = time.perf_counter()
+        sub_n, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W,
+                                         want_map=False)
+        oracle.adapter_fwd(w.X[:r1], sub_n, 0, r1, w.Wd, w.Wc, w.Wu)
+        dt = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        oracle.build_index(w.coords, w.frame_off, T, w.H, w.W, want_map=True)
+        idx_cpu_ms = 1e3 * (time.perf_counter() - t1)
+        cpu = {"value": r1 / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
+               "sample": f"index build + adapter forward on the first {frames} of {T} frames ({r1} tokens); "
+                         f"single-threaded C, fp64; 1 core used of {os.cpu_count()}",
+               "index_build_full_ms": idx_cpu_ms}
+
+    if rank == 0:
+        peaks = load_peaks()
+        flops = 2 * n * (D * R + 9 * R * R + R * D)
+        ad_work = {"bytes": 2 * n * D * 2 + 36 * n + 2 * (2 * D * R + 9 * R * R), "flops": flops}
+        roof = roofline_entry("adapter_fwd", ad_work, ad_ms, peaks)
+        roof["kernel"] = f"adapter_fwd ({3 * n_chunks} tcgen05 GEMM launches, timed together)"
+        roof["traffic"] = None
+        roof["peak_source"] = peaks["source"]
+        idx_work = algorithmic_work(n, T, R, R)["build_index"]
+        tokens = n * world
+        line = {
+            "metric": METRIC, "value": tokens * args.steps / (total_ms * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "n_kept_per_gpu": n, "T": T, "H": w.H, "W": w.W, "D": D, "R": R,
+                       "chunk_T": chunk_T, "step": "build_index+adapter_fwd (in place)",
+                       "l2": "inputs larger than L2 (X read and written in place each step); no flush",
+                       "graph": "step replayed from a CUDA graph", "parallelism": f"dp{world}",
+                       "peak_device_bytes": peak},
+            "roofline": roof,
+            "kernels": {"adapter_fwd": dict(ms=ad_ms, **roofline_entry("adapter_fwd", ad_work, ad_ms, peaks)),
+                        "build_index": dict(ms=idx_ms, **roofline_entry("build_index", idx_work, idx_ms, peaks))},
+            "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        del g, g_ad
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,16 +680,16 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="small_c",
-                    help="small_c (default: the headline configuration), large_c_fwd, large_c_bwd")
+                    help="small_c (default: the headline configuration), large_c_fwd, large_c_bwd, adapter")
     args = ap.parse_args()
     global WORKLOAD
     WORKLOAD = args.workload
-    if args.workload == "adapter":
-        raise SystemExit("the adapter workload is timed by its own step; not wired yet")
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "adapter":
+        return run_adapter(args)
     return run_b200(args)
 
 
