@@ -227,6 +227,24 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, uint32_t issued, int 
   __syncwarp();
 }
 
+// A warp copies `count` neighbour-table entries (int32) from global src to shared dst and
+// accounts for them on `bar`, whose expected arrival count includes all 32 lanes plus one
+// expect_tx arrival by lane 0.  With bulk_ok (src 16-byte aligned) the 16-byte-aligned
+// prefix goes as one bulk copy on the TMA engine and at most 3 trailing entries by 4-byte
+// cp.async; otherwise every entry by 4-byte cp.async.  extra_tx: bytes of other TMA copies
+// that lane 0 issues on the same barrier phase (they are declared in the same arrival).
+__device__ __forceinline__ void copy_index_entries(uint32_t dst, const int32_t* src, int count, bool bulk_ok,
+                                                   uint64_t* bar, uint32_t extra_tx) {
+  const int lane = threadIdx.x & 31;
+  const int pre = bulk_ok ? (count & ~3) : 0;  // entries covered by the bulk copy (16-byte multiple)
+  for (int e = pre + lane; e < count; e += 32) cp_async_4(dst + 4u * e, src + e, 4u);
+  cp_async_arrive_noinc(bar);
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar, (uint32_t)pre * 4u + extra_tx);
+    if (pre > 0) bulk_copy_g2s(dst, src, (uint32_t)pre * 4u, bar);
+  }
+}
+
 // Writers of generic shared memory publish a stage to the async proxy (the MMA).
 __device__ __forceinline__ void warp_publish(uint64_t* bar) {
   fence_proxy_async_smem();
@@ -431,8 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int nbr_base = p.nbr_abs ? lo : 0;
 
   if (threadIdx.x == 0) {
-    // afull: one builder group per A stage; ifull: the 32 cp.async arrivals of the loader lanes
-    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 32, kProdWarps);
+    // afull: one builder group per A stage; ifull: the loader lanes' 32 cp.async arrivals + lane 0's expect_tx
+    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 33, kProdWarps);
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -463,13 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         }
         const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
         const int lim = min(M - m0, kBM) * 9;
-        const uint32_t dst = smem_u32(sm.idx + slot * kConvIdx);
-#pragma unroll
-        for (int i = 0; i < kConvIdx / 32; ++i) {
-          const int e = lane + 32 * i;
-          cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
-        }
-        cp_async_arrive_noinc(&bar->ifull[slot]);
+        copy_index_entries(smem_u32(sm.idx + slot * kConvIdx), src, lim,
+                           ((reinterpret_cast<uintptr_t>(src) & 15u) == 0), &bar->ifull[slot], 0u);
+        __syncwarp();
         ++ni;
         for (int cb = 0; cb < kb_per_tap; ++cb, ++hi) {
           const int hb = hi & 1;
@@ -728,15 +742,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
     const int m0 = tile * kBM;
     const int32_t* src = p.nbr + (size_t)m0 * 9;
     const int lim = min(M - m0, kBM) * 9;
-    const uint32_t dst = smem_u32(sidx + slot * kConvIdx);
-#pragma unroll
-    for (int i = 0; i < kConvIdx / 32; ++i) {
-      const int e = lane + 32 * i;
-      cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
-    }
-    cp_async_arrive_noinc(&bar->lfull[slot]);
+    copy_index_entries(smem_u32(sidx + slot * kConvIdx), src, lim, ((reinterpret_cast<uintptr_t>(src) & 15u) == 0),
+                       &bar->lfull[slot], kHaloBufBytes);
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bar->lfull[slot], kHaloBufBytes);
       const uint32_t hdst = smem_u32(shalo + slot * kHaloBufBytes);
 #pragma unroll
       for (int q = 0; q < kConvHaloRows / kHaloBox; ++q)
@@ -1021,15 +1029,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         const int k0 = kb * kBK;
         const int lim = min(p.n - k0, kBK) * 9;
         const int32_t* src = p.nbr + (size_t)k0 * 9;
-        const uint32_t dst = smem_u32(sm.idx + slot * kWgIdx);
-#pragma unroll
-        for (int i = 0; i < kWgIdx / 32; ++i) {
-          const int e = lane + 32 * i;
-          cp_async_4(dst + 4u * e, src + (e < lim ? e : 0), e < lim ? 4u : 0u);
-        }
-        cp_async_arrive_noinc(&bar->ifull[slot]);
+        copy_index_entries(smem_u32(sm.idx + slot * kWgIdx), src, lim, ((reinterpret_cast<uintptr_t>(src) & 15u) == 0),
+                           &bar->ifull[slot], kHaloBufBytes);
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bar->ifull[slot], kHaloBufBytes);
           const uint32_t hb = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
 #pragma unroll
           for (int b = 0; b < kWgHaloRows / kHaloBox; ++b)
