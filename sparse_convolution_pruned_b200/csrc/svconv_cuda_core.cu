@@ -113,18 +113,20 @@ __global__ void __launch_bounds__(256) f32_wgrad_partial_kernel(const float* __r
   }
 }
 
-// One thread per (dW row m = j * Cin + i, output channel o); 32 x 32 tiles so that
-// both the partial reads (along o) and the transposed dW writes (along m) are
-// coalesced.  The split sums are issued 8 loads at a time so they overlap.
+// One thread per (dW row m = j * Cin + i, output channel o); blocks of 8 rows x 32 output
+// channels (about one block per SM at the small-channel size), so that the partial reads
+// (along o) are coalesced and many are in flight; the transposed dW writes go through a
+// shared-memory tile.  The split sums are issued 16 loads at a time, summed in split order.
 // grouped = 0: partial row m (db at 9 Cin); grouped = 1 (tensor-core layout, Cin a
 // multiple of 64): partial row ((i / 64) * 10 + j) * 64 + i % 64, db at 9 * 64.
-__global__ void __launch_bounds__(1024) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
-                                                            int rows_pad, int Cin, int Cout, int grouped,
-                                                            float* __restrict__ dW, float* __restrict__ db) {
-  __shared__ float tile[32][33];
+constexpr int kRedRows = 8;
+__global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restrict__ partial, int splits,
+                                                           int rows_pad, int Cin, int Cout, int grouped,
+                                                           float* __restrict__ dW, float* __restrict__ db) {
+  __shared__ float tile[kRedRows][33];
   const int rows = 9 * Cin + 1;
-  const int m0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int m0 = blockIdx.x * kRedRows, o0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   {
     const int m = m0 + ty, o = o0 + tx;
     Dot2 s;
@@ -136,25 +138,27 @@ __global__ void __launch_bounds__(1024) wgrad_reduce_kernel(const float* __restr
       }
       const size_t stride = (size_t)rows_pad * Cout;
       const float* src = partial + (size_t)pm * Cout + o;
-      for (int sp0 = 0; sp0 < splits; sp0 += 8) {
-        float v[8];
+      for (int sp0 = 0; sp0 < splits; sp0 += 16) {
+        float v[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = (sp0 + q < splits) ? __ldg(src + (size_t)(sp0 + q) * stride) : 0.0f;
+        for (int q = 0; q < 16; ++q) v[q] = (sp0 + q < splits) ? __ldg(src + (size_t)(sp0 + q) * stride) : 0.0f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+        for (int q = 0; q < 16; ++q)
           if (sp0 + q < splits) s.add(v[q]);
       }
     }
     tile[ty][tx] = s.value();
   }
   __syncthreads();
+  // write: each warp takes 4 output channels, its lanes 8 consecutive rows of each
   {
-    const int o = o0 + ty, m = m0 + tx;
+    const int o = o0 + ty * 4 + (tx >> 3), r = tx & 7, m = m0 + r;
     if (o < Cout) {
+      const float v = tile[r][ty * 4 + (tx >> 3)];
       if (m < 9 * Cin)
-        dW[(size_t)o * 9 * Cin + m] = tile[tx][ty];
+        dW[(size_t)o * 9 * Cin + m] = v;
       else if (m == 9 * Cin && db)
-        db[o] = tile[tx][ty];
+        db[o] = v;
     }
   }
 }
@@ -197,8 +201,8 @@ cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int
 cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, int grouped,
                                 float* dW, float* db, cudaStream_t s) {
   const int rows = 9 * Cin + 1;
-  dim3 grid((rows + 31) / 32, (Cout + 31) / 32);
-  wgrad_reduce_kernel<<<grid, dim3(32, 32), 0, s>>>(partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
+  dim3 grid((rows + kRedRows - 1) / kRedRows, (Cout + 31) / 32);
+  wgrad_reduce_kernel<<<grid, 256, 0, s>>>(partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
   return cudaGetLastError();
 }
 

@@ -316,34 +316,57 @@ __device__ __forceinline__ MmaIssuer make_issuer(const Carve& sm, uint32_t b_sta
 
 // One thread issues the MMAs of one tile (num_kb K-blocks) into accumulator d.
 // A_TMEM: A stages in tensor memory (written by the builder warps with tcgen05.st).
-template <bool A_TMEM>
+// GROUP: stages whose barriers are checked back to back before their MMAs are issued.
+// The first shared-memory access (an mbarrier wait) after a batch of MMAs stalls until
+// those MMAs have read their operands, so checking two stages per batch halves that cost
+// when MMAs are short (N = 64); GROUP = 1 keeps the deepest pipelining for long MMAs.
+template <bool A_TMEM, int GROUP>
 __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                          volatile int* abort_flag, int* err, uint64_t timeout_ns) {
-  for (int kb = 0; kb < num_kb; ++kb) {
-    if (!mbar_wait(&bar->afull[m.sa], m.pa, abort_flag, err, timeout_ns)) return false;
-    if (!mbar_wait(&bar->bfull[m.sb], m.pb, abort_flag, err, timeout_ns)) return false;
-    const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sb * m.b_stage16);
-    if constexpr (A_TMEM) {
-      tc_fence_after();  // the A stage was written to tensor memory by other threads
-      const uint32_t at = m.a_tmem0 + (uint32_t)m.sa * kTmemAStageCols;
+  for (int kb = 0; kb < num_kb; kb += GROUP) {
+    const int cnt = min(GROUP, num_kb - kb);
+    int sa[GROUP], sb[GROUP];
+    {
+      int a = m.sa, b = m.sb;
+      uint32_t pa = m.pa, pb = m.pb;
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k)
-        tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
-    } else {
-      const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
+      for (int g = 0; g < GROUP; ++g) {
+        if (g < cnt) {
+          if (!mbar_wait(&bar->afull[a], pa, abort_flag, err, timeout_ns)) return false;
+          if (!mbar_wait(&bar->bfull[b], pb, abort_flag, err, timeout_ns)) return false;
+        }
+        sa[g] = a;
+        sb[g] = b;
+        if (++a == m.SA) a = 0, pa ^= 1u;
+        if (++b == m.SB) b = 0, pb ^= 1u;
+      }
+    }
+    if constexpr (A_TMEM) tc_fence_after();  // the A stages were written to tensor memory by other threads
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k)
-        tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb | k) != 0 ? 1u : 0u);
-    }
-    tc_commit(&bar->aempty[m.sa]);
-    tc_commit(&bar->bempty[m.sb]);
-    if (++m.sa == m.SA) {
-      m.sa = 0;
-      m.pa ^= 1u;
-    }
-    if (++m.sb == m.SB) {
-      m.sb = 0;
-      m.pb ^= 1u;
+    for (int g = 0; g < GROUP; ++g) {
+      if (g >= cnt) break;
+      const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)sb[g] * m.b_stage16);
+      if constexpr (A_TMEM) {
+        const uint32_t at = m.a_tmem0 + (uint32_t)sa[g] * kTmemAStageCols;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+      } else {
+        const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)sa[g] * m.a_stage16);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+      }
+      tc_commit(&bar->aempty[sa[g]]);
+      tc_commit(&bar->bempty[sb[g]]);
+      if (++m.sa == m.SA) {
+        m.sa = 0;
+        m.pa ^= 1u;
+      }
+      if (++m.sb == m.SB) {
+        m.sb = 0;
+        m.pb ^= 1u;
+      }
     }
   }
   return true;
@@ -659,8 +682,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, n_acc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        const bool ok = gather ? mma_tile<true>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)
-                               : mma_tile<false>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        constexpr int kGroup = BN == 256 ? 1 : 2;
+        const bool ok =
+            gather ? mma_tile<true, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)
+                   : mma_tile<false, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
         if (!ok) break;
         tc_commit(&bar->tfull[ab]);
       }
@@ -1189,7 +1214,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, kAcc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile<true>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
+        if (!mma_tile<true, 2>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
         tc_commit(&bar->tfull[ab]);
       }
       mma_drain(bar, issued, err, p.timeout_ns);
