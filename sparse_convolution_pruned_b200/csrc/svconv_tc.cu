@@ -399,8 +399,17 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
 #pragma unroll
       for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[hh][q]);
       if (p.bias) {
+        if ((reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0) {  // n0 + c is a multiple of 32
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + c);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c + q);
+          for (int q = 0; q < 8; ++q) {
+            const float4 b = __ldg(b4 + q);
+            f[4 * q] += b.x, f[4 * q + 1] += b.y, f[4 * q + 2] += b.z, f[4 * q + 3] += b.w;
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c + q);
+        }
       }
       if (p.gelu) {
 #pragma unroll
