@@ -997,6 +997,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
 // exactly the (channel lane, token-pair column) order of tcgen05.st.16x128b, so A
 // is transposed and gathered on the way in, with no shared-memory stores.  B is
 // dY by TMA (MN-major).
+// Weight-gradient builder, rare path (kept out of line so the builders' loop stays small):
+// the 16 registers of a 16-channel piece hold zeros for entries outside the halo window;
+// fetch those elements from global memory.
+struct Regs16 {
+  uint32_t v[16];
+};
+__device__ __noinline__ Regs16 wgrad_patch_far(Regs16 R, uint32_t sidx_s, const uint16_t* X16, int n, int Cin, int k0,
+                                               int hlo, int j, int ch0) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int k4 = r >> 2, m = r & 3;
+    const int ch = ch0 + 8 * (m & 1) + (lane >> 2);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int tk = 16 * k4 + 8 * (m >> 1) + 2 * (lane & 3) + e;
+      const int x = k0 + tk < n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
+      if (x >= 0 && x < n && (unsigned)(x - hlo) >= (unsigned)kWgHaloRows) {
+        const uint32_t v = __ldg(X16 + (size_t)x * Cin + ch);
+        R.v[r] = e == 0 ? ((R.v[r] & 0xFFFF0000u) | v) : ((R.v[r] & 0x0000FFFFu) | (v << 16));
+      }
+    }
+  }
+  return R;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_constant__ TcWgradParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -1164,20 +1190,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
             }
             if (__any_sync(0xffffffffu, far)) {
               // entries outside the halo window read as zero above: fetch them from global memory
+              Regs16 rr;
 #pragma unroll
-              for (int r = 0; r < 16; ++r) {
-                const int k4 = r >> 2, m = r & 3;
-                const int ch = cb * kBK + c16 + 8 * (m & 1) + (lane >> 2);
+              for (int r = 0; r < 16; ++r) rr.v[r] = R[r];
+              rr = wgrad_patch_far(rr, sidx_s, X16, p.n, p.Cin, k0, hlo, j, cb * kBK + c16);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int tk = 16 * k4 + 8 * (m >> 1) + 2 * (lane & 3) + e;
-                  const int x = k0 + tk < p.n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
-                  if (x >= 0 && x < p.n && (unsigned)(x - hlo) >= (unsigned)kWgHaloRows) {
-                    const uint32_t v = __ldg(X16 + (size_t)x * p.Cin + ch);
-                    R[r] = e == 0 ? ((R[r] & 0xFFFF0000u) | v) : ((R[r] & 0x0000FFFFu) | (v << 16));
-                  }
-                }
-              }
+              for (int r = 0; r < 16; ++r) R[r] = rr.v[r];
             }
             tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
           }
