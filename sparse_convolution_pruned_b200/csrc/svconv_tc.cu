@@ -1168,26 +1168,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
           for (int sub = 0; sub < 2; ++sub) {
             const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
             uint32_t R[16];
-            bool far = false;
+            bool far = false, bad = false;
+            const int chunk = (c16 >> 3) + (mi & 1);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
+              // branch-free: entries of tokens past n (stale slot contents) count as missing
               const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
-              int x = k0 + tk < p.n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
-              if (x >= p.n) {
-                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-                x = -1;
-              }
+              const int raw = ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j));
+              const bool tok_ok = k0 + tk < p.n;
+              bad |= tok_ok & (raw >= p.n);
+              const int x = (tok_ok & (raw < p.n)) ? raw : -1;
               const int h = x - hlo;
-              const int chunk = (c16 >> 3) + (mi & 1);
-              uint32_t addr = zero_addr;
-              if (x >= 0) {
-                if ((unsigned)h < (unsigned)kWgHaloRows)
-                  addr = halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4);
-                else
-                  far = true;
-              }
+              const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kWgHaloRows);
+              far |= (x >= 0) & !in_win;
+              const uint32_t addr =
+                  in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_addr;
               ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
             }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
             if (__any_sync(0xffffffffu, far)) {
               // entries outside the halo window read as zero above: fetch them from global memory
               Regs16 rr;
