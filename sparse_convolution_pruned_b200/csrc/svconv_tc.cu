@@ -76,7 +76,7 @@ constexpr int kTmemAStages = 4;                    // gather conv: A stages held
 constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
 struct __align__(16) TcBarriers {
-  uint32_t zero16[4];                              // 16 zero bytes (row source for missing neighbours)
+  uint32_t zero16[32];                             // 128 zero bytes (row source for missing neighbours)
   uint64_t afull[kMaxStages], aempty[kMaxStages];  // A stages
   uint64_t bfull[kMaxStages], bempty[kMaxStages];  // B stages
   uint64_t ifull[kMaxStages], iempty[kMaxStages];  // neighbour-row slots (and their halos, weight gradient)
@@ -179,7 +179,7 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
 // nslots neighbour-row slots with the given arrival counts; everything else fixed.
 __device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uint32_t afull_count, int nslots,
                                               uint32_t ifull_count, uint32_t iempty_count) {
-  for (int i = 0; i < 4; ++i) b->zero16[i] = 0u;
+  for (int i = 0; i < 32; ++i) b->zero16[i] = 0u;
   for (int i = 0; i < nslots; ++i) {
     mbar_init(&b->ifull[i], ifull_count);
     mbar_init(&b->iempty[i], iempty_count);
@@ -602,6 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       const int quarter = warp & 3;             // TMEM lane quarter of this warp
       const int r = quarter * 32 + lane;        // the tile row this thread writes
       const uint32_t a_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + a_tmem_col;
+      const uint32_t zero_row = smem_u32(bar->zero16);
       uint32_t ti = 0, hi = 0, it = 0;
       bool aborted = false;
       for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
@@ -630,33 +631,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
               break;
             }
             tc_fence_after();  // the MMAs that read this stage are complete
-            int idx = row_ok ? ld_shared_s32(sidx_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
-            if (idx >= 0) {
-              idx -= nbr_base;
-              if ((unsigned)idx >= (unsigned)p.a_rows) {
-                atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-                idx = -1;
-              }
-            }
+            // branch-free row selection: halo row, or the zero row for a missing neighbour;
+            // rows outside the halo window are read from global memory behind a warp vote
+            const int raw = row_ok ? ld_shared_s32(sidx_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
+            const int rel = raw - nbr_base;
+            const bool bad = (raw >= 0) & ((unsigned)rel >= (unsigned)p.a_rows);
+            const int idx = ((raw >= 0) & !bad) ? rel : -1;
             const int h = idx - hlo;
+            const bool in_win = (idx >= 0) & ((unsigned)h < (unsigned)kConvHaloRows);
+            const uint32_t row = in_win ? halo + (uint32_t)h * 128u : zero_row;
+            const int sw = in_win ? (h & 7) : 0;
             uint32_t v[32];
-            if (idx >= 0 && (unsigned)h < (unsigned)kConvHaloRows) {
-              const uint32_t row = halo + h * 128;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint4 q = ld_shared_16(row + ((c ^ (h & 7)) << 4));
-                v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+            for (int c = 0; c < 8; ++c) {
+              const uint4 q = ld_shared_16(row + ((c ^ sw) << 4));
+              v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+            }
+            const bool far = (idx >= 0) & !in_win;
+            if (__any_sync(0xffffffffu, far | bad)) {
+              if (bad) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+              if (far) {
+                const __nv_bfloat16* src = p.A + (size_t)idx * p.lda + cb * kBK;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const uint4 q = ldg_16(src + c * 8);
+                  v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+                }
               }
-            } else if (idx >= 0) {
-              const __nv_bfloat16* src = p.A + (size_t)idx * p.lda + cb * kBK;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint4 q = ldg_16(src + c * 8);
-                v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
-              }
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c) v[c] = 0u;
             }
             tmem_st_32x32b_x32(a_lane + (uint32_t)sa * kTmemAStageCols, v);
             tmem_st_wait();
@@ -744,6 +745,7 @@ constexpr uint32_t kSmallTmemCols = 512;          // 128 + 9 * 32 = 416 columns 
 constexpr uint32_t kSmallWBytes = 9 * 64 * 64 * 2;
 
 struct __align__(16) SmallBars {
+  uint32_t zero128[32];          // 128 zero bytes (row source for missing neighbours)
   uint64_t wfull;
   uint64_t lfull[2], lempty[2];  // index entries + halo window of a tile
   uint64_t afull[2], aempty[2];  // per builder group
@@ -818,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
     }
     __syncwarp();
   } else if (threadIdx.x == 0) {
+    for (int i = 0; i < 32; ++i) bar->zero128[i] = 0u;
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bar->afull[g], kProdWarps / 2);
       mbar_init(&bar->aempty[g], 1);
@@ -868,6 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
     const int r = quarter * 32 + lane;
     const int j0 = grp ? kSmallTaps0 : 0, j1 = grp ? 9 : kSmallTaps0;
     const uint32_t a_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + kSmallACol;
+    const uint32_t zero_row = smem_u32(bar->zero128);
     uint32_t ti = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
       const int slot = ti & 1;
@@ -882,30 +886,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
       const uint32_t si_s = smem_u32(sidx + slot * kConvIdx);
       for (int j = j0; j < j1; ++j) {
         const int jj = MIRROR ? 8 - j : j;
-        int idx = row_ok ? ld_shared_s32(si_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
-        if (idx >= 0 && (unsigned)idx >= (unsigned)p.a_rows) {
-          atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-          idx = -1;
-        }
+        // branch-free row selection (see the general kernel's builders)
+        const int raw = row_ok ? ld_shared_s32(si_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
+        const bool bad = (raw >= 0) & ((unsigned)raw >= (unsigned)p.a_rows);
+        const int idx = bad ? -1 : raw;
         const int h = idx - hlo;
+        const bool in_win = (idx >= 0) & ((unsigned)h < (unsigned)kConvHaloRows);
+        const uint32_t row = in_win ? halo + (uint32_t)h * 128u : zero_row;
+        const int sw = in_win ? (h & 7) : 0;
         uint32_t v[32];
-        if (idx >= 0 && (unsigned)h < (unsigned)kConvHaloRows) {
-          const uint32_t row = halo + h * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 q = ld_shared_16(row + ((c ^ (h & 7)) << 4));
-            v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+        for (int c = 0; c < 8; ++c) {
+          const uint4 q = ld_shared_16(row + ((c ^ sw) << 4));
+          v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+        }
+        const bool far = (idx >= 0) & !in_win;
+        if (__any_sync(0xffffffffu, far | bad)) {
+          if (bad) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+          if (far) {
+            const __nv_bfloat16* src = p.A + (size_t)idx * p.lda;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 q = ldg_16(src + c * 8);
+              v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
+            }
           }
-        } else if (idx >= 0) {
-          const __nv_bfloat16* src = p.A + (size_t)idx * p.lda;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 q = ldg_16(src + c * 8);
-            v[4 * c] = q.x, v[4 * c + 1] = q.y, v[4 * c + 2] = q.z, v[4 * c + 3] = q.w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) v[c] = 0u;
         }
         tmem_st_32x32b_x32(a_lane + (uint32_t)j * kTmemAStageCols, v);
       }
