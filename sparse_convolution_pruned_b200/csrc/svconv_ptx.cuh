@@ -119,6 +119,13 @@ __device__ __forceinline__ uint4 ld_shared_16(uint32_t src) {
   return v;
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t dst, uint4 v) { st_shared_16(dst, v.x, v.y, v.z, v.w); }
+
+// 32-byte global store (sm_100); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_32(void* dst, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 __device__ __forceinline__ int ld_shared_s32(uint32_t src) {
   int v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(src) : "memory");

@@ -429,14 +429,20 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
           }
         }
       }
-      uint4* op = reinterpret_cast<uint4*>(p.out + orow * p.ldo + n0 + c);
+      uint32_t packed[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 u;
-        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+      for (int q = 0; q < 16; ++q) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * q], f[2 * q + 1]);
+        packed[q] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      __nv_bfloat16* orow_p = p.out + orow * p.ldo + n0 + c;
+      if ((reinterpret_cast<uintptr_t>(orow_p) & 31u) == 0) {  // two 32-byte stores per 32 columns
+        st_global_32(orow_p, packed);
+        st_global_32(orow_p + 16, packed + 8);
+      } else {
+        uint4* op = reinterpret_cast<uint4*>(orow_p);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(f[q * 8 + 2 * e], f[q * 8 + 2 * e + 1]);
-        op[q] = u;
+        for (int q = 0; q < 4; ++q) op[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
       }
     }
   }
