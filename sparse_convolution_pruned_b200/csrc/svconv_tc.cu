@@ -714,12 +714,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     const int out_base = p.out_abs ? lo : 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
       const uint32_t ab = tc % (uint32_t)n_acc;
-      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, n_acc), abort_flag, err, p.timeout_ns)) break;
-      tc_fence_after();
       const int m0 = (tile / n_tiles) * kBM;
       const int n0 = (tile % n_tiles) * BN;
       const int row = m0 + warp * 32 + lane;
       const int orow_i = out_base + row;
+      if (p.residual && row < M && orow_i >= 0 && orow_i < p.out_rows) {
+        // bring this row's residual segment toward L2 while the tile's MMAs run
+        const char* rp = reinterpret_cast<const char*>(p.residual + (size_t)orow_i * p.ldo + n0);
+#pragma unroll
+        for (int b = 0; b < BN * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(rp + b));
+      }
+      if (!warp_wait(&bar->tfull[ab], ring_parity(tc, n_acc), abort_flag, err, p.timeout_ns)) break;
+      tc_fence_after();
       const bool valid = row < M && orow_i >= 0 && orow_i < p.out_rows;
       epilogue_rows<BN>(p, tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN, valid, (size_t)orow_i, n0);
       tc_fence_before();
