@@ -270,6 +270,7 @@ def run_b200(args):
     import torch.distributed as dist
 
     from sparse_convolution_pruned_b200 import svconv as sv
+    from sparse_convolution_pruned_b200.data_parallel import allreduce_grads
 
     rank, local, world = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
@@ -325,7 +326,7 @@ def run_b200(args):
     def one_step():
         g.replay()
         if world > 1:
-            dist.all_reduce(grads)
+            allreduce_grads(grads)
 
     def timed_loop(fn, steps, warmup, flush_l2=True):
         with torch.cuda.stream(stream):
@@ -411,7 +412,7 @@ def run_b200(args):
         dY.copy_(h_dY, non_blocking=True)
         step_kernels()
         if world > 1:
-            dist.all_reduce(grads)
+            allreduce_grads(grads)
         h_Y.copy_(Y, non_blocking=True)
         h_dX.copy_(dX, non_blocking=True)
         h_grads.copy_(grads, non_blocking=True)
