@@ -141,13 +141,37 @@ SVCONV_API size_t svconv_bwd_weight_workspace_size(int dtype, int n, int Cin, in
  *   - All calls share the array: calls that overlap on the GPU race.  Serialise them.
  *   - If the usual number of token splits does not fit, fewer are used (a different
  *     summation order, same tolerance); if one split's partials
- *     ((9*Cin+1 rounded up to 128) * Cout floats for bf16) exceed the array, it
- *     returns SVCONV_ERR_SIZE.
+ *     (640 * Cin / 64 rows of Cout floats for bf16, 9 * Cin + 1 rows for fp32)
+ *     exceed the array, it returns SVCONV_ERR_SIZE.
  *   - It calls no cudaMalloc / cudaFree and no allocating library routine.
  */
 #define SVCONV_NOALLOC_SCRATCH_BYTES (16u << 20)
 SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin,
                                          int Cout, float* dW, float* db, void* stream);
+
+/*
+ * Fused backward: the data gradient of svconv_bwd_data and the weight / bias
+ * gradients of svconv_bwd_weight in one call (SV-TAD page, Key Design 2: the
+ * dedicated backward kernels; both are the adjoints of the forward).
+ *   Arguments as in those two calls; dX [n][Cin] of dtype, dW [Cout][9][Cin] and
+ *   db [Cout] fp32 (db may be NULL) are overwritten.
+ *   workspace: device, at least svconv_bwd_workspace_size(...) bytes, 16-byte
+ *   aligned, no initial contents required.
+ *   bf16 with C_in = C_out = 64: the two gradients run side by side on disjoint
+ *   groups of SMs, the weight gradient on a side stream of the library that is
+ *   forked from and joined back to `stream` with events, so the call stays ordered
+ *   on `stream` and can be captured in a CUDA graph.  The first such call on a
+ *   device creates that stream and its two events: make it outside stream capture.
+ *   Calls from several host threads are serialised inside the library.  dX is
+ *   bitwise identical to svconv_bwd_data's; dW / db use fewer token splits than
+ *   svconv_bwd_weight (another fixed summation order: deterministic, same
+ *   tolerance).  Other shapes and fp32 run the two calls in order on `stream`.
+ *   Errors: as the two calls; SVCONV_ERR_CUDA if the side stream cannot be created.
+ */
+SVCONV_API int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
+                          const void* Wt, void* dX, float* dW, float* db, void* workspace, size_t ws_bytes,
+                          void* stream);
+SVCONV_API size_t svconv_bwd_workspace_size(int dtype, int n, int Cin, int Cout);
 
 /*
  * Chunked bottleneck adapter forward (Key Design 2, "chunked execution" that

@@ -74,6 +74,45 @@ static int conv_bn(int N) { return N % 256 == 0 ? 256 : N % 128 == 0 ? 128 : 64;
 
 using namespace svc;
 
+namespace svc {
+int tc_bwd_data(const void* dY, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt, void* dX, int max_ctas,
+                cudaStream_t s) {
+  TcConvArgs a{};
+  a.A = dY;
+  a.lda = Cout;
+  a.a_rows = n;
+  a.nbr = nbr;
+  a.taps = 9;
+  a.mirror = 1;
+  a.Kc = Cout;
+  a.b_mn_major = 1;
+  a.M = n;
+  a.N = Cin;
+  a.out = dX;
+  a.ldo = Cin;
+  a.out_rows = n;
+  a.max_ctas = max_ctas;
+  return cuda_rc(launch_tc_conv(a, Wt, 0, 0, conv_bn(Cin), s));
+}
+
+int tc_bwd_weight(const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout, float* dW, float* db,
+                  float* partial, int ctas, cudaStream_t s) {
+  TcWgradArgs a{};
+  a.dY = dY;
+  a.X = X;
+  a.nbr = nbr;
+  a.n = n;
+  a.Cin = Cin;
+  a.Cout = Cout;
+  a.partial = partial;
+  int bn;
+  tc_wgrad_plan_ctas(n, Cin, Cout, ctas > 0 ? ctas : sm_count(), &a.splits, &a.rows_pad, &bn);
+  cudaError_t e = launch_tc_wgrad_with_splits(a, s);
+  if (e != cudaSuccess) return SVCONV_ERR_CUDA;
+  return cuda_rc(launch_wgrad_reduce(partial, a.splits, a.rows_pad, Cin, Cout, 1, dW, db, s));
+}
+}  // namespace svc
+
 extern "C" {
 
 int svconv_version(void) { return 100; }
@@ -158,22 +197,10 @@ int svconv_bwd_data(int dtype, const void* dY, const int32_t* nbr, int n, int Ci
   if (dtype != SVCONV_BF16) return SVCONV_ERR_UNSUPPORTED;
   if (!bf16_channels_ok(Cin) || !bf16_channels_ok(Cout)) return SVCONV_ERR_UNSUPPORTED;
   if (!aligned16(dY) || !aligned16(Wt) || !aligned16(dX)) return SVCONV_ERR_ALIGN;
-  TcConvArgs a{};
-  a.A = dY;
-  a.lda = Cout;
-  a.a_rows = n;
-  a.nbr = nbr;
-  a.taps = 9;
-  a.mirror = 1;
-  a.Kc = Cout;
-  a.b_mn_major = 1;
-  a.M = n;
-  a.N = Cin;
-  a.out = dX;
-  a.ldo = Cin;
-  a.out_rows = n;
-  return cuda_rc(launch_tc_conv(a, Wt, 0, 0, conv_bn(Cin), s));
+  return tc_bwd_data(dY, nbr, n, Cin, Cout, Wt, dX, 0, s);
 }
+
+
 
 size_t svconv_bwd_weight_workspace_size(int dtype, int n, int Cin, int Cout) {
   if (n <= 0 || Cin <= 0 || Cout <= 0) return 0;
@@ -219,19 +246,7 @@ int svconv_bwd_weight(int dtype, const void* dY, const void* X, const int32_t* n
     return cuda_rc(launch_wgrad_reduce(partial, splits, rows, Cin, Cout, 0, dW, db, s));
   }
   if (!aligned16(dY) || !aligned16(X)) return SVCONV_ERR_ALIGN;
-  TcWgradArgs a{};
-  a.dY = dY;
-  a.X = X;
-  a.nbr = nbr;
-  a.n = n;
-  a.Cin = Cin;
-  a.Cout = Cout;
-  a.partial = partial;
-  int bn;
-  tc_wgrad_plan(n, Cin, Cout, &a.splits, &a.rows_pad, &bn);
-  cudaError_t e = launch_tc_wgrad(a, s);
-  if (e != cudaSuccess) return SVCONV_ERR_CUDA;
-  return cuda_rc(launch_wgrad_reduce(partial, a.splits, a.rows_pad, Cin, Cout, 1, dW, db, s));
+  return tc_bwd_weight(dY, X, nbr, n, Cin, Cout, dW, db, partial, 0, s);
 }
 
 size_t svconv_adapter_workspace_size(int R, int max_chunk_rows) {

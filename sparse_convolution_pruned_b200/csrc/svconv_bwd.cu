@@ -1,0 +1,114 @@
+// Fused backward entry point (svconv_bwd): the data gradient and the weight / bias
+// gradients of one SparseConv2D in a single call (SV-TAD page, Key Design 2: dedicated
+// backward kernels; the formulas are the adjoints of the forward).
+//
+// Both gradients read the same dY and neighbour table and do not depend on each other.
+// At 64 input and output channels both kernels are latency-bound (each CTA waits ~3 us
+// for its first operands and carries one or two tiles), so running them side by side on
+// disjoint groups of SMs finishes sooner than running them one after the other: the data
+// gradient takes about 3/8 of the SMs on the caller's stream, the weight gradient and its
+// split reduce the rest on a side stream owned by the library, joined back to the caller's
+// stream with events.  Other shapes, and fp32, run the two entry points in order on the
+// caller's stream.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "svconv.h"
+#include "svconv_internal.h"
+
+namespace svc {
+namespace {
+
+constexpr int kMaxDev = 64;
+
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[kMaxDev];
+std::mutex g_side_mu;  // guards creation and each call's fork / launch / join sequence
+
+bool concurrent_shape(int dtype, int Cin, int Cout) { return dtype == SVCONV_BF16 && Cin == 64 && Cout == 64; }
+
+// CTA budgets: weight gradient 94 of 148 SMs, data gradient the rest (measured best split).
+void budgets(int* data_ctas, int* weight_ctas) {
+  const int sms = sm_count();
+  int w = sms * 94 / 148;
+  if (w < 5) w = 5;
+  int d = sms - w;
+  if (d < 1) d = 1;
+  *data_ctas = d;
+  *weight_ctas = w;
+}
+
+// Side stream and events of the current device, created on first use (call with g_side_mu held).
+SideStream* side_stream() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDev) return nullptr;
+  SideStream& r = g_side[d];
+  if (!r.stream) {
+    if (cudaStreamCreateWithFlags(&r.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(r.stream);
+      r.stream = nullptr;
+      return nullptr;
+    }
+  }
+  return &r;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace svc
+
+using namespace svc;
+
+extern "C" {
+
+size_t svconv_bwd_workspace_size(int dtype, int n, int Cin, int Cout) {
+  if (!concurrent_shape(dtype, Cin, Cout) || n <= 0) return svconv_bwd_weight_workspace_size(dtype, n, Cin, Cout);
+  int dc, wc, splits, rows_pad, bn;
+  budgets(&dc, &wc);
+  tc_wgrad_plan_ctas(n, Cin, Cout, wc, &splits, &rows_pad, &bn);
+  return (size_t)splits * rows_pad * Cout * sizeof(float);
+}
+
+int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
+               const void* Wt, void* dX, float* dW, float* db, void* workspace, size_t ws_bytes, void* stream) {
+  if (n < 0 || Cin <= 0 || Cout <= 0) return SVCONV_ERR_SIZE;
+  if (!concurrent_shape(dtype, Cin, Cout) || n == 0) {
+    const int rc = svconv_bwd_data(dtype, dY, nbr, n, Cin, Cout, Wt, dX, stream);
+    if (rc) return rc;
+    return svconv_bwd_weight(dtype, dY, X, nbr, n, Cin, Cout, dW, db, workspace, ws_bytes, stream);
+  }
+  if (!dY || !X || !nbr || !Wt || !dX || !dW) return SVCONV_ERR_NULL;
+  int major = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return SVCONV_ERR_CUDA;
+  if (major != 10) return SVCONV_ERR_DEVICE;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(Wt) || !aligned16(dX)) return SVCONV_ERR_ALIGN;
+  if (!workspace || ws_bytes < svconv_bwd_workspace_size(dtype, n, Cin, Cout)) return SVCONV_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SVCONV_ERR_ALIGN;
+  int dc, wc;
+  budgets(&dc, &wc);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  SideStream* side = side_stream();
+  if (!side) return SVCONV_ERR_CUDA;
+  // fork: the side stream waits for everything before this call on the caller's stream
+  if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+    return SVCONV_ERR_CUDA;
+  const int rc_data = tc_bwd_data(dY, nbr, n, Cin, Cout, Wt, dX, dc, s);
+  const int rc_weight = tc_bwd_weight(dY, X, nbr, n, Cin, Cout, dW, db, static_cast<float*>(workspace), wc,
+                                      side->stream);
+  // join: the caller's stream waits for the side stream's work (also after a failed launch)
+  if (cudaEventRecord(side->join, side->stream) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess)
+    return SVCONV_ERR_CUDA;
+  return rc_data ? rc_data : rc_weight;
+}
+
+}  // extern "C"

@@ -71,6 +71,7 @@ struct TcConvArgs {
   int ldo;
   int out_rows;           // rows of out / residual (range check of absolute output rows)
   int32_t* status;        // caller status word or nullptr (library word used otherwise)
+  int max_ctas;           // CTA budget (0: one per SM)
 };
 cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s);
 
@@ -83,8 +84,17 @@ struct TcWgradArgs {
   int splits, rows_pad;
 };
 void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn);
+// the same plan for a budget of `ctas` CTAs (launch with launch_tc_wgrad_with_splits)
+void tc_wgrad_plan_ctas(int n, int Cin, int Cout, int ctas, int* splits, int* rows_pad, int* bn);
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s);
 cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s);
+
+// bf16 tensor-core bodies of the data / weight gradients (arguments already validated);
+// max_ctas / ctas: CTA budget (0: all SMs).  Return SVCONV_* codes.
+int tc_bwd_data(const void* dY, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt, void* dX, int max_ctas,
+                cudaStream_t s);
+int tc_bwd_weight(const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout, float* dW, float* db,
+                  float* partial, int ctas, cudaStream_t s);
 
 // failure-detection self test
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s);

@@ -1454,6 +1454,7 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / bn);
   if (tiles == 0) return cudaSuccess;
   int grid = sm_count();
+  if (a.max_ctas > 0 && grid > a.max_ctas) grid = a.max_ctas;
   if (grid > tiles) grid = tiles;
   // 64 gathered channels and 64 output columns, whole-table rows: W-resident small-channel kernel
   if (a.nbr && a.Kc == 64 && a.N == 64 && bn == 64 && !a.row_lo && !a.a_abs && !a.nbr_abs && !a.out_abs)
@@ -1467,11 +1468,15 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
 static int wgrad_bn(int Cout) { return Cout % 256 == 0 ? 256 : Cout % 128 == 0 ? 128 : 64; }
 
 void tc_wgrad_plan(int n, int Cin, int Cout, int* splits, int* rows_pad, int* bn) {
+  tc_wgrad_plan_ctas(n, Cin, Cout, sm_count(), splits, rows_pad, bn);
+}
+
+void tc_wgrad_plan_ctas(int n, int Cin, int Cout, int ctas, int* splits, int* rows_pad, int* bn) {
   const int b = wgrad_bn(Cout);
   const int rp = (Cin / kBK) * kWgTiles * kBM;  // 10 half-tiles of 64 rows per 64-channel block
   const int base_units = (rp / kBM) * (Cout / b);
   const int kbt = (n + kBK - 1) / kBK;
-  int sp = sm_count() / base_units;
+  int sp = ctas / base_units;
   if (sp < 1) sp = 1;
   if (sp > kbt) sp = kbt > 0 ? kbt : 1;
   *splits = sp;

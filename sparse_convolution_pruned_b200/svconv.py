@@ -48,6 +48,10 @@ def lib() -> ctypes.CDLL:
         L.svconv_fwd.argtypes = [I, P, P, I, I, I, P, P, P, P]
         L.svconv_bwd_data.argtypes = [I, P, P, I, I, I, P, P, P]
         L.svconv_bwd_weight.argtypes = [I, P, P, P, I, I, I, P, P, P, Z, P]
+        L.svconv_bwd.argtypes = [I, P, P, P, I, I, I, P, P, P, P, P, Z, P]
+        L.svconv_bwd.restype = I
+        L.svconv_bwd_workspace_size.argtypes = [I, I, I, I]
+        L.svconv_bwd_workspace_size.restype = Z
         L.svconv_bwd_weight_noalloc.argtypes = [I, P, P, P, I, I, I, P, P, P]
         L.svconv_bwd_weight_noalloc.restype = I
         L.svconv_bwd_weight_workspace_size.argtypes = [I, I, I, I]
@@ -209,6 +213,33 @@ def svconv_bwd_weight_noalloc(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tens
                                          _ptr(db), _stream(X, stream))
     _check("svconv_bwd_weight_noalloc", rc)
     return dW, db
+
+
+def svconv_bwd_workspace_size(dtype: int, n: int, Cin: int, Cout: int) -> int:
+    return int(lib().svconv_bwd_workspace_size(int(dtype), int(n), int(Cin), int(Cout)))
+
+
+def svconv_bwd(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tensor, Wt: torch.Tensor, *,
+               dX: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None, db: Optional[torch.Tensor] = None,
+               want_db: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """(dX, dW, db): the data gradient and the weight / bias gradients in one call."""
+    _cuda(dY, X, nbr, Wt, dX, dW, db, workspace)
+    n, Cout = dY.shape
+    Cin = X.shape[1]
+    dt = _dtype_code(X)
+    if dX is None:
+        dX = torch.empty((n, Cin), dtype=dY.dtype, device=dY.device)
+    if dW is None:
+        dW = torch.empty((Cout, 9, Cin), dtype=torch.float32, device=X.device)
+    if db is None and want_db:
+        db = torch.empty((Cout,), dtype=torch.float32, device=X.device)
+    need = svconv_bwd_workspace_size(dt, n, Cin, Cout)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=X.device)
+    rc = lib().svconv_bwd(dt, _ptr(dY), _ptr(X), _ptr(nbr), n, Cin, Cout, _ptr(Wt), _ptr(dX), _ptr(dW), _ptr(db),
+                          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(X, stream))
+    _check("svconv_bwd", rc)
+    return dX, dW, db
 
 
 def svconv_adapter_workspace_size(R: int, max_chunk_rows: int) -> int:

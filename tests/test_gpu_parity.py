@@ -208,6 +208,58 @@ def test_bf16_full_size_sampled(sv, orc, make):
     assert sv.svconv_read_error_word() == 0
 
 
+FUSED_BWD_CASES = [
+    ("small_c_concurrent", lambda: wl.small_c_bf16(), torch.bfloat16),
+    ("C64_tiny_frames_concurrent", lambda: wl.custom_conv(seed=42, T=5, H=4, W=4, keep_frac=[0.0, 1 / 16, 0.0, 1.0, 0.5],
+                                                          Cin=64, Cout=64, dtype="bf16"), torch.bfloat16),
+    ("C128x192_sequential", lambda: wl.custom_conv(seed=31, T=7, H=9, W=14, keep_frac=0.55, Cin=128, Cout=192,
+                                                   dtype="bf16", shuffle=True, empty_frames=(3,)), torch.bfloat16),
+    ("tiny_f32_sequential", lambda: wl.tiny_f32(), torch.float32),
+]
+
+
+@pytest.mark.parametrize("name,make,dtype", FUSED_BWD_CASES, ids=[c[0] for c in FUSED_BWD_CASES])
+def test_fused_bwd(sv, orc, name, make, dtype):
+    w = make()
+    nbr, _, st = gpu_index(sv, w, want_map=False)
+    assert st == 0
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    X, Wt, dY = dev(w.X, dtype), dev(w.Wt, dtype), dev(w.dY, dtype)
+    dX, dW, db = sv.svconv_bwd(dY, X, nbr, Wt)
+    dX2, dW2, db2 = sv.svconv_bwd(dY, X, nbr, Wt)
+    dX_sep = sv.svconv_bwd_data(dY, nbr, Wt)
+    torch.cuda.synchronize()
+    assert torch.equal(dX, dX_sep)                                   # same kernel, same sums
+    assert torch.equal(dX, dX2) and torch.equal(dW, dW2) and torch.equal(db, db2)  # deterministic
+    check = check_bf16 if dtype == torch.bfloat16 else check_f32
+    check(dX.float().cpu().numpy(), orc.bwd_data(w.dY, ref_n, w.Wt), "dX")
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    check(dW.cpu().numpy(), rdW, "dW")
+    check(db.cpu().numpy(), rdb, "db")
+    assert sv.svconv_read_error_word() == 0
+
+
+def test_fused_bwd_in_cuda_graph(sv):
+    w = wl.small_c_bf16(T=96)
+    nbr, _, st = gpu_index(sv, w, want_map=False)
+    X, Wt, dY = dev(w.X, torch.bfloat16), dev(w.Wt, torch.bfloat16), dev(w.dY, torch.bfloat16)
+    ref = [t.clone() for t in sv.svconv_bwd(dY, X, nbr, Wt)]  # first call outside capture
+    dX = torch.zeros_like(ref[0])
+    dW = torch.zeros_like(ref[1])
+    db = torch.zeros_like(ref[2])
+    ws = torch.empty(sv.svconv_bwd_workspace_size(sv.BF16, w.n, 64, 64), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            sv.svconv_bwd(dY, X, nbr, Wt, dX=dX, dW=dW, db=db, workspace=ws)
+        g.replay()
+    torch.cuda.synchronize()
+    for got, want in zip((dX, dW, db), ref):
+        assert torch.equal(got, want)
+    assert sv.svconv_read_error_word() == 0
+
+
 def test_bf16_deterministic(sv):
     w = wl.large_c_bwd_bf16(T=48)
     a = run_bf16(sv, w)
