@@ -20,6 +20,7 @@
 //  * wgrad_reduce_kernel: sums the splits in index order (deterministic, and
 //    compensated) and transposes to dW[o][j][i] through a 32x32 shared tile.
 #include "svconv_internal.h"
+#include "svconv_ptx.cuh"
 
 namespace svc {
 namespace {
@@ -124,6 +125,8 @@ __global__ void __launch_bounds__(256) wgrad_reduce_kernel(const float* __restri
                                                            int rows_pad, int Cin, int Cout, int grouped,
                                                            float* __restrict__ dW, float* __restrict__ db) {
   __shared__ float tile[kRedRows][33];
+  pdl_wait();  // the partials come from the kernel before this one
+  pdl_trigger();
   const int rows = 9 * Cin + 1;
   const int m0 = blockIdx.x * kRedRows, o0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -202,8 +205,7 @@ cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, 
                                 float* dW, float* db, cudaStream_t s) {
   const int rows = 9 * Cin + 1;
   dim3 grid((rows + kRedRows - 1) / kRedRows, (Cout + 31) / 32);
-  wgrad_reduce_kernel<<<grid, 256, 0, s>>>(partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
-  return cudaGetLastError();
+  return launch_pdl(wgrad_reduce_kernel, grid, dim3(256), 0, s, partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
 }
 
 }  // namespace svc

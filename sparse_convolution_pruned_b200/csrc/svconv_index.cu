@@ -8,6 +8,7 @@
 // and 36 B of N written; the writes are fully coalesced because consecutive
 // threads produce consecutive (k, j) entries of the frame's contiguous N rows.
 #include "svconv_internal.h"
+#include "svconv_ptx.cuh"
 
 namespace svc {
 namespace {
@@ -25,6 +26,8 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   __shared__ int s_flags;
   __shared__ int s_lo, s_hi;
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) {
     int flags = 0;
     int lo = frame_off[t], hi = frame_off[t + 1];
@@ -97,8 +100,7 @@ cudaError_t launch_build_index(const int32_t* coords, const int32_t* frame_off, 
     cudaError_t e = ensure_smem_attr(build_index_kernel, smem, done);
     if (e != cudaSuccess) return e;
   }
-  build_index_kernel<<<T, 256, smem, s>>>(coords, frame_off, T, H, W, n, nbr, M, status);
-  return cudaGetLastError();
+  return launch_pdl(build_index_kernel, dim3(T), dim3(256), smem, s, coords, frame_off, T, H, W, n, nbr, M, status);
 }
 
 }  // namespace svc

@@ -22,6 +22,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// The library's kernels are launched with programmatic stream serialization: a kernel
+// may start while the previous kernel on its stream is still draining.  Each thread
+// calls pdl_wait() before its first access to global memory (reads of inputs, writes
+// of outputs, the error word): it returns once the previous grid has completed and its
+// writes are visible, and is a no-op without a programmatic dependency.  pdl_trigger()
+// lets the next kernel's CTAs start their own set-up early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -467,6 +467,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const uint32_t a_tmem_col = (uint32_t)(n_acc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kConvHaloRows * 128;
 
+  if (threadIdx.x == 0) {
+    // afull: one builder group per A stage; ifull: the loader lanes' 32 cp.async arrivals + lane 0's expect_tx
+    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 33, kProdWarps);
+    prefetch_tmap(&p.tmap_a);
+    prefetch_tmap(&p.tmap_b);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bar->tmem_base, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();  // inputs, outputs and the row bounds may come from the kernel before this one
+  pdl_trigger();
   // rows handled by this launch (device-side bounds for the chunked adapter)
   int lo = 0, M = p.M;
   if (p.row_lo) {
@@ -486,19 +501,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int num_kb = taps * kb_per_tap;
   const int nbr_base = p.nbr_abs ? lo : 0;
 
-  if (threadIdx.x == 0) {
-    // afull: one builder group per A stage; ifull: the loader lanes' 32 cp.async arrivals + lane 0's expect_tx
-    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 33, kProdWarps);
-    prefetch_tmap(&p.tmap_a);
-    prefetch_tmap(&p.tmap_b);
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(&bar->tmem_base, tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
 
@@ -814,12 +816,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
       prefetch_tmap(&p.tmap_a);
     }
     __syncwarp();
+    pdl_wait();  // the neighbour table and features may come from the kernel before this one
     for (int t = blockIdx.x; t < num_tiles && issued < 2; t += gridDim.x) issue_tile(t, (int)issued++);
   } else if (warp == kBWarp) {
     if (lane == 0) {
       mbar_init(&bar->wfull, 1);
       fence_barrier_init();
       fence_proxy_async_smem();
+      pdl_wait();
       mbar_arrive_expect_tx(&bar->wfull, kSmallWBytes);
       const uint32_t dst = smem_u32(sw);
       for (int j = 0; j < 9; ++j) {
@@ -850,6 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
 
@@ -1074,6 +1080,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // inputs and outputs may belong to the kernel before this one
+  pdl_trigger();
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
 
@@ -1398,8 +1406,7 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
-  tc_conv_kernel<BN, MIRROR><<<grid, kThreads, smem, s>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(tc_conv_kernel<BN, MIRROR>, dim3(grid), dim3(kThreads), smem, s, prm);
 }
 
 template <bool MIRROR>
@@ -1408,8 +1415,7 @@ static cudaError_t launch_small_inst(const TcConvParams& prm, int grid, cudaStre
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_small_kernel<MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
-  tc_conv_small_kernel<MIRROR><<<grid, kThreads, smem, s>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(tc_conv_small_kernel<MIRROR>, dim3(grid), dim3(kThreads), smem, s, prm);
 }
 
 cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s) {
@@ -1494,8 +1500,7 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
   if (e != cudaSuccess) return e;
-  tc_wgrad_kernel<BN><<<grid, kThreads, smem, s>>>(prm);
-  return cudaGetLastError();
+  return launch_pdl(tc_wgrad_kernel<BN>, dim3(grid), dim3(kThreads), smem, s, prm);
 }
 
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
