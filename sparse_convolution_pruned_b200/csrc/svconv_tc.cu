@@ -90,6 +90,7 @@ struct __align__(16) TcBarriers {
 struct TcConvParams {
   CUtensorMap tmap_a;  // gather: halo boxes {64, 64}; dense: A tile {64, 128}
   CUtensorMap tmap_b;
+  CUtensorMap tmap_out;  // out_tma: out [out_rows][N] (row stride ldo), box {64, 32}
   const __nv_bfloat16* A;
   const int32_t* nbr;
   const int32_t* row_lo;
@@ -102,6 +103,7 @@ struct TcConvParams {
   int lda, a_rows, taps, Kc;
   int M, a_abs, nbr_abs, out_abs, N;
   int gelu, ldo, out_rows, stages_a, stages_b;
+  int out_tma;  // dense mode, residual == out: the epilogue adds into out with TMA reduce-adds
 };
 
 struct TcWgradParams {
@@ -123,21 +125,27 @@ __host__ __device__ constexpr int tmem_cols_for(int bn) {
 struct Carve {
   uint8_t* a;      // A ring
   uint8_t* b;      // B ring
+  uint8_t* epi;    // dense epilogue staging: 2 boxes of 32 rows x 128 bytes per epilogue warp
   uint8_t* halo;   // conv: 2 halo buffers; weight gradient: 2 slots x 2 halos
   int32_t* idx;    // 2 neighbour-row slots
   TcBarriers* bar;
 };
 
 struct Geometry {
-  size_t a_bytes, b_bytes, halo_bytes, idx_bytes;
+  size_t a_bytes, b_bytes, halo_bytes, idx_bytes, epi_bytes;
 };
 
 __host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// a_in_tmem: the gathered A stages live in tensor memory, so no shared A ring.
-__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem) {
+// a_in_tmem (the gather path): the gathered A stages live in tensor memory, so no shared A
+// ring, but two halo buffers and two index slots.  Dense path: an A ring by TMA, no halo,
+// and with epi_stage the epilogue's staging boxes.
+constexpr uint32_t kEpiBoxBytes = 32 * 128;  // 32 rows x 64 bf16 columns
+__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem, bool epi_stage = false) {
   return {a_in_tmem ? (size_t)0 : (size_t)sa * kABytes, (size_t)sb * bn * kBK * 2,
-          (size_t)2 * kConvHaloRows * 128, round_up((size_t)2 * kConvIdx * 4, 16)};
+          a_in_tmem ? (size_t)2 * kConvHaloRows * 128 : (size_t)0,
+          a_in_tmem ? round_up((size_t)2 * kConvIdx * 4, 16) : (size_t)0,
+          (!a_in_tmem && epi_stage) ? (size_t)kEpiWarps * 2 * kEpiBoxBytes : (size_t)0};
 }
 
 // Tensor-memory plan of the conv kernel: accumulator buffers first, then the A stages.
@@ -161,7 +169,7 @@ __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
 }
 
 __host__ __device__ inline size_t smem_total(const Geometry& g) {
-  return 1024 + g.a_bytes + g.b_bytes + g.halo_bytes + g.idx_bytes + sizeof(TcBarriers);
+  return 1024 + g.a_bytes + g.b_bytes + g.epi_bytes + g.halo_bytes + g.idx_bytes + sizeof(TcBarriers);
 }
 
 __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
@@ -170,7 +178,8 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
   Carve c;
   c.a = smem_raw + pad;
   c.b = c.a + g.a_bytes;
-  c.halo = c.b + g.b_bytes;
+  c.epi = c.b + g.b_bytes;  // 1024-aligned: the A and B stages are multiples of 1 KB
+  c.halo = c.epi + g.epi_bytes;
   c.idx = reinterpret_cast<int32_t*>(c.halo + g.halo_bytes);
   c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
   return c;
@@ -372,6 +381,35 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
   return true;
 }
 
+// Dense GEMM whose whole K extent of B fits in the B stages (num_kb <= SB): a run of
+// consecutive tiles of this CTA with the same output columns loads B once and keeps it
+// in shared memory.  b_load: first tile of a run (wait for the B stages to fill);
+// b_last: last tile of a run (release the B stages after its MMAs).  A streams per tile.
+__device__ __forceinline__ bool mma_tile_resident_b(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
+                                                    bool b_load, bool b_last, volatile int* abort_flag, int* err,
+                                                    uint64_t timeout_ns) {
+  int b = m.sb;
+  uint32_t pb = m.pb;
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!mbar_wait(&bar->afull[m.sa], m.pa, abort_flag, err, timeout_ns)) return false;
+    if (b_load && !mbar_wait(&bar->bfull[b], pb, abort_flag, err, timeout_ns)) return false;
+    const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
+    const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)b * m.b_stage16);
+#pragma unroll
+    for (int k = 0; k < kBK / 16; ++k)
+      tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, kb | k ? 1u : 0u);
+    tc_commit(&bar->aempty[m.sa]);
+    if (b_last) tc_commit(&bar->bempty[b]);
+    if (++m.sa == m.SA) {
+      m.sa = 0;
+      m.pa ^= 1u;
+    }
+    if (++b == m.SB) b = 0, pb ^= 1u;
+  }
+  if (b_last) m.sb = b, m.pb = pb;
+  return true;
+}
+
 __device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err, uint64_t timeout_ns) {
   if (issued) {
     volatile int never = 0;
@@ -383,6 +421,29 @@ __device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err
 // Epilogue of one output tile row: the fp32 accumulator row at TMEM address acc (this
 // warp's lane quarter, column 0 of the tile) + bias, GELU, residual -> bf16 row orow,
 // columns n0 .. n0 + BN - 1.  Two 32-column loads are in flight per wait.
+// 32 accumulator columns (raw fp32 bits) + bias[col ..], then GELU when asked.
+__device__ __forceinline__ void epi_bias_gelu(const TcConvParams& p, const uint32_t (&v)[32], float (&f)[32], int col) {
+#pragma unroll
+  for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
+  if (p.bias) {
+    if ((reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0) {  // col is a multiple of 32
+      const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 b = __ldg(b4 + q);
+        f[4 * q] += b.x, f[4 * q + 1] += b.y, f[4 * q + 2] += b.z, f[4 * q + 3] += b.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + col + q);
+    }
+  }
+  if (p.gelu) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) f[q] = 0.5f * f[q] * (1.0f + erff(f[q] * 0.70710678118654752f));
+  }
+}
+
 template <int BN>
 __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t acc, bool valid, size_t orow, int n0) {
 #pragma unroll 1
@@ -396,25 +457,7 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
     for (int hh = 0; hh < 2; ++hh) {
       const int c = c0 + 32 * hh;
       float f[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[hh][q]);
-      if (p.bias) {
-        if ((reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0) {  // n0 + c is a multiple of 32
-          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + c);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 b = __ldg(b4 + q);
-            f[4 * q] += b.x, f[4 * q + 1] += b.y, f[4 * q + 2] += b.z, f[4 * q + 3] += b.w;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) f[q] += __ldg(p.bias + n0 + c + q);
-        }
-      }
-      if (p.gelu) {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) f[q] = 0.5f * f[q] * (1.0f + erff(f[q] * 0.70710678118654752f));
-      }
+      epi_bias_gelu(p, v[hh], f, n0 + c);
       if (p.residual) {
         const uint4* rp = reinterpret_cast<const uint4*>(p.residual + orow * p.ldo + n0 + c);
 #pragma unroll
@@ -448,6 +491,55 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
   }
 }
 
+// Dense-mode epilogue with the residual add done by the TMA engine (residual == out):
+// this warp's 32 tile rows (+ bias, GELU) are rounded to bf16 and staged 64 columns at a
+// time in a 128-byte-swizzled box of shared memory (two boxes per warp, alternating),
+// and each box is added into out[orow0 .. orow0 + 31][n0 + c0 ..] by one tiled bulk
+// reduce-add, so the residual never crosses the SM and the output leaves it in whole
+// lines.  All 32 rows must be rows of out that this tile owns.  q counts the boxes this
+// warp has issued (it picks the box and the wait depth).
+template <int BN>
+__device__ __forceinline__ void epilogue_reduce_add(const TcConvParams& p, uint32_t acc, uint32_t boxes, uint32_t& q,
+                                                    int orow0, int n0) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t row_off = (uint32_t)lane * 128u;
+  const uint32_t sw = (uint32_t)(lane & 7);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 64, ++q) {
+    uint32_t v[2][32];
+    tmem_ld_32x32b_x32(acc + c0, v[0]);
+    tmem_ld_32x32b_x32(acc + c0 + 32, v[1]);
+    const uint32_t box = boxes + (q & 1u) * kEpiBoxBytes;
+    if (lane == 0) bulk_wait_group_read<1>();  // the reduce issued from this box two boxes ago has read it
+    __syncwarp();
+    tmem_ld_wait();
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float f[32];
+      epi_bias_gelu(p, v[hh], f, n0 + c0 + 32 * hh);
+      uint32_t packed[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+        packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      // 16-byte chunk k of the row lands at chunk k ^ (row & 7) (the map's 128-byte swizzle)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t kk = (uint32_t)(4 * hh + k);
+        st_shared_16(box + row_off + ((kk ^ sw) << 4), packed[4 * k], packed[4 * k + 1], packed[4 * k + 2],
+                     packed[4 * k + 3]);
+      }
+    }
+    fence_proxy_async_smem();  // make the generic-proxy stores visible to the TMA engine
+    __syncwarp();
+    if (lane == 0) {
+      tma_reduce_add_2d(&p.tmap_out, box, n0 + c0, orow0);
+      bulk_commit_group();
+    }
+  }
+}
+
 // ============================================================================ conv / dense GEMM
 // MIRROR: gather through column 8-j (data gradient); it always pairs with an
 // MN-major weight operand.
@@ -456,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   const bool gather = p.nbr != nullptr;  // gathered A lives in tensor memory
   const int SA = p.stages_a, SB = p.stages_b;
-  const Geometry geo = conv_geometry(BN, SA, SB, gather);
+  const bool tma_epi = p.out_tma != 0;  // set by the host only in dense mode
+  const Geometry geo = conv_geometry(BN, SA, SB, gather, tma_epi);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -500,6 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const int taps = p.taps;
   const int num_kb = taps * kb_per_tap;
   const int nbr_base = p.nbr_abs ? lo : 0;
+  // dense GEMM with all of K in the B stages: B stays resident across this CTA's tiles
+  // with the same output columns (with the stride order, every tile when gridDim.x is a
+  // multiple of the column-tile count), so per tile only A crosses into the SM
+  const bool res_b = !gather && num_kb <= SB;
 
   const uint32_t tmem_base = bar->tmem_base;
   volatile int* abort_flag = &bar->abort_flag;
@@ -571,8 +668,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     // ------------------------------------------------------------ weight loader
     uint32_t it = 0;
     bool aborted = false;
+    int prev_nt = -1;
     for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
-      const int n0 = (tile % n_tiles) * BN;
+      const int nt = tile % n_tiles;
+      if (res_b && nt == prev_nt) continue;  // this run's B is still resident
+      prev_nt = nt;
+      const int n0 = nt * BN;
       for (int cb = 0; cb < kb_per_tap && !aborted; ++cb)
         for (int j = 0; j < taps; ++j, ++it) {
           const int sb = it % SB;
@@ -695,15 +796,27 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       mi.a_tmem0 = tmem_base + a_tmem_col;
       uint32_t tc = 0;
       bool issued = false;
+      int prev_nt = -1;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
         const uint32_t ab = tc % (uint32_t)n_acc;
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, n_acc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
         constexpr int kGroup = BN == 256 ? 1 : 2;
-        const bool ok =
-            gather ? mma_tile<true, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)
-                   : mma_tile<false, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        bool ok;
+        if (gather) {
+          ok = mma_tile<true, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        } else if (res_b) {
+          const int nt = tile % n_tiles;
+          const int next = tile + (int)gridDim.x;
+          const bool b_load = nt != prev_nt;
+          const bool b_last = next >= num_tiles || next % n_tiles != nt;
+          prev_nt = nt;
+          ok = mma_tile_resident_b(bar, mi, num_kb, tmem_base + ab * BN, b_load, b_last, abort_flag, err,
+                                   p.timeout_ns);
+        } else {
+          ok = mma_tile<false, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        }
         if (!ok) break;
         tc_commit(&bar->tfull[ab]);
       }
@@ -712,8 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (warps 0-3)
-    uint32_t tc = 0;
+    uint32_t tc = 0, nbox = 0;
     const int out_base = p.out_abs ? lo : 0;
+    const uint32_t epi_boxes = smem_u32(sm.epi) + (uint32_t)warp * 2u * kEpiBoxBytes;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
       const uint32_t ab = tc % (uint32_t)n_acc;
       const int m0 = (tile / n_tiles) * kBM;
@@ -729,10 +843,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       if (!warp_wait(&bar->tfull[ab], ring_parity(tc, n_acc), abort_flag, err, p.timeout_ns)) break;
       tc_fence_after();
       const bool valid = row < M && orow_i >= 0 && orow_i < p.out_rows;
-      epilogue_rows<BN>(p, tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN, valid, (size_t)orow_i, n0);
+      const uint32_t acc = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN;
+      if (tma_epi && __all_sync(0xffffffffu, valid))
+        epilogue_reduce_add<BN>(p, acc, epi_boxes, nbox, orow_i - lane, n0);
+      else
+        epilogue_rows<BN>(p, acc, valid, (size_t)orow_i, n0);
       tc_fence_before();
       warp_arrive(&bar->tempty[ab]);
     }
+    if (tma_epi && lane == 0) bulk_wait_group<0>();  // reduce-adds complete before the CTA exits
   }
 
   tc_fence_before();
@@ -1370,14 +1489,26 @@ static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint
   return make_tmap(m, base, 2, dims, strides, box);
 }
 
-// Stage counts for the dense path: up to 4 A stages (short latency) and as many
-// B stages (TMA from L2) as fit in about 220 KB of shared memory.
-static void pick_stages(int bn, int* sa, int* sb) {
+// Stage counts for the dense path (about 220 KB of shared memory).  When all num_kb
+// K-blocks of B fit, take that many B stages (B then stays resident across a CTA's tiles
+// with the same columns) and as many A stages (2-4) as remain; otherwise up to 4 A stages
+// (short latency) and as many B stages (TMA from L2) as fit.
+static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
   const size_t budget = 220 * 1024;
-  for (int a = 4; a >= 2; a -= 2) {  // two builder groups alternate A stages: keep it even
+  if (num_kb <= kMaxStages) {
+    for (int a = 4; a >= 2; --a) {
+      const int b = num_kb < 2 ? 2 : num_kb;
+      if (smem_total(conv_geometry(bn, a, b, false, epi)) <= budget) {
+        *sa = a;
+        *sb = b;
+        return;
+      }
+    }
+  }
+  for (int a = 4; a >= 2; a -= 2) {
     int b_best = 0;
     for (int b = 2; b <= kMaxStages; ++b) {
-      const Geometry g = conv_geometry(bn, a, b, false);
+      const Geometry g = conv_geometry(bn, a, b, false, epi);
       if (smem_total(g) <= budget) b_best = b;
     }
     if (b_best >= 3 || (a == 2 && b_best >= 2)) {
@@ -1400,9 +1531,9 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
     for (int b = 2; b <= kMaxStages; ++b)
       if (smem_total(conv_geometry(BN, 0, b, true)) <= 220 * 1024) prm.stages_b = b;
   } else {
-    pick_stages(BN, &prm.stages_a, &prm.stages_b);
+    pick_stages(BN, prm.taps * (prm.Kc / kBK), prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
   }
-  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b, a_in_tmem));
+  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b, a_in_tmem, prm.out_tma != 0));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
   if (e != cudaSuccess) return e;
@@ -1435,6 +1566,15 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
     const uint64_t strides[2] = {(uint64_t)a.N * 2, (uint64_t)a.N * 9 * 2};
     const uint32_t box[3] = {64u, 1u, 64u};
     if (!make_tmap(&prm.tmap_b, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  // in-place residual of a dense GEMM: the epilogue adds into out with TMA reduce-adds
+  // (out [out_rows][N], row stride ldo; boxes of 32 rows x 64 columns)
+  if (!a.nbr && a.residual && a.residual == a.out && a.N % 64 == 0 && a.out_rows > 0 && (a.ldo * 2) % 16 == 0 &&
+      (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0) {
+    const uint64_t dims[2] = {(uint64_t)a.N, (uint64_t)a.out_rows};
+    const uint64_t strides[1] = {(uint64_t)a.ldo * 2};
+    const uint32_t box[2] = {64u, 32u};
+    prm.out_tma = make_tmap(&prm.tmap_out, a.out, 2, dims, strides, box) ? 1 : 0;
   }
   prm.A = static_cast<const __nv_bfloat16*>(a.A);
   prm.nbr = a.nbr;
