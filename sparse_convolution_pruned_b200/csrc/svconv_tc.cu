@@ -103,7 +103,7 @@ struct TcConvParams {
   int lda, a_rows, taps, Kc;
   int M, a_abs, nbr_abs, out_abs, N;
   int gelu, ldo, out_rows, stages_a, stages_b;
-  int out_tma;  // dense mode, residual == out: the epilogue adds into out with TMA reduce-adds
+  int out_tma;  // 1: the epilogue writes out with TMA stores; 2: adds into out (residual == out) with TMA reduce-adds
 };
 
 struct TcWgradParams {
@@ -138,14 +138,14 @@ struct Geometry {
 __host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // a_in_tmem (the gather path): the gathered A stages live in tensor memory, so no shared A
-// ring, but two halo buffers and two index slots.  Dense path: an A ring by TMA, no halo,
-// and with epi_stage the epilogue's staging boxes.
+// ring, but two halo buffers and two index slots.  Dense path: an A ring by TMA, no halo.
+// epi_stage: the epilogue's staging boxes (TMA stores).
 constexpr uint32_t kEpiBoxBytes = 32 * 128;  // 32 rows x 64 bf16 columns
 __host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem, bool epi_stage = false) {
   return {a_in_tmem ? (size_t)0 : (size_t)sa * kABytes, (size_t)sb * bn * kBK * 2,
           a_in_tmem ? (size_t)2 * kConvHaloRows * 128 : (size_t)0,
           a_in_tmem ? round_up((size_t)2 * kConvIdx * 4, 16) : (size_t)0,
-          (!a_in_tmem && epi_stage) ? (size_t)kEpiWarps * 2 * kEpiBoxBytes : (size_t)0};
+          epi_stage ? (size_t)kEpiWarps * 2 * kEpiBoxBytes : (size_t)0};
 }
 
 // Tensor-memory plan of the conv kernel: accumulator buffers first, then the A stages.
@@ -153,9 +153,16 @@ __host__ __device__ constexpr int conv_acc_buffers(int bn, bool a_in_tmem) { ret
 __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c) {
   return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
 }
-__host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem) {
+__host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem, int a_stages) {
   return pow2_cols((uint32_t)(conv_acc_buffers(bn, a_in_tmem) * bn) +
-                   (a_in_tmem ? (uint32_t)(kTmemAStages * kTmemAStageCols) : 0u));
+                   (a_in_tmem ? (uint32_t)(a_stages * kTmemAStageCols) : 0u));
+}
+// Gather conv: as many A stages in tensor memory as fit next to the accumulators (an even
+// number: the two builder groups take alternate stages; at most kMaxStages).
+__host__ __device__ constexpr int conv_tmem_a_stages(int bn) {
+  return (512 - conv_acc_buffers(bn, true) * bn) / (int)kTmemAStageCols >= kMaxStages
+             ? kMaxStages
+             : ((512 - conv_acc_buffers(bn, true) * bn) / (int)kTmemAStageCols) & ~1;
 }
 
 // Weight gradient: A lives in tensor memory; wgrad_slots(bn) slots of (index entries, halo).
@@ -187,7 +194,8 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
 
 // nslots neighbour-row slots with the given arrival counts; everything else fixed.
 __device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uint32_t afull_count, int nslots,
-                                              uint32_t ifull_count, uint32_t iempty_count) {
+                                              uint32_t ifull_count, uint32_t iempty_count,
+                                              uint32_t tempty_count = kEpiWarps) {
   for (int i = 0; i < 32; ++i) b->zero16[i] = 0u;
   for (int i = 0; i < nslots; ++i) {
     mbar_init(&b->ifull[i], ifull_count);
@@ -205,7 +213,7 @@ __device__ __forceinline__ void init_barriers(TcBarriers* b, int sa, int sb, uin
     mbar_init(&b->hfull[i], 1);
     mbar_init(&b->hempty[i], kProdWarps);
     mbar_init(&b->tfull[i], 1);
-    mbar_init(&b->tempty[i], kEpiWarps);
+    mbar_init(&b->tempty[i], tempty_count);
   }
   mbar_init(&b->done, 1);
   b->abort_flag = 0;
@@ -329,7 +337,9 @@ __device__ __forceinline__ MmaIssuer make_issuer(const Carve& sm, uint32_t b_sta
 // The first shared-memory access (an mbarrier wait) after a batch of MMAs stalls until
 // those MMAs have read their operands, so checking two stages per batch halves that cost
 // when MMAs are short (N = 64); GROUP = 1 keeps the deepest pipelining for long MMAs.
-template <bool A_TMEM, int GROUP>
+// PAIR: M = 256 MMAs of a CTA pair (issued by rank 0; the stage barriers count both
+// CTAs' producers and the commits arrive in both CTAs).
+template <bool A_TMEM, int GROUP, bool PAIR = false>
 __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                          volatile int* abort_flag, int* err, uint64_t timeout_ns) {
   for (int kb = 0; kb < num_kb; kb += GROUP) {
@@ -358,16 +368,31 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
       if constexpr (A_TMEM) {
         const uint32_t at = m.a_tmem0 + (uint32_t)sa[g] * kTmemAStageCols;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+        for (int k = 0; k < kBK / 16; ++k) {
+          if constexpr (PAIR)
+            tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+          else
+            tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+        }
       } else {
         const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)sa[g] * m.a_stage16);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+        for (int k = 0; k < kBK / 16; ++k) {
+          if constexpr (PAIR)
+            tc_mma_bf16_pair(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc,
+                             (kb + g) | k ? 1u : 0u);
+          else
+            tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc,
+                        (kb + g) | k ? 1u : 0u);
+        }
       }
-      tc_commit(&bar->aempty[sa[g]]);
-      tc_commit(&bar->bempty[sb[g]]);
+      if constexpr (PAIR) {
+        tc_commit_pair(&bar->aempty[sa[g]]);
+        tc_commit_pair(&bar->bempty[sb[g]]);
+      } else {
+        tc_commit(&bar->aempty[sa[g]]);
+        tc_commit(&bar->bempty[sb[g]]);
+      }
       if (++m.sa == m.SA) {
         m.sa = 0;
         m.pa ^= 1u;
@@ -381,10 +406,54 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
   return true;
 }
 
+// Gather conv: A stage s (tensor memory) and B stage s (shared memory) advance together on
+// one full / empty barrier pair (full counts the builder warps and the weight loader), so a
+// stage costs the issuing thread one wait and one commit.  The tensor pipe queues only a
+// few MMAs, so every cycle the issuing thread spends between MMA bursts is a cycle the pipe
+// may sit idle.  GROUP: stages whose barriers are checked before their MMAs are issued.
+template <int GROUP, bool PAIR>
+__device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
+                                                 volatile int* abort_flag, int* err, uint64_t timeout_ns) {
+  for (int kb = 0; kb < num_kb; kb += GROUP) {
+    const int cnt = min(GROUP, num_kb - kb);
+    {
+      int st = m.sa;
+      uint32_t ps = m.pa;
+#pragma unroll
+      for (int g = 0; g < GROUP; ++g) {
+        if (g < cnt && !mbar_wait(&bar->afull[st], ps, abort_flag, err, timeout_ns)) return false;
+        if (++st == m.SA) st = 0, ps ^= 1u;
+      }
+    }
+    tc_fence_after();  // the A stages were written to tensor memory by other threads
+#pragma unroll
+    for (int g = 0; g < GROUP; ++g) {
+      if (g >= cnt) break;
+      const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sa * m.b_stage16);
+      const uint32_t at = m.a_tmem0 + (uint32_t)m.sa * kTmemAStageCols;
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        if constexpr (PAIR)
+          tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+        else
+          tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+      }
+      if constexpr (PAIR) {
+        tc_commit_pair(&bar->aempty[m.sa]);
+      } else {
+        tc_commit(&bar->aempty[m.sa]);
+      }
+      if (++m.sa == m.SA) m.sa = 0, m.pa ^= 1u;
+    }
+  }
+  return true;
+}
+
 // Dense GEMM whose whole K extent of B fits in the B stages (num_kb <= SB): a run of
 // consecutive tiles of this CTA with the same output columns loads B once and keeps it
 // in shared memory.  b_load: first tile of a run (wait for the B stages to fill);
 // b_last: last tile of a run (release the B stages after its MMAs).  A streams per tile.
+template <bool PAIR = false>
 __device__ __forceinline__ bool mma_tile_resident_b(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                                     bool b_load, bool b_last, volatile int* abort_flag, int* err,
                                                     uint64_t timeout_ns) {
@@ -396,10 +465,19 @@ __device__ __forceinline__ bool mma_tile_resident_b(TcBarriers* bar, MmaIssuer& 
     const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
     const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)b * m.b_stage16);
 #pragma unroll
-    for (int k = 0; k < kBK / 16; ++k)
-      tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, kb | k ? 1u : 0u);
-    tc_commit(&bar->aempty[m.sa]);
-    if (b_last) tc_commit(&bar->bempty[b]);
+    for (int k = 0; k < kBK / 16; ++k) {
+      if constexpr (PAIR)
+        tc_mma_bf16_pair(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, kb | k ? 1u : 0u);
+      else
+        tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc, kb | k ? 1u : 0u);
+    }
+    if constexpr (PAIR) {
+      tc_commit_pair(&bar->aempty[m.sa]);
+      if (b_last) tc_commit_pair(&bar->bempty[b]);
+    } else {
+      tc_commit(&bar->aempty[m.sa]);
+      if (b_last) tc_commit(&bar->bempty[b]);
+    }
     if (++m.sa == m.SA) {
       m.sa = 0;
       m.pa ^= 1u;
@@ -410,10 +488,17 @@ __device__ __forceinline__ bool mma_tile_resident_b(TcBarriers* bar, MmaIssuer& 
   return true;
 }
 
+// PAIR: the commit always goes out (to both CTAs), so the other CTA's wait on its own
+// copy of `done` ends even when no tile was issued.
+template <bool PAIR = false>
 __device__ __forceinline__ void mma_drain(TcBarriers* bar, bool issued, int* err, uint64_t timeout_ns) {
-  if (issued) {
+  if (issued || PAIR) {
     volatile int never = 0;
-    tc_commit(&bar->done);
+    if constexpr (PAIR) {
+      tc_commit_pair(&bar->done);
+    } else {
+      tc_commit(&bar->done);
+    }
     mbar_wait(&bar->done, 0, &never, err, timeout_ns);
   }
 }
@@ -491,16 +576,17 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
   }
 }
 
-// Dense-mode epilogue with the residual add done by the TMA engine (residual == out):
-// this warp's 32 tile rows (+ bias, GELU) are rounded to bf16 and staged 64 columns at a
-// time in a 128-byte-swizzled box of shared memory (two boxes per warp, alternating),
-// and each box is added into out[orow0 .. orow0 + 31][n0 + c0 ..] by one tiled bulk
-// reduce-add, so the residual never crosses the SM and the output leaves it in whole
-// lines.  All 32 rows must be rows of out that this tile owns.  q counts the boxes this
-// warp has issued (it picks the box and the wait depth).
-template <int BN>
-__device__ __forceinline__ void epilogue_reduce_add(const TcConvParams& p, uint32_t acc, uint32_t boxes, uint32_t& q,
-                                                    int orow0, int n0) {
+// Epilogue through the TMA engine: this warp's 32 tile rows (+ bias, GELU) are rounded
+// to bf16 and staged 64 columns at a time in a 128-byte-swizzled box of shared memory
+// (two boxes per warp, alternating), and each box goes to out[orow0 .. orow0 + 31]
+// [n0 + c0 ..] as one tiled bulk store (REDUCE: a bulk reduce-add into out, which holds
+// the residual), so the output leaves the SM in whole lines and a residual never enters
+// it.  release() runs once the last accumulator columns are in registers, so the MMAs of
+// the next tile may start while the last boxes are still being written.  All 32 rows must
+// be rows of out that this tile owns.  q counts the boxes this warp has issued.
+template <int BN, bool REDUCE, typename Release>
+__device__ __forceinline__ void epilogue_tma(const TcConvParams& p, uint32_t acc, uint32_t boxes, uint32_t& q,
+                                             int orow0, int n0, Release release) {
   const int lane = threadIdx.x & 31;
   const uint32_t row_off = (uint32_t)lane * 128u;
   const uint32_t sw = (uint32_t)(lane & 7);
@@ -510,9 +596,10 @@ __device__ __forceinline__ void epilogue_reduce_add(const TcConvParams& p, uint3
     tmem_ld_32x32b_x32(acc + c0, v[0]);
     tmem_ld_32x32b_x32(acc + c0 + 32, v[1]);
     const uint32_t box = boxes + (q & 1u) * kEpiBoxBytes;
-    if (lane == 0) bulk_wait_group_read<1>();  // the reduce issued from this box two boxes ago has read it
+    if (lane == 0) bulk_wait_group_read<1>();  // the copy issued from this box two boxes ago has read it
     __syncwarp();
     tmem_ld_wait();
+    if (c0 + 64 >= BN) release();
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float f[32];
@@ -534,7 +621,10 @@ __device__ __forceinline__ void epilogue_reduce_add(const TcConvParams& p, uint3
     fence_proxy_async_smem();  // make the generic-proxy stores visible to the TMA engine
     __syncwarp();
     if (lane == 0) {
-      tma_reduce_add_2d(&p.tmap_out, box, n0 + c0, orow0);
+      if constexpr (REDUCE)
+        tma_reduce_add_2d(&p.tmap_out, box, n0 + c0, orow0);
+      else
+        tma_store_2d(&p.tmap_out, box, n0 + c0, orow0);
       bulk_commit_group();
     }
   }
@@ -543,35 +633,62 @@ __device__ __forceinline__ void epilogue_reduce_add(const TcConvParams& p, uint3
 // ============================================================================ conv / dense GEMM
 // MIRROR: gather through column 8-j (data gradient); it always pairs with an
 // MN-major weight operand.
-template <int BN, bool MIRROR>
+// PAIR: a cluster of two CTAs computes 256-row tiles with M = 256 MMAs: each CTA gathers
+// (or loads) its own 128 rows of A and holds their accumulator, loads half of the tile's
+// B columns, and CTA rank 0 issues the MMAs for both.  Every SM then streams half of B
+// per 128 output rows.  Barriers that count both CTAs' producers (A and B stages,
+// accumulator release) live in rank 0; the MMA commits arrive in both CTAs.
+template <int BN, bool MIRROR, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
+  static_assert(!PAIR || BN == 256, "CTA pairs run 256-column tiles");
   extern __shared__ uint8_t smem_raw[];
   const bool gather = p.nbr != nullptr;  // gathered A lives in tensor memory
   const int SA = p.stages_a, SB = p.stages_b;
-  const bool tma_epi = p.out_tma != 0;  // set by the host only in dense mode
-  const Geometry geo = conv_geometry(BN, SA, SB, gather, tma_epi);
+  const bool tma_epi = p.out_tma != 0;
+  constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns this CTA loads per stage
+  constexpr int kRows = PAIR ? 2 * kBM : kBM;  // output rows per tile
+  const Geometry geo = conv_geometry(kBCols, SA, SB, gather, tma_epi);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
-  constexpr uint32_t kBBytes = BN * kBK * 2;
-  const uint32_t tmem_cols = conv_tmem_cols(BN, gather);
+  constexpr uint32_t kBBytes = kBCols * kBK * 2;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // first tile of this CTA (pair)
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;    // tile stride
+  const int row_off = (int)rank * kBM;                                  // this CTA's rows within a tile
+  // rank 0's copy of a barrier (PAIR)
+  auto lead = [](uint64_t* b) -> uint32_t { return mapa_shared(smem_u32(b), 0u); };
+  const uint32_t tmem_cols = conv_tmem_cols(BN, gather, SA);
   const int n_acc = conv_acc_buffers(BN, gather);
   const uint32_t a_tmem_col = (uint32_t)(n_acc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kConvHaloRows * 128;
 
   if (threadIdx.x == 0) {
     // afull: one builder group per A stage; ifull: the loader lanes' 32 cp.async arrivals + lane 0's expect_tx
-    init_barriers(bar, SA, SB, gather ? kProdWarps / 2 : 1, 2, 33, kProdWarps);
+    // gather: afull / aempty serve A and B stage s together (SA == SB); afull counts the
+    // builder warps (of both CTAs of a pair) and the weight loader's expect_tx arrival
+    init_barriers(bar, SA, SB, gather ? (PAIR ? kProdWarps : kProdWarps / 2) + 1 : 1, 2, 33, kProdWarps,
+                  PAIR ? 2 * kEpiWarps : kEpiWarps);
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&bar->tmem_base, tmem_cols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&bar->tmem_base, tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&bar->tmem_base, tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrival
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   pdl_wait();  // inputs, outputs and the row bounds may come from the kernel before this one
   pdl_trigger();
@@ -586,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     }
     M = m < 0 ? 0 : m;
   }
-  const int m_tiles = (M + kBM - 1) / kBM;
+  const int m_tiles = (M + kRows - 1) / kRows;
   const int n_tiles = p.N / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int kb_per_tap = p.Kc / kBK;
@@ -609,15 +726,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       // are issued right away and both loads are in flight together.
       uint32_t ti = 0, hi = 0, ni = 0;  // ni: index loads issued
       bool aborted = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
-        const int m0 = (tile / n_tiles) * kBM;
+      for (int tile = unit0; tile < num_tiles && !aborted; tile += units, ++ti) {
+        const int m0 = (tile / n_tiles) * kRows + row_off;
         const int slot = ti & 1;
         if (!warp_wait(&bar->iempty[slot], ring_parity(ti, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
         const int32_t* src = p.nbr + (size_t)(nbr_base + m0) * 9;
-        const int lim = min(M - m0, kBM) * 9;
+        const int lim = max(0, min(M - m0, kBM)) * 9;  // PAIR: rank 1's rows may all lie past M
         copy_index_entries(smem_u32(sm.idx + slot * kConvIdx), src, lim,
                            ((reinterpret_cast<uintptr_t>(src) & 15u) == 0), &bar->ifull[slot], 0u);
         __syncwarp();
@@ -647,8 +764,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       const int a_base = p.a_abs ? lo : 0;
       uint32_t it = 0;
       bool aborted = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
-        const int m0 = (tile / n_tiles) * kBM;
+      for (int tile = unit0; tile < num_tiles && !aborted; tile += units) {
+        const int m0 = (tile / n_tiles) * kRows + row_off;
         for (int cb = 0; cb < kb_per_tap; ++cb, ++it) {
           const int sa = it % SA;
           if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
@@ -656,20 +773,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             break;
           }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&bar->afull[sa], (uint32_t)kABytes);
-            tma_load_2d(smem_u32(sm.a + (size_t)sa * kABytes), &p.tmap_a, &bar->afull[sa], cb * kBK, a_base + m0);
+            const uint32_t dst = smem_u32(sm.a + (size_t)sa * kABytes);
+            if constexpr (PAIR) {
+              if (leader) mbar_arrive_expect_tx(&bar->afull[sa], 2u * (uint32_t)kABytes);  // both CTAs' rows
+              tma_load_2d_pair(dst, &p.tmap_a, lead(&bar->afull[sa]), cb * kBK, a_base + m0);
+            } else {
+              mbar_arrive_expect_tx(&bar->afull[sa], (uint32_t)kABytes);
+              tma_load_2d(dst, &p.tmap_a, &bar->afull[sa], cb * kBK, a_base + m0);
+            }
           }
           __syncwarp();
         }
       }
-      if (aborted) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
+      if (aborted && leader) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
     }
   } else if (warp == kBWarp) {
     // ------------------------------------------------------------ weight loader
+    // (gather: on the A stages' barrier pair; dense: its own ring)
+    uint64_t* const bf = gather ? bar->afull : bar->bfull;
+    uint64_t* const be = gather ? bar->aempty : bar->bempty;
     uint32_t it = 0;
     bool aborted = false;
     int prev_nt = -1;
-    for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x) {
+    for (int tile = unit0; tile < num_tiles && !aborted; tile += units) {
       const int nt = tile % n_tiles;
       if (res_b && nt == prev_nt) continue;  // this run's B is still resident
       prev_nt = nt;
@@ -677,25 +803,50 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       for (int cb = 0; cb < kb_per_tap && !aborted; ++cb)
         for (int j = 0; j < taps; ++j, ++it) {
           const int sb = it % SB;
-          if (!warp_wait(&bar->bempty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          if (!warp_wait(&be[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
             aborted = true;
             break;
           }
           if (lane == 0) {
             const uint32_t dst = smem_u32(sm.b + (size_t)sb * kBBytes);
-            mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
-            if constexpr (!MIRROR) {
-              tma_load_2d(dst, &p.tmap_b, &bar->bfull[sb], j * p.Kc + cb * kBK, n0);
-            } else {
+            const int nb = n0 + (int)rank * kBCols;  // this CTA's B columns
+            if constexpr (PAIR) {
+              if (leader) mbar_arrive_expect_tx(&bf[sb], 2u * kBBytes);  // both halves
+              const uint32_t fb = lead(&bf[sb]);
+              if constexpr (!MIRROR) {
+                tma_load_2d_pair(dst, &p.tmap_b, fb, j * p.Kc + cb * kBK, nb);
+              } else {
 #pragma unroll
-              for (int q = 0; q < BN / 64; ++q)
-                tma_load_3d(dst + q * 8192, &p.tmap_b, &bar->bfull[sb], n0 + q * 64, j, cb * kBK);
+                for (int q = 0; q < kBCols / 64; ++q) tma_load_3d_pair(dst + q * 8192, &p.tmap_b, fb, nb + q * 64, j, cb * kBK);
+              }
+            } else {
+              mbar_arrive_expect_tx(&bf[sb], kBBytes);
+              if constexpr (!MIRROR) {
+                tma_load_2d(dst, &p.tmap_b, &bf[sb], j * p.Kc + cb * kBK, nb);
+              } else {
+#pragma unroll
+                for (int q = 0; q < kBCols / 64; ++q)
+                  tma_load_3d(dst + q * 8192, &p.tmap_b, &bf[sb], nb + q * 64, j, cb * kBK);
+              }
             }
           }
           __syncwarp();
         }
     }
-    if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+    if (aborted) {
+      if (gather || !leader) {
+        // the full barriers also count other producers (or live in the other CTA): give
+        // this warp's copies in flight time to land instead of waiting on a phase
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000u) {
+          }
+        }
+        __syncwarp();
+      } else {
+        drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+      }
+    }
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders
     // Two groups of four warps build alternate K-blocks (group g takes the K-blocks
@@ -714,13 +865,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       const uint32_t zero_row = smem_u32(bar->zero16);
       uint32_t ti = 0, hi = 0, it = 0;
       bool aborted = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti) {
+      for (int tile = unit0; tile < num_tiles && !aborted; tile += units, ++ti) {
         const int slot = ti & 1;
         if (!warp_wait(&bar->ifull[slot], ring_parity(ti, 2), abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
-        const int m0 = (tile / n_tiles) * kBM;
+        const int m0 = (tile / n_tiles) * kRows + row_off;
         const bool row_ok = m0 + r < M;
         const int hlo = m0 - kConvPad;  // A row of halo row 0
         const uint32_t sidx_s = smem_u32(sm.idx + slot * kConvIdx);
@@ -771,7 +922,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             tmem_st_32x32b_x32(a_lane + (uint32_t)sa * kTmemAStageCols, v);
             tmem_st_wait();
             tc_fence_before();
-            warp_arrive(&bar->afull[sa]);
+            if (PAIR && !leader) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(lead(&bar->afull[sa]));
+            } else {
+              warp_arrive(&bar->afull[sa]);
+            }
           }
           if (!aborted) {
             warp_arrive(&bar->hempty[hb]);
@@ -783,9 +939,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       MmaCfg c;
-      c.idesc = idesc_bf16_f32(kBM, BN, 0, MIRROR ? 1 : 0);
+      c.idesc = idesc_bf16_f32(kRows, BN, 0, MIRROR ? 1 : 0);
       c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // smem A (dense): K-major, 128-byte rows
       if (MIRROR) {
         c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // B: MN-major, 64-wide MN groups 8 KB apart
@@ -797,30 +953,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       uint32_t tc = 0;
       bool issued = false;
       int prev_nt = -1;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+      for (int tile = unit0; tile < num_tiles; tile += units, ++tc) {
         const uint32_t ab = tc % (uint32_t)n_acc;
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, n_acc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        constexpr int kGroup = BN == 256 ? 1 : 2;
+        constexpr int kGroup = 2;
         bool ok;
         if (gather) {
-          ok = mma_tile<true, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+          ok = mma_tile_unified<kGroup, PAIR>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
         } else if (res_b) {
           const int nt = tile % n_tiles;
-          const int next = tile + (int)gridDim.x;
+          const int next = tile + units;
           const bool b_load = nt != prev_nt;
           const bool b_last = next >= num_tiles || next % n_tiles != nt;
           prev_nt = nt;
-          ok = mma_tile_resident_b(bar, mi, num_kb, tmem_base + ab * BN, b_load, b_last, abort_flag, err,
-                                   p.timeout_ns);
+          ok = mma_tile_resident_b<PAIR>(bar, mi, num_kb, tmem_base + ab * BN, b_load, b_last, abort_flag, err,
+                                         p.timeout_ns);
         } else {
-          ok = mma_tile<false, kGroup>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+          ok = mma_tile<false, kGroup, PAIR>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
         }
         if (!ok) break;
-        tc_commit(&bar->tfull[ab]);
+        if constexpr (PAIR) {
+          tc_commit_pair(&bar->tfull[ab]);
+        } else {
+          tc_commit(&bar->tfull[ab]);
+        }
       }
-      mma_drain(bar, issued, err, p.timeout_ns);
+      mma_drain<PAIR>(bar, issued, err, p.timeout_ns);
+    } else if (PAIR && lane == 0) {
+      // the other CTA's MMAs read this CTA's tensor and shared memory: wait for them to finish
+      volatile int never = 0;
+      mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
     }
     __syncwarp();
   } else {
@@ -828,9 +992,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     uint32_t tc = 0, nbox = 0;
     const int out_base = p.out_abs ? lo : 0;
     const uint32_t epi_boxes = smem_u32(sm.epi) + (uint32_t)warp * 2u * kEpiBoxBytes;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tc) {
+    for (int tile = unit0; tile < num_tiles; tile += units, ++tc) {
       const uint32_t ab = tc % (uint32_t)n_acc;
-      const int m0 = (tile / n_tiles) * kBM;
+      const int m0 = (tile / n_tiles) * kRows + row_off;
       const int n0 = (tile % n_tiles) * BN;
       const int row = m0 + warp * 32 + lane;
       const int orow_i = out_base + row;
@@ -844,21 +1008,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       tc_fence_after();
       const bool valid = row < M && orow_i >= 0 && orow_i < p.out_rows;
       const uint32_t acc = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN;
-      if (tma_epi && __all_sync(0xffffffffu, valid))
-        epilogue_reduce_add<BN>(p, acc, epi_boxes, nbox, orow_i - lane, n0);
-      else
+      // hand the accumulator back to the MMA issuer (at rank 0 of a pair)
+      auto release = [&]() {
+        tc_fence_before();
+        if (PAIR && !leader) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead(&bar->tempty[ab]));
+        } else {
+          warp_arrive(&bar->tempty[ab]);
+        }
+      };
+      if (tma_epi && __all_sync(0xffffffffu, valid)) {
+        if (p.out_tma == 2)
+          epilogue_tma<BN, true>(p, acc, epi_boxes, nbox, orow_i - lane, n0, release);
+        else
+          epilogue_tma<BN, false>(p, acc, epi_boxes, nbox, orow_i - lane, n0, release);
+      } else {
         epilogue_rows<BN>(p, acc, valid, (size_t)orow_i, n0);
-      tc_fence_before();
-      warp_arrive(&bar->tempty[ab]);
+        release();
+      }
     }
-    if (tma_epi && lane == 0) bulk_wait_group<0>();  // reduce-adds complete before the CTA exits
+    if (tma_epi && lane == 0) bulk_wait_group<0>();  // bulk copies complete before the CTA exits
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync();  // no CTA leaves while the other may still arrive on or read its memory
+  } else {
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_cols);
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem_base, tmem_cols);
+    } else {
+      tmem_dealloc(tmem_base, tmem_cols);
+    }
   }
 }
 
@@ -1521,23 +1706,55 @@ static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
   *sb = 2;
 }
 
-template <int BN, bool MIRROR>
+// grid: CTAs (PAIR: an even number, two per cluster).
+template <int BN, bool MIRROR, bool PAIR>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
   const bool a_in_tmem = prm.nbr != nullptr;
+  constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns per CTA
   if (a_in_tmem) {
-    // A stages in tensor memory: the whole shared-memory budget goes to B stages
-    prm.stages_a = kTmemAStages;
-    prm.stages_b = 2;
+    // A stage s in tensor memory and B stage s in shared memory advance together: as many
+    // stages as both the free tensor-memory columns and the shared-memory budget allow
+    int sb = 2;
     for (int b = 2; b <= kMaxStages; ++b)
-      if (smem_total(conv_geometry(BN, 0, b, true)) <= 220 * 1024) prm.stages_b = b;
+      if (smem_total(conv_geometry(kBCols, 0, b, true, prm.out_tma != 0)) <= 220 * 1024) sb = b;
+    prm.stages_a = prm.stages_b = conv_tmem_a_stages(BN) < sb ? conv_tmem_a_stages(BN) : sb;
   } else {
-    pick_stages(BN, prm.taps * (prm.Kc / kBK), prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
+    pick_stages(kBCols, prm.taps * (prm.Kc / kBK), prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
   }
-  const size_t smem = smem_total(conv_geometry(BN, prm.stages_a, prm.stages_b, a_in_tmem, prm.out_tma != 0));
+  const size_t smem = smem_total(conv_geometry(kBCols, prm.stages_a, prm.stages_b, a_in_tmem, prm.out_tma != 0));
   static int done[64];
-  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR>, smem, done);
+  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR, PAIR>, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tc_conv_kernel<BN, MIRROR>, dim3(grid), dim3(kThreads), smem, s, prm);
+  if constexpr (PAIR) {
+    // no more clusters than can be resident at once (the kernel loops over tiles)
+    static int occ_smem[64], occ_clusters[64];
+    int d = 0;
+    e = cudaGetDevice(&d);
+    if (e != cudaSuccess) return e;
+    if (d < 0 || d >= 64 || occ_smem[d] != (int)smem) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, tc_conv_kernel<BN, MIRROR, PAIR>, &cfg);
+      if (e != cudaSuccess) return e;
+      if (n < 1) return cudaErrorInvalidConfiguration;
+      if (d >= 0 && d < 64) occ_smem[d] = (int)smem, occ_clusters[d] = n;
+      if (grid > 2 * n) grid = 2 * n;
+    } else if (grid > 2 * occ_clusters[d]) {
+      grid = 2 * occ_clusters[d];
+    }
+    return launch_pdl_cluster(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
+  } else
+    return launch_pdl(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, prm);
 }
 
 template <bool MIRROR>
@@ -1557,9 +1774,13 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   // A operand: halo boxes of 64 rows (gather) or the 128-row tile itself (dense)
   if (!make_rows_tmap(&prm.tmap_a, a.A, (uint64_t)a.a_rows, (uint64_t)a.lda, a.nbr ? (uint32_t)kHaloBox : (uint32_t)kBM))
     return cudaErrorInvalidValue;
+  // 256-column tiles run on CTA pairs (each CTA loads 128 of the B columns) unless the
+  // CTA budget is below two
+  const bool pair = bn == 256 && a.max_ctas != 1;
   if (!a.b_mn_major) {
     // W viewed as [w_rows][w_cols] (rows = output channels, K contiguous)
-    if (!make_rows_tmap(&prm.tmap_b, Wt, (uint64_t)w_rows, (uint64_t)w_cols, (uint32_t)bn)) return cudaErrorInvalidValue;
+    if (!make_rows_tmap(&prm.tmap_b, Wt, (uint64_t)w_rows, (uint64_t)w_cols, (uint32_t)(pair ? bn / 2 : bn)))
+      return cudaErrorInvalidValue;
   } else {
     // W [Kc rows (o)][9][N cols (i)]: dims (i, j, o), box (64, 1, 64)
     const uint64_t dims[3] = {(uint64_t)a.N, 9u, (uint64_t)a.Kc};
@@ -1567,14 +1788,15 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
     const uint32_t box[3] = {64u, 1u, 64u};
     if (!make_tmap(&prm.tmap_b, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
-  // in-place residual of a dense GEMM: the epilogue adds into out with TMA reduce-adds
-  // (out [out_rows][N], row stride ldo; boxes of 32 rows x 64 columns)
-  if (!a.nbr && a.residual && a.residual == a.out && a.N % 64 == 0 && a.out_rows > 0 && (a.ldo * 2) % 16 == 0 &&
+  // Output through TMA stores (boxes of 32 rows x 64 columns of out [out_rows][N], row
+  // stride ldo); an in-place residual (residual == out) through TMA reduce-adds.  A
+  // residual elsewhere keeps the per-thread epilogue.
+  if ((!a.residual || a.residual == a.out) && a.N % 64 == 0 && a.out_rows > 0 && (a.ldo * 2) % 16 == 0 &&
       (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0) {
     const uint64_t dims[2] = {(uint64_t)a.N, (uint64_t)a.out_rows};
     const uint64_t strides[1] = {(uint64_t)a.ldo * 2};
     const uint32_t box[2] = {64u, 32u};
-    prm.out_tma = make_tmap(&prm.tmap_out, a.out, 2, dims, strides, box) ? 1 : 0;
+    if (make_tmap(&prm.tmap_out, a.out, 2, dims, strides, box)) prm.out_tma = a.residual ? 2 : 1;
   }
   prm.A = static_cast<const __nv_bfloat16*>(a.A);
   prm.nbr = a.nbr;
@@ -1605,9 +1827,22 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   // 64 gathered channels and 64 output columns, whole-table rows: W-resident small-channel kernel
   if (a.nbr && a.Kc == 64 && a.N == 64 && bn == 64 && !a.row_lo && !a.a_abs && !a.nbr_abs && !a.out_abs)
     return a.mirror ? launch_small_inst<true>(prm, grid, s) : launch_small_inst<false>(prm, grid, s);
-  if (bn == 256) return a.mirror ? launch_conv_inst<256, true>(prm, grid, s) : launch_conv_inst<256, false>(prm, grid, s);
-  if (bn == 128) return a.mirror ? launch_conv_inst<128, true>(prm, grid, s) : launch_conv_inst<128, false>(prm, grid, s);
-  if (bn == 64) return a.mirror ? launch_conv_inst<64, true>(prm, grid, s) : launch_conv_inst<64, false>(prm, grid, s);
+  if (pair) {
+    // one cluster per 256-row tile, at most one CTA per SM
+    const int pair_tiles = ((a.M + 2 * kBM - 1) / (2 * kBM)) * (a.N / bn);
+    int clusters = sm_count() / 2;
+    if (a.max_ctas > 0 && clusters > a.max_ctas / 2) clusters = a.max_ctas / 2;
+    if (clusters > pair_tiles) clusters = pair_tiles;
+    if (clusters < 1) clusters = 1;
+    return a.mirror ? launch_conv_inst<256, true, true>(prm, 2 * clusters, s)
+                    : launch_conv_inst<256, false, true>(prm, 2 * clusters, s);
+  }
+  if (bn == 256)
+    return a.mirror ? launch_conv_inst<256, true, false>(prm, grid, s) : launch_conv_inst<256, false, false>(prm, grid, s);
+  if (bn == 128)
+    return a.mirror ? launch_conv_inst<128, true, false>(prm, grid, s) : launch_conv_inst<128, false, false>(prm, grid, s);
+  if (bn == 64)
+    return a.mirror ? launch_conv_inst<64, true, false>(prm, grid, s) : launch_conv_inst<64, false, false>(prm, grid, s);
   return cudaErrorInvalidValue;
 }
 
