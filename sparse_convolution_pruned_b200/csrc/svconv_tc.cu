@@ -72,7 +72,8 @@ __host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: ind
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
-constexpr int kTmemAStages = 4;                    // gather conv: A stages held in tensor memory
+constexpr int kTmemAStages = 4;
+constexpr int kGatherKb = 2;  // gather conv: K-blocks (of 64) per pipeline stage                    // gather conv: A stages held in tensor memory
 constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
 struct __align__(16) TcBarriers {
@@ -155,14 +156,14 @@ __host__ __device__ constexpr uint32_t pow2_cols(uint32_t c) {
 }
 __host__ __device__ constexpr uint32_t conv_tmem_cols(int bn, bool a_in_tmem, int a_stages) {
   return pow2_cols((uint32_t)(conv_acc_buffers(bn, a_in_tmem) * bn) +
-                   (a_in_tmem ? (uint32_t)(a_stages * kTmemAStageCols) : 0u));
+                   (a_in_tmem ? (uint32_t)(a_stages * kGatherKb * kTmemAStageCols) : 0u));
 }
-// Gather conv: as many A stages in tensor memory as fit next to the accumulators (an even
-// number: the two builder groups take alternate stages; at most kMaxStages).
+// Gather conv: as many stages (kGatherKb K-blocks of A each) in tensor memory as fit next
+// to the accumulators, at most kMaxStages.
 __host__ __device__ constexpr int conv_tmem_a_stages(int bn) {
-  return (512 - conv_acc_buffers(bn, true) * bn) / (int)kTmemAStageCols >= kMaxStages
+  return (512 - conv_acc_buffers(bn, true) * bn) / (int)(kGatherKb * kTmemAStageCols) >= kMaxStages
              ? kMaxStages
-             : ((512 - conv_acc_buffers(bn, true) * bn) / (int)kTmemAStageCols) & ~1;
+             : (512 - conv_acc_buffers(bn, true) * bn) / (int)(kGatherKb * kTmemAStageCols);
 }
 
 // Weight gradient: A lives in tensor memory; wgrad_slots(bn) slots of (index entries, halo).
@@ -411,11 +412,15 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
 // stage costs the issuing thread one wait and one commit.  The tensor pipe queues only a
 // few MMAs, so every cycle the issuing thread spends between MMA bursts is a cycle the pipe
 // may sit idle.  GROUP: stages whose barriers are checked before their MMAs are issued.
+// A stage holds kGatherKb K-blocks (the last stage of a tile fewer when num_kb is not a
+// multiple): A at 32-column steps in tensor memory, B at b_stage16 / kGatherKb steps.
 template <int GROUP, bool PAIR>
 __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                                  volatile int* abort_flag, int* err, uint64_t timeout_ns) {
-  for (int kb = 0; kb < num_kb; kb += GROUP) {
-    const int cnt = min(GROUP, num_kb - kb);
+  const int nst = (num_kb + kGatherKb - 1) / kGatherKb;
+  const uint32_t b_kb16 = m.b_stage16 / kGatherKb;
+  for (int q = 0; q < nst; q += GROUP) {
+    const int cnt = min(GROUP, nst - q);
     {
       int st = m.sa;
       uint32_t ps = m.pa;
@@ -429,14 +434,19 @@ __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, 
 #pragma unroll
     for (int g = 0; g < GROUP; ++g) {
       if (g >= cnt) break;
-      const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sa * m.b_stage16);
-      const uint32_t at = m.a_tmem0 + (uint32_t)m.sa * kTmemAStageCols;
+      const int kb0 = (q + g) * kGatherKb;
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k) {
-        if constexpr (PAIR)
-          tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
-        else
-          tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb + g) | k ? 1u : 0u);
+      for (int h = 0; h < kGatherKb; ++h) {
+        if (kb0 + h >= num_kb) break;
+        const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sa * m.b_stage16 + (uint32_t)h * b_kb16);
+        const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * kGatherKb + h) * kTmemAStageCols;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          if constexpr (PAIR)
+            tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+          else
+            tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+        }
       }
       if constexpr (PAIR) {
         tc_commit_pair(&bar->aempty[m.sa]);
@@ -647,7 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   const bool tma_epi = p.out_tma != 0;
   constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns this CTA loads per stage
   constexpr int kRows = PAIR ? 2 * kBM : kBM;  // output rows per tile
-  const Geometry geo = conv_geometry(kBCols, SA, SB, gather, tma_epi);
+  // gather: a B stage holds kGatherKb K-blocks (geometry counts them as wider stages)
+  const Geometry geo = conv_geometry(gather ? kBCols * kGatherKb : kBCols, SA, SB, gather, tma_epi);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -787,11 +798,67 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       }
       if (aborted && leader) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
     }
+  } else if (warp == kBWarp && gather) {
+    // ------------------------------------------------------------ weight loader (gather)
+    // B slab of K-block kb goes to slot kb % kGatherKb of stage q, on the A stages' barrier
+    // pair; the full barrier's expect_tx (rank 0) covers all slabs of the stage (both CTAs)
+    uint32_t q0 = 0;
+    bool aborted = false;
+    for (int tile = unit0; tile < num_tiles && !aborted; tile += units) {
+      const int n0 = (tile % n_tiles) * BN;
+      const int nb = n0 + (int)rank * kBCols;  // this CTA's B columns
+      int kb = 0;
+      for (int cb = 0; cb < kb_per_tap && !aborted; ++cb)
+        for (int j = 0; j < taps; ++j, ++kb) {
+          const uint32_t q = q0 + (uint32_t)(kb / kGatherKb);
+          const int half = kb % kGatherKb;
+          const int st = q % SB;
+          if (half == 0) {
+            if (!warp_wait(&bar->aempty[st], ring_parity(q, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
+              aborted = true;
+              break;
+            }
+            if (lane == 0 && leader) {
+              const uint32_t slabs = (uint32_t)min(kGatherKb, num_kb - kb);
+              mbar_arrive_expect_tx(&bar->afull[st], slabs * kBBytes * (PAIR ? 2u : 1u));
+            }
+          }
+          if (lane == 0) {
+            const uint32_t dst = smem_u32(sm.b + ((size_t)st * kGatherKb + half) * kBBytes);
+            const uint32_t fb = PAIR ? lead(&bar->afull[st]) : smem_u32(&bar->afull[st]);
+            if constexpr (!MIRROR) {
+              if constexpr (PAIR)
+                tma_load_2d_pair(dst, &p.tmap_b, fb, j * p.Kc + cb * kBK, nb);
+              else
+                tma_load_2d(dst, &p.tmap_b, &bar->afull[st], j * p.Kc + cb * kBK, nb);
+            } else {
+#pragma unroll
+              for (int g = 0; g < kBCols / 64; ++g) {
+                if constexpr (PAIR)
+                  tma_load_3d_pair(dst + g * 8192, &p.tmap_b, fb, nb + g * 64, j, cb * kBK);
+                else
+                  tma_load_3d(dst + g * 8192, &p.tmap_b, &bar->afull[st], nb + g * 64, j, cb * kBK);
+              }
+            }
+          }
+          __syncwarp();
+        }
+      q0 += (uint32_t)((num_kb + kGatherKb - 1) / kGatherKb);
+    }
+    if (aborted) {
+      // the full barriers also count the builders (or live in the other CTA): give this
+      // warp's copies in flight time to land instead of waiting on a phase
+      if (lane == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000u) {
+        }
+      }
+      __syncwarp();
+    }
   } else if (warp == kBWarp) {
-    // ------------------------------------------------------------ weight loader
-    // (gather: on the A stages' barrier pair; dense: its own ring)
-    uint64_t* const bf = gather ? bar->afull : bar->bfull;
-    uint64_t* const be = gather ? bar->aempty : bar->bempty;
+    // ------------------------------------------------------------ weight loader (dense)
+    uint64_t* const bf = bar->bfull;
+    uint64_t* const be = bar->bempty;
     uint32_t it = 0;
     bool aborted = false;
     int prev_nt = -1;
@@ -834,9 +901,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         }
     }
     if (aborted) {
-      if (gather || !leader) {
-        // the full barriers also count other producers (or live in the other CTA): give
-        // this warp's copies in flight time to land instead of waiting on a phase
+      if (!leader) {
+        // the full barriers live in the other CTA: give this warp's copies in flight time
+        // to land instead of waiting on a phase
         if (lane == 0) {
           const uint64_t t0 = globaltimer_ns();
           while (globaltimer_ns() - t0 < 200000u) {
@@ -863,10 +930,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       const int r = quarter * 32 + lane;        // the tile row this thread writes
       const uint32_t a_lane = tmem_base + ((uint32_t)(quarter * 32) << 16) + a_tmem_col;
       const uint32_t zero_row = smem_u32(bar->zero16);
-      uint32_t ti = 0, hi = 0, it = 0;
+      // stage q (counted over all tiles) holds K-blocks kGatherKb * (q - q0) .. of the tile
+      // that starts at stage q0; builder group q & 1 writes it
+      uint32_t ti = 0, hi = 0, q0 = 0;
       bool aborted = false;
       for (int tile = unit0; tile < num_tiles && !aborted; tile += units, ++ti) {
         const int slot = ti & 1;
+        int kb = 0;  // K-block within the tile
         if (!warp_wait(&bar->ifull[slot], ring_parity(ti, 2), abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
@@ -882,15 +952,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             break;
           }
           const uint32_t halo = smem_u32(sm.halo + hb * kHaloBufBytes);
-          for (int j = 0; j < 9; ++j, ++it) {
-            if ((int)(it & 1u) != grp) continue;
+          for (int j = 0; j < 9; ++j, ++kb) {
+            const uint32_t q = q0 + (uint32_t)(kb / kGatherKb);
+            if ((int)(q & 1u) != grp) continue;
+            const int half = kb % kGatherKb;  // slab of the stage
+            const bool stage_done = half == kGatherKb - 1 || kb == num_kb - 1;
             const int jj = MIRROR ? 8 - j : j;
-            const int sa = it % SA;
-            if (!warp_wait(&bar->aempty[sa], ring_parity(it, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
-              aborted = true;
-              break;
+            const int sa = q % SA;
+            if (half == 0) {
+              if (!warp_wait(&bar->aempty[sa], ring_parity(q, SA) ^ 1u, abort_flag, err, p.timeout_ns)) {
+                aborted = true;
+                break;
+              }
+              tc_fence_after();  // the MMAs that read this stage are complete
             }
-            tc_fence_after();  // the MMAs that read this stage are complete
             // branch-free row selection: halo row, or the zero row for a missing neighbour;
             // rows outside the halo window are read from global memory behind a warp vote
             const int raw = row_ok ? ld_shared_s32(sidx_s + 4u * (uint32_t)(r * 9 + jj)) : -1;
@@ -919,14 +994,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
                 }
               }
             }
-            tmem_st_32x32b_x32(a_lane + (uint32_t)sa * kTmemAStageCols, v);
-            tmem_st_wait();
-            tc_fence_before();
-            if (PAIR && !leader) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(lead(&bar->afull[sa]));
-            } else {
-              warp_arrive(&bar->afull[sa]);
+            tmem_st_32x32b_x32(a_lane + (uint32_t)(sa * kGatherKb + half) * kTmemAStageCols, v);
+            if (stage_done) {
+              tmem_st_wait();
+              tc_fence_before();
+              if (PAIR && !leader) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(lead(&bar->afull[sa]));
+              } else {
+                warp_arrive(&bar->afull[sa]);
+              }
             }
           }
           if (!aborted) {
@@ -934,6 +1011,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
             ++hi;
           }
         }
+        q0 += (uint32_t)((num_kb + kGatherKb - 1) / kGatherKb);
         if (!aborted) warp_arrive(&bar->iempty[slot]);
       }
     }
@@ -948,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       } else {
         c.b_lbo = 16, c.b_sbo = 1024, c.b_step = 32;
       }
-      MmaIssuer mi = make_issuer(sm, kBBytes, SA, SB, c);
+      MmaIssuer mi = make_issuer(sm, gather ? kGatherKb * kBBytes : kBBytes, SA, SB, c);
       mi.a_tmem0 = tmem_base + a_tmem_col;
       uint32_t tc = 0;
       bool issued = false;
@@ -1716,12 +1794,14 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
     // stages as both the free tensor-memory columns and the shared-memory budget allow
     int sb = 2;
     for (int b = 2; b <= kMaxStages; ++b)
-      if (smem_total(conv_geometry(kBCols, 0, b, true, prm.out_tma != 0)) <= 220 * 1024) sb = b;
+      if (smem_total(conv_geometry(kBCols * kGatherKb, 0, b, true, prm.out_tma != 0)) <= 220 * 1024) sb = b;
     prm.stages_a = prm.stages_b = conv_tmem_a_stages(BN) < sb ? conv_tmem_a_stages(BN) : sb;
   } else {
     pick_stages(kBCols, prm.taps * (prm.Kc / kBK), prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
   }
-  const size_t smem = smem_total(conv_geometry(kBCols, prm.stages_a, prm.stages_b, a_in_tmem, prm.out_tma != 0));
+  // (the same geometry the kernel carves: gather B stages hold kGatherKb K-blocks)
+  const size_t smem = smem_total(conv_geometry(a_in_tmem ? kBCols * kGatherKb : kBCols, prm.stages_a, prm.stages_b,
+                                               a_in_tmem, prm.out_tma != 0));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR, PAIR>, smem, done);
   if (e != cudaSuccess) return e;
