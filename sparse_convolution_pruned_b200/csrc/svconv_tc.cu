@@ -72,8 +72,8 @@ __host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: ind
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
-constexpr int kTmemAStages = 4;
-constexpr int kGatherKb = 2;  // gather conv: K-blocks (of 64) per pipeline stage                    // gather conv: A stages held in tensor memory
+constexpr int kTmemAStages = 4;                    // weight gradient: A stages held in tensor memory
+constexpr int kGatherKb = 2;                       // gather conv: K-blocks (of 64) per pipeline stage
 constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
 struct __align__(16) TcBarriers {
@@ -412,13 +412,13 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
 // stage costs the issuing thread one wait and one commit.  The tensor pipe queues only a
 // few MMAs, so every cycle the issuing thread spends between MMA bursts is a cycle the pipe
 // may sit idle.  GROUP: stages whose barriers are checked before their MMAs are issued.
-// A stage holds kGatherKb K-blocks (the last stage of a tile fewer when num_kb is not a
-// multiple): A at 32-column steps in tensor memory, B at b_stage16 / kGatherKb steps.
-template <int GROUP, bool PAIR>
+// A stage holds KBS K-blocks (the last stage of a tile fewer when num_kb is not a
+// multiple): A at 32-column steps in tensor memory, B at b_stage16 / KBS steps.
+template <int GROUP, bool PAIR, int KBS = kGatherKb>
 __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                                  volatile int* abort_flag, int* err, uint64_t timeout_ns) {
-  const int nst = (num_kb + kGatherKb - 1) / kGatherKb;
-  const uint32_t b_kb16 = m.b_stage16 / kGatherKb;
+  const int nst = (num_kb + KBS - 1) / KBS;
+  const uint32_t b_kb16 = m.b_stage16 / KBS;
   for (int q = 0; q < nst; q += GROUP) {
     const int cnt = min(GROUP, nst - q);
     {
@@ -434,12 +434,12 @@ __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, 
 #pragma unroll
     for (int g = 0; g < GROUP; ++g) {
       if (g >= cnt) break;
-      const int kb0 = (q + g) * kGatherKb;
+      const int kb0 = (q + g) * KBS;
 #pragma unroll
-      for (int h = 0; h < kGatherKb; ++h) {
+      for (int h = 0; h < KBS; ++h) {
         if (kb0 + h >= num_kb) break;
         const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sa * m.b_stage16 + (uint32_t)h * b_kb16);
-        const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * kGatherKb + h) * kTmemAStageCols;
+        const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * KBS + h) * kTmemAStageCols;
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           if constexpr (PAIR)
@@ -1036,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, n_acc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        constexpr int kGroup = 2;
+        constexpr int kGroup = 1;
         bool ok;
         if (gather) {
           ok = mma_tile_unified<kGroup, PAIR>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
