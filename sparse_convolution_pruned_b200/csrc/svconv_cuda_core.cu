@@ -201,9 +201,75 @@ cudaError_t launch_f32_wgrad_partials(const float* dY, const float* X, const int
   return cudaGetLastError();
 }
 
+// The same reduction with four adjacent output channels per thread (16-byte loads of the
+// partials, up to 8 splits in flight per load batch).  The sum is bound by how many bytes
+// are in flight, and at one channel per thread the kernel's register use caps it at a few
+// MB across the GPU; four channels per thread carry four times as many.  Each element gets
+// the same compensated sum over the splits in the same order as in wgrad_reduce_kernel, so
+// the results are bitwise identical.  Needs Cout % 4 == 0 (16-byte aligned rows).
+template <int CW>  // output channels per block
+__global__ void __launch_bounds__(256) wgrad_reduce4_kernel(const float* __restrict__ partial, int splits,
+                                                            int rows_pad, int Cin, int Cout, int grouped,
+                                                            float* __restrict__ dW, float* __restrict__ db) {
+  constexpr int kLanesPerRow = CW / 4;
+  constexpr int kRows = 256 / kLanesPerRow;  // partial rows per block
+  __shared__ float tile[kRows][CW + 1];
+  pdl_wait();  // the partials come from the kernel before this one
+  pdl_trigger();
+  const int rows = 9 * Cin + 1;
+  const int m0 = blockIdx.x * kRows, o0 = blockIdx.y * CW;
+  const int r = threadIdx.x / kLanesPerRow, cl = threadIdx.x % kLanesPerRow;
+  const int m = m0 + r, o = o0 + 4 * cl;
+  Dot2 acc[4];
+  if (m < rows && o < Cout) {
+    int pm = m;
+    if (grouped) {
+      const int j = m / Cin, i = m - j * Cin;
+      pm = m == 9 * Cin ? 9 * 64 : ((i >> 6) * 10 + j) * 64 + (i & 63);
+    }
+    const size_t stride4 = (size_t)rows_pad * Cout / 4;
+    const float4* src = reinterpret_cast<const float4*>(partial + (size_t)pm * Cout + o);
+    for (int sp0 = 0; sp0 < splits; sp0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        v[q] = (sp0 + q < splits) ? __ldg(src + (size_t)(sp0 + q) * stride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (sp0 + q < splits) {
+          acc[0].add(v[q].x);
+          acc[1].add(v[q].y);
+          acc[2].add(v[q].z);
+          acc[3].add(v[q].w);
+        }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tile[r][4 * cl + k] = acc[k].value();
+  __syncthreads();
+  // write: consecutive threads take consecutive rows of one output channel
+  for (int e = threadIdx.x; e < CW * kRows; e += 256) {
+    const int oc = e / kRows, rr = e - oc * kRows;
+    const int oo = o0 + oc, mm = m0 + rr;
+    if (oo < Cout) {
+      const float v = tile[rr][oc];
+      if (mm < 9 * Cin)
+        dW[(size_t)oo * 9 * Cin + mm] = v;
+      else if (mm == 9 * Cin && db)
+        db[oo] = v;
+    }
+  }
+}
+
 cudaError_t launch_wgrad_reduce(const float* partial, int splits, int rows_pad, int Cin, int Cout, int grouped,
                                 float* dW, float* db, cudaStream_t s) {
   const int rows = 9 * Cin + 1;
+  if (Cout >= 128 && Cout % 4 == 0 && (reinterpret_cast<uintptr_t>(partial) & 15u) == 0) {
+    constexpr int kCW = 128, kRows = 256 / (kCW / 4);
+    dim3 grid((rows + kRows - 1) / kRows, (Cout + kCW - 1) / kCW);
+    return launch_pdl(wgrad_reduce4_kernel<kCW>, grid, dim3(256), 0, s, partial, splits, rows_pad, Cin, Cout, grouped,
+                      dW, db);
+  }
   dim3 grid((rows + kRedRows - 1) / kRedRows, (Cout + 31) / 32);
   return launch_pdl(wgrad_reduce_kernel, grid, dim3(256), 0, s, partial, splits, rows_pad, Cin, Cout, grouped, dW, db);
 }
