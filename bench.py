@@ -643,7 +643,7 @@ def run_adapter(args):
         ad_work = {"bytes": 2 * n * D * 2 + 36 * n + 2 * (2 * D * R + 9 * R * R), "flops": flops}
         roof = roofline_entry("adapter_fwd", ad_work, ad_ms, peaks)
         roof["kernel"] = f"adapter_fwd ({3 * n_chunks} tcgen05 GEMM launches, timed together)"
-        roof["traffic"] = None
+        roof["traffic"] = kernel_traffic(args.workload, "adapter_fwd")  # DRAM bytes of the 18 launches
         roof["peak_source"] = peaks["source"]
         idx_work = algorithmic_work(n, T, R, R)["build_index"]
         tokens = n * world
