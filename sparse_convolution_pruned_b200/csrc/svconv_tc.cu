@@ -263,27 +263,9 @@ __device__ __forceinline__ void copy_index_entries(uint32_t dst, const int32_t* 
   }
 }
 
-// Writers of generic shared memory publish a stage to the async proxy (the MMA).
-__device__ __forceinline__ void warp_publish(uint64_t* bar) {
-  fence_proxy_async_smem();
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
-__device__ __forceinline__ int warp_min(int v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ int warp_max(int v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
 }
 
 __device__ __forceinline__ uint4 ldg_16(const void* p) {
