@@ -105,6 +105,7 @@ struct TcConvParams {
   int M, a_abs, nbr_abs, out_abs, N;
   int gelu, ldo, out_rows, stages_a, stages_b;
   int out_tma;  // 1: the epilogue writes out with TMA stores; 2: adds into out (residual == out) with TMA reduce-adds
+  int dense_pair_ring;  // dense, B not resident: A and B stage s on one barrier pair (stages_a == stages_b)
 };
 
 struct TcWgradParams {
@@ -396,9 +397,11 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
 // may sit idle.  GROUP: stages whose barriers are checked before their MMAs are issued.
 // A stage holds KBS K-blocks (the last stage of a tile fewer when num_kb is not a
 // multiple): A at 32-column steps in tensor memory, B at b_stage16 / KBS steps.
-template <int GROUP, bool PAIR, int KBS = kGatherKb>
+// A_TMEM = false: dense GEMM, A stage s in shared memory as well (one K-block per stage).
+template <int GROUP, bool PAIR, int KBS = kGatherKb, bool A_TMEM = true>
 __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                                  volatile int* abort_flag, int* err, uint64_t timeout_ns) {
+  static_assert(A_TMEM || KBS == 1, "dense stages hold one K-block");
   const int nst = (num_kb + KBS - 1) / KBS;
   const uint32_t b_kb16 = m.b_stage16 / KBS;
   for (int q = 0; q < nst; q += GROUP) {
@@ -412,7 +415,7 @@ __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, 
         if (++st == m.SA) st = 0, ps ^= 1u;
       }
     }
-    tc_fence_after();  // the A stages were written to tensor memory by other threads
+    if constexpr (A_TMEM) tc_fence_after();  // the A stages were written to tensor memory by other threads
 #pragma unroll
     for (int g = 0; g < GROUP; ++g) {
       if (g >= cnt) break;
@@ -421,13 +424,26 @@ __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, 
       for (int h = 0; h < KBS; ++h) {
         if (kb0 + h >= num_kb) break;
         const uint64_t bd = m.b_desc0 + (uint64_t)((uint32_t)m.sa * m.b_stage16 + (uint32_t)h * b_kb16);
-        const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * KBS + h) * kTmemAStageCols;
+        if constexpr (A_TMEM) {
+          const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * KBS + h) * kTmemAStageCols;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          if constexpr (PAIR)
-            tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
-          else
-            tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k) {
+            if constexpr (PAIR)
+              tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+            else
+              tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+          }
+        } else {
+          const uint64_t ad = m.a_desc0 + (uint64_t)((uint32_t)m.sa * m.a_stage16);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            if constexpr (PAIR)
+              tc_mma_bf16_pair(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc,
+                               (kb0 + h) | k ? 1u : 0u);
+            else
+              tc_mma_bf16(d, ad + (uint64_t)(k * m.a_k16), bd + (uint64_t)(k * m.b_k16), m.idesc,
+                          (kb0 + h) | k ? 1u : 0u);
+          }
         }
       }
       if constexpr (PAIR) {
@@ -677,8 +693,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     // afull: one builder group per A stage; ifull: the loader lanes' 32 cp.async arrivals + lane 0's expect_tx
     // gather: afull / aempty serve A and B stage s together (SA == SB); afull counts the
     // builder warps (of both CTAs of a pair) and the weight loader's expect_tx arrival
-    init_barriers(bar, SA, SB, gather ? (PAIR ? kProdWarps : kProdWarps / 2) + 1 : 1, 2, 33, kProdWarps,
-                  PAIR ? 2 * kEpiWarps : kEpiWarps);
+    // dense with dense_pair_ring: afull counts the A and the B loader's expect_tx arrivals
+    init_barriers(bar, SA, SB, gather ? (PAIR ? kProdWarps : kProdWarps / 2) + 1 : (p.dense_pair_ring ? 2 : 1), 2,
+                  33, kProdWarps, PAIR ? 2 * kEpiWarps : kEpiWarps);
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
   }
@@ -793,7 +810,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
           __syncwarp();
         }
       }
-      if (aborted && leader) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
+      if (aborted && leader && !p.dense_pair_ring) drain_ring(bar->afull, it, SA, err, p.timeout_ns);
+      if (aborted && (p.dense_pair_ring || !leader)) {
+        // the full barriers also count the other loader (or live in the other CTA): give this
+        // warp's copies in flight time to land instead of waiting on a phase
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000u) {
+          }
+        }
+        __syncwarp();
+      }
     }
   } else if (warp == kBWarp && gather) {
     // ------------------------------------------------------------ weight loader (gather)
@@ -854,8 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     }
   } else if (warp == kBWarp) {
     // ------------------------------------------------------------ weight loader (dense)
-    uint64_t* const bf = bar->bfull;
-    uint64_t* const be = bar->bempty;
+    uint64_t* const bf = p.dense_pair_ring ? bar->afull : bar->bfull;
+    uint64_t* const be = p.dense_pair_ring ? bar->aempty : bar->bempty;
     uint32_t it = 0;
     bool aborted = false;
     int prev_nt = -1;
@@ -898,9 +925,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         }
     }
     if (aborted) {
-      if (!leader) {
-        // the full barriers live in the other CTA: give this warp's copies in flight time
-        // to land instead of waiting on a phase
+      if (!leader || p.dense_pair_ring) {
+        // the full barriers live in the other CTA or also count the A loader: give this
+        // warp's copies in flight time to land instead of waiting on a phase
         if (lane == 0) {
           const uint64_t t0 = globaltimer_ns();
           while (globaltimer_ns() - t0 < 200000u) {
@@ -1045,6 +1072,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
           prev_nt = nt;
           ok = mma_tile_resident_b<PAIR>(bar, mi, num_kb, tmem_base + ab * BN, b_load, b_last, abort_flag, err,
                                          p.timeout_ns);
+        } else if (p.dense_pair_ring) {
+          ok = mma_tile_unified<1, PAIR, 1, false>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err,
+                                                   p.timeout_ns);
         } else {
           ok = mma_tile<false, kGroup, PAIR>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
         }
@@ -1794,7 +1824,16 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
       if (smem_total(conv_geometry(kBCols * kGatherKb, 0, b, true, prm.out_tma != 0)) <= 220 * 1024) sb = b;
     prm.stages_a = prm.stages_b = conv_tmem_a_stages(BN) < sb ? conv_tmem_a_stages(BN) : sb;
   } else {
-    pick_stages(kBCols, prm.taps * (prm.Kc / kBK), prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
+    const int num_kb = prm.taps * (prm.Kc / kBK);
+    pick_stages(kBCols, num_kb, prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
+    if (num_kb > prm.stages_b) {
+      // B streams: A stage s and B stage s on one barrier pair, as many stages as fit
+      int st = 2;
+      for (int b = 2; b <= kMaxStages; ++b)
+        if (smem_total(conv_geometry(kBCols, b, b, false, prm.out_tma != 0)) <= 220 * 1024) st = b;
+      prm.stages_a = prm.stages_b = st;
+      prm.dense_pair_ring = 1;
+    }
   }
   // (the same geometry the kernel carves: gather B stages hold kGatherKb K-blocks)
   const size_t smem = smem_total(conv_geometry(a_in_tmem ? kBCols * kGatherKb : kBCols, prm.stages_a, prm.stages_b,
