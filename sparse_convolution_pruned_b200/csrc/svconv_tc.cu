@@ -45,6 +45,7 @@
 
 #include <climits>
 #include <cstring>
+#include <mutex>
 
 #include "svconv_internal.h"
 #include "svconv_ptx.cuh"
@@ -1843,10 +1844,14 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
   if (e != cudaSuccess) return e;
   if constexpr (PAIR) {
     // no more clusters than can be resident at once (the kernel loops over tiles)
+    // per device: resident clusters at this shared-memory size (queried once; host threads may
+    // launch concurrently)
     static int occ_smem[64], occ_clusters[64];
+    static std::mutex occ_mu;
     int d = 0;
     e = cudaGetDevice(&d);
     if (e != cudaSuccess) return e;
+    std::unique_lock<std::mutex> lk(occ_mu);
     if (d < 0 || d >= 64 || occ_smem[d] != (int)smem) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(grid);
@@ -1868,6 +1873,7 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
     } else if (grid > 2 * occ_clusters[d]) {
       grid = 2 * occ_clusters[d];
     }
+    lk.unlock();
     return launch_pdl_cluster(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
   } else
     return launch_pdl(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, prm);
