@@ -112,12 +112,14 @@ struct TcConvParams {
 struct TcWgradParams {
   CUtensorMap tmap_x;   // X [n][Cin], halo boxes {64, 64}
   CUtensorMap tmap_dy;  // dY [n][Cout], box {64, 64}
+  CUtensorMap tmap_part;  // part_tma: partial [splits * rows_pad][Cout] fp32, box {32, 32}
   const __nv_bfloat16* X;
   const int32_t* nbr;
   float* partial;
   int* status;
   unsigned long long timeout_ns;
   int n, Cin, Cout, splits, rows_pad, stages_a, stages_b;
+  int part_tma;  // the last unit of a CTA writes its partial rows with TMA stores
 };
 
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
@@ -1692,25 +1694,57 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       tc_fence_after();
       const int row = mt * kBM + warp * 32 + lane;
       float* dst = p.partial + ((size_t)sp * p.rows_pad + row) * p.Cout + n0;
+      // The CTA's last unit: its MMAs are done and no dY tile will be loaded any more, so the
+      // dY ring is free and stages the partial rows for TMA stores (whole lines, no per-thread
+      // row stores); other units store their rows directly.
+      if (p.part_tma && u + (int)gridDim.x >= num_units) {
+        const uint32_t boxes = smem_u32(sm.b) + (uint32_t)warp * 2u * 4096u;
+        const uint32_t sw = (uint32_t)(lane & 7);
+        const int prow0 = sp * p.rows_pad + mt * kBM + warp * 32;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
-        tmem_ld_wait();
-        float4* o4 = reinterpret_cast<float4*>(dst + c0);
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
+          const uint32_t box = boxes + (uint32_t)((c0 / 32) & 1) * 4096u;
+          if (lane == 0) bulk_wait_group_read<1>();  // the store issued from this box two boxes ago has read it
+          __syncwarp();
+          tmem_ld_wait();
+          // row `lane` of the box: 16-byte chunk k lands at chunk k ^ (lane & 7) (128-byte swizzle)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 w;
-          w.x = empty_range ? 0.f : __uint_as_float(v[4 * q]);
-          w.y = empty_range ? 0.f : __uint_as_float(v[4 * q + 1]);
-          w.z = empty_range ? 0.f : __uint_as_float(v[4 * q + 2]);
-          w.w = empty_range ? 0.f : __uint_as_float(v[4 * q + 3]);
-          o4[q] = w;
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t a0 = empty_range ? 0u : v[4 * k], a1 = empty_range ? 0u : v[4 * k + 1];
+            const uint32_t a2 = empty_range ? 0u : v[4 * k + 2], a3 = empty_range ? 0u : v[4 * k + 3];
+            st_shared_16(box + (uint32_t)lane * 128u + (((uint32_t)k ^ sw) << 4), a0, a1, a2, a3);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tmap_part, box, n0 + c0, prow0);
+            bulk_commit_group();
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN + c0, v);
+          tmem_ld_wait();
+          float4* o4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 w;
+            w.x = empty_range ? 0.f : __uint_as_float(v[4 * q]);
+            w.y = empty_range ? 0.f : __uint_as_float(v[4 * q + 1]);
+            w.z = empty_range ? 0.f : __uint_as_float(v[4 * q + 2]);
+            w.w = empty_range ? 0.f : __uint_as_float(v[4 * q + 3]);
+            o4[q] = w;
+          }
         }
       }
       tc_fence_before();
       warp_arrive(&bar->tempty[ab]);
     }
+    if (p.part_tma && lane == 0) bulk_wait_group<0>();  // partial-row stores complete before the CTA exits
   }
 
   tc_fence_before();
@@ -1756,7 +1790,7 @@ static EncodeTiledFn encode_fn() {
 // bf16 tensor map with 128-byte swizzle and zero fill outside the tensor;
 // dims / strides innermost first (strides in bytes, rank-1 of them).
 static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-                      const uint32_t* box) {
+                      const uint32_t* box, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[3], gs[2];
@@ -1766,7 +1800,7 @@ static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t
     bx[i] = box[i];
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -1989,6 +2023,13 @@ void tc_wgrad_plan_ctas(int n, int Cin, int Cout, int ctas, int* splits, int* ro
 
 template <int BN>
 static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t s) {
+  // partial rows [splits * rows_pad][Cout] fp32 through TMA stores (boxes of 32 rows x 32 columns)
+  if ((reinterpret_cast<uintptr_t>(prm.partial) & 15u) == 0 && prm.Cout % 32 == 0) {
+    const uint64_t dims[2] = {(uint64_t)prm.Cout, (uint64_t)prm.splits * prm.rows_pad};
+    const uint64_t strides[1] = {(uint64_t)prm.Cout * 4};
+    const uint32_t box[2] = {32u, 32u};
+    prm.part_tma = make_tmap(&prm.tmap_part, prm.partial, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 1 : 0;
+  }
   prm.stages_a = kTmemAStages;
   prm.stages_b = 2;
   for (int b = 2; b <= kMaxStages; ++b)
