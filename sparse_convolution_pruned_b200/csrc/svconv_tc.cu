@@ -20,26 +20,36 @@
 //
 // Warp roles (480 threads):
 //   warps 0-3    epilogue: tcgen05.ld the fp32 accumulator (warp w owns TMEM
-//                lanes 32w..32w+31 = tile rows), bias / GELU / residual, bf16 store.
-//   warps 4-11   A builders: copy each tile row's neighbour segment from the halo
-//                into the 128B-swizzled K-major A stage (zeros for -1 = padding).
-//   warp 12      index / halo loader: cp.async of the tile's neighbour entries and
-//                the halo window's TMA boxes (or, for the dense adapter
+//                lanes 32w..32w+31 = tile rows), bias / GELU, bf16 boxes staged in
+//                shared memory and written by TMA stores (an in-place residual by TMA
+//                reduce-adds); rows of a ragged last tile are stored per thread.
+//   warps 4-11   A builders (gather): copy each tile row's neighbour segment from the
+//                halo (zeros for -1 = padding) straight into the tensor-memory A stage
+//                with tcgen05.st; idle in dense mode.
+//   warp 12      index / halo loader: cp.async / bulk copy of the tile's neighbour
+//                entries and the halo window's TMA boxes (or, for the dense adapter
 //                projections, TMA of the A tile itself).
 //   warp 13      weight loader: TMA of the B tile (W_j, or W_j^T straight from
 //                W[o][j][i] as an MN-major operand for the data gradient).
-//   warp 14      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN, K=16) into
-//                a double-buffered TMEM accumulator; tcgen05.commit frees stages.
+//   warp 14      MMA issuer: one thread issues tcgen05.mma (K=16) into a TMEM
+//                accumulator and tcgen05.commit frees stages.  A gather stage holds two
+//                64-deep K-blocks, and A stage s and B stage s share one full / empty
+//                barrier pair, so the issuer waits and commits once per 8 MMAs.
+//
+// 256-column tiles run on CTA pairs (clusters of 2, cta_group::2): M = 256 MMAs over
+// both SMs' tensor memory, issued by CTA rank 0; each CTA gathers its own 128 rows and
+// loads half of B, and rank 0's barriers count both CTAs' producers.
 //
 // The data gradient is the same kernel: the gather goes through the mirrored
 // column N[k][8-j] of dY.  The weight gradient dW^T[(j,i)][o] = sum_k X[N[k,j]][i]
-// dY[k][o] is a GEMM with K = tokens, A (gathered X, MN-major, assembled from a
-// halo per 64-token block) and B (dY by TMA, MN-major).  The bias gradient comes
-// out of the same MMAs: the A row after the last (j, i) row is 1 for every valid
-// token, so its accumulator row is sum_k dY[k][o].  Token ranges are split over
-// CTAs into fp32 partials, reduced afterwards in a fixed order.
+// dY[k][o] is a GEMM with K = tokens, A (gathered X, transposed into tensor memory,
+// assembled from a halo per 64-token block) and B (dY by TMA, MN-major).  The bias
+// gradient comes out of the same MMAs: the A row after the last (j, i) row is 1 for
+// every valid token, so its accumulator row is sum_k dY[k][o].  Token ranges are split
+// over CTAs into fp32 partials, reduced afterwards in a fixed order.
 //
-// No TMA multicast is used anywhere.
+// No TMA or bulk load uses cluster multicast; the only multicast is tcgen05.commit's
+// arrival on the barriers of both CTAs of a pair.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
