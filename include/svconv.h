@@ -97,6 +97,9 @@ SVCONV_API int svconv_build_index(const int32_t* coords, const int32_t* frame_of
  *   X [n][Cin], Y [n][Cout] of dtype; Wt [Cout][9][Cin] of dtype;
  *   bias [Cout] fp32 device or NULL.  Y must not alias X.
  *   fp32 limit: 9*Cin*Cout <= 49152.  bf16: Cin, Cout multiples of 64, Cout <= 4096.
+ *   bf16 launches: persistent, at most one CTA per SM; output tiles of 256 columns run on
+ *   clusters of two CTAs (a pair of SMs shares each 256-row tile), so the device must
+ *   allow 2-CTA clusters for those shapes.
  */
 SVCONV_API int svconv_fwd(int dtype, const void* X, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt,
                const float* bias, void* Y, void* stream);
