@@ -312,11 +312,12 @@ def test_adapter_small_full(sv, orc):
     check_bf16(out - a.X, ref - a.X, "adapter delta")
 
 
-def test_adapter_long_video_config(sv, orc):
+@pytest.mark.parametrize("chunk_T", [512, 1024])  # 1024: the chunking bench.py times
+def test_adapter_long_video_config(sv, orc, chunk_T):
     torch.cuda.reset_peak_memory_stats()
     a = wl.adapter_bf16()
     ref_n, _, _ = orc.build_index(a.coords, a.frame_off, a.T, a.H, a.W, want_map=False)
-    out = adapter_gpu(sv, a, chunk_T=512)
+    out = adapter_gpu(sv, a, chunk_T=chunk_T)
     peak = torch.cuda.max_memory_allocated()
     assert peak <= 1 << 30, f"peak {peak / 2**20:.0f} MiB"
     out = out.float().cpu().numpy()
