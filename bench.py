@@ -1,25 +1,36 @@
-"""Benchmark: SparseConv2D fwd+bwd step on B200 through the svconv C ABI.
-
-One step = the whole hot path on one batch of pruned tokens, the small-channel
-adapter convolution workload (T=384 token-frames, 16x16 patch grid, top-77
-blob-saliency keep per frame, C_in=C_out=64, bf16 with fp32 accumulation):
-    neighbour-index build -> forward -> data gradient -> weight/bias gradient
-(and, with --gpus N > 1, an NCCL all-reduce of dW/db: data-parallel weak scaling,
-every rank owning its own batch of frames).
+"""Benchmark: SparseConv2D on B200 through the svconv C ABI, every workload in one run.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME] [--no-cpu-baseline] [--sustained-s S]
 
-Timing: each step is replayed from a CUDA graph, the 126 MB L2 is flushed by a
-256 MiB write between steps (the workload's 8.7 MB would otherwise stay in L2),
-and only the step is inside the CUDA-event region.  The roofline object is for
-the step's slowest kernel, timed by events around each kernel on the launching
-stream in a second pass.  ``--impl reference`` times the CPU oracle instead.
+Workloads (the five SparseConv2D configurations, synthetic seeded inputs):
+  tiny_f32     T=4, 8x8 grid, 32 kept per frame, C=16, fp32 (fwd + bwd)
+  small_c      T=384, 16x16, top-77 blob-saliency keep, C=64, bf16 (fwd + bwd)
+  large_c_fwd  T=384, 16x16, keep 50%, C=256, bf16 + fp32 bias (fwd)
+  large_c_bwd  T=384, 16x16, keep U(0.2, 0.8) per frame, C=256, bf16 (fwd + bwd)
+  adapter      T=3072 token frames, 16x16, keep 36%, Linear 1024->256, SparseConv 256->256,
+               GELU, Linear 256->1024 + residual, chunked over frames (fwd)
+
+One step is one pass of the workload's whole path over its batch: neighbour-index build ->
+forward [-> data gradient -> weight / bias gradient] (adapter: index build -> chunked adapter
+forward).  The headline (top-level ``value``) is the largest fwd+bwd configuration that fits
+one GPU, ``large_c_bwd``; with N = 1 every workload is also reported under ``configs`` with its
+own roofline (dominant kernel), per-kernel times, end-to-end leg, CPU-oracle baseline and a
+sustained leg (>= 1 s of back-to-back graph replays with its own clock samples).  With N > 1
+(torchrun, NCCL) each rank runs its own batch of the headline workload (weak scaling) and the
+weight / bias gradients are all-reduced.
+
+Timing: steps are replayed from CUDA graphs and timed with CUDA events on the launching
+stream; the 126 MB L2 is flushed by a 256 MiB write between timed steps (outside the events)
+for the conv workloads, whose working sets fit in L2; the adapter's in-place X (579 MB) is
+larger than L2 and is not flushed.  ``--impl reference`` times the CPU oracle instead.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -33,8 +44,21 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SparseConv2D kept-tokens/sec (fwd, fwd+bwd) and % of roofline on 1 B200"
 UNIT = "kept-tokens/s"
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops (FMA) x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FLUSH_BYTES = 256 << 20
+
+# name: (generator in workloads.py, base seed, step kind, compute dtype)
+WORKLOADS = {
+    "tiny_f32": ("tiny_f32", 0, "fwd+bwd", "f32"),
+    "small_c": ("small_c_bf16", 1, "fwd+bwd", "bf16"),
+    "large_c_fwd": ("large_c_fwd_bf16", 2, "fwd", "bf16"),
+    "large_c_bwd": ("large_c_bwd_bf16", 3, "fwd+bwd", "bf16"),
+    "adapter": ("adapter_bf16", 4, "adapter", "bf16"),
+}
+ORDER = ["tiny_f32", "small_c", "large_c_fwd", "large_c_bwd", "adapter"]
+HEADLINE = "large_c_bwd"
 
 
 def load_peaks():
@@ -44,35 +68,57 @@ def load_peaks():
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
-    return {"hbm_gbs": FALLBACK_PEAKS["hbm_gbs"], "bf16_tflops": FALLBACK_PEAKS["bf16_tflops"],
-            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+    return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def algorithmic_work(n, T, Cin, Cout):
-    """Per-launch algorithmic bytes and flops (unique data touched once)."""
-    bf = 2
+def make_inputs(key, seed_offset=0):
+    from sparse_convolution_pruned_b200 import workloads as wl
+    gen, seed, _, _ = WORKLOADS[key]
+    return getattr(wl, gen)(seed=seed + seed_offset)
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def conv_work(n, T, Cin, Cout, elem, bias):
+    """Per-launch algorithmic bytes and flops: unique data touched once (features, the
+    neighbour table at 36 B per token, weights, bias, fp32 weight gradients)."""
     nbr = 36 * n
-    w_bytes = 9 * Cin * Cout * bf
+    w_bytes = 9 * Cin * Cout * elem
+    fl = 2 * n * 9 * Cin * Cout
     return {
         "build_index": {"bytes": 12 * n + 4 * (T + 1) + nbr, "flops": 0},
-        "fwd": {"bytes": n * Cin * bf + n * Cout * bf + nbr + w_bytes, "flops": 2 * n * 9 * Cin * Cout},
-        "bwd_data": {"bytes": n * Cout * bf + n * Cin * bf + nbr + w_bytes, "flops": 2 * n * 9 * Cin * Cout},
-        "bwd_weight": {"bytes": n * Cout * bf + n * Cin * bf + nbr + 4 * (9 * Cin * Cout + Cout),
-                       "flops": 2 * n * 9 * Cin * Cout},
+        "fwd": {"bytes": n * (Cin + Cout) * elem + nbr + w_bytes + (4 * Cout if bias else 0), "flops": fl},
+        "bwd_data": {"bytes": n * (Cin + Cout) * elem + nbr + w_bytes, "flops": fl},
+        "bwd_weight": {"bytes": n * (Cin + Cout) * elem + nbr + 4 * (9 * Cin * Cout + Cout), "flops": fl},
     }
 
 
-def roofline_entry(name, work, ms, peaks):
+def adapter_work(n, D, R):
+    return {"bytes": 2 * n * D * 2 + 36 * n + 2 * (2 * D * R + 9 * R * R),
+            "flops": 2 * n * (D * R + 9 * R * R + R * D)}
+
+
+def floor_seconds(work, peaks, alu=False):
+    t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    peak_fl = FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"]
+    t_fl = work["flops"] / (peak_fl * 1e12) if work["flops"] else 0.0
+    return max(t_mem, t_fl)
+
+
+def roofline_entry(work, ms, peaks, alu=False):
+    """The larger of the byte floor (HBM) and the flop floor (bf16 tensor, or fp32 ALU)."""
     sec = ms * 1e-3
-    t_hbm = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = work["flops"] / (peaks["bf16_tflops"] * 1e12) if work["flops"] else 0.0
-    if t_tc > t_hbm:
+    t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    peak_fl = FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"]
+    t_fl = work["flops"] / (peak_fl * 1e12) if work["flops"] else 0.0
+    if t_fl > t_mem:
         achieved = work["flops"] / sec / 1e12
-        return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"]}
+        return {"bound": "alu" if alu else "tensor", "achieved": achieved, "peak": peak_fl, "unit": "TFLOP/s",
+                "frac": achieved / peak_fl, "algorithmic": work["flops"],
+                "peak_note": ("fp32 CUDA-core peak derived from 148 SMs x 128 lanes x FMA x 1.965 GHz" if alu
+                              else "bf16 dense, burst (kernel timed alone)")}
     achieved = work["bytes"] / sec / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": achieved / peaks["hbm_gbs"]}
+            "frac": achieved / peaks["hbm_gbs"], "algorithmic": work["bytes"]}
 
 
 def kernel_traffic(workload_key, kernel_key):
@@ -90,6 +136,7 @@ def kernel_traffic(workload_key, kernel_key):
     return ent["dram_bytes_per_launch"]
 
 
+# ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -132,6 +179,7 @@ class ClockSampler:
         try:
             sm = [float(r[1]) for r in rows]
             mx = float(rows[0][2])
+            pw = [float(r[3]) for r in rows]
         except (ValueError, IndexError):
             return None
         reasons = set()
@@ -140,9 +188,14 @@ class ClockSampler:
             for i, nm in enumerate(names):
                 if len(r) > 5 + i and r[5 + i].strip().lower() == "active":
                     reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(rows)}
+        # samples under load: power above the idle level (the first sample is taken before the load)
+        loaded = [s for s, p in zip(sm, pw) if p > pw[0] + 30.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded) if loaded is not sm else 0,
+                "power_w_max": max(pw)}
 
 
+# ----------------------------------------------------------------------------- process group
 def dist_setup(n_gpus):
     import torch
     import torch.distributed as dist
@@ -161,335 +214,6 @@ def dist_setup(n_gpus):
     return rank, local, world
 
 
-WORKLOADS = {
-    # name: (generator, base seed)
-    "small_c": ("small_c_bf16", 1),
-    "large_c_fwd": ("large_c_fwd_bf16", 2),
-    "large_c_bwd": ("large_c_bwd_bf16", 3),
-    "adapter": ("adapter_bf16", 4),
-}
-WORKLOAD = "small_c"
-
-
-def make_inputs(seed_offset=0, workload=None):
-    from sparse_convolution_pruned_b200 import workloads as wl
-    gen, seed = WORKLOADS[workload or WORKLOAD]
-    return getattr(wl, gen)(seed=seed + seed_offset)
-
-
-# ----------------------------------------------------------------------------- reference arm (CPU oracle)
-def cpu_oracle_step(w, frames):
-    """One oracle step on the first `frames` frames (frames are independent)."""
-    import oracle
-    r1 = int(w.frame_off[frames])
-    coords = w.coords[:r1]
-    off = w.frame_off[: frames + 1]
-    t0 = time.perf_counter()
-    nbr, _, st = oracle.build_index(coords, off, frames, w.H, w.W, want_map=False)
-    oracle.fwd(w.X[:r1], nbr, w.Wt, w.bias)
-    oracle.bwd_data(w.dY[:r1], nbr, w.Wt)
-    oracle.bwd_weight(w.dY[:r1], w.X[:r1], nbr)
-    return time.perf_counter() - t0, r1
-
-
-def oracle_frames(w, mac_budget):
-    """How many leading frames of the workload fit a budget of oracle multiply-adds."""
-    per_token = 3 * 9 * w.Cin * w.Cout  # fwd + bwd_data + bwd_weight
-    per_frame = per_token * w.n / max(1, w.T)
-    return int(max(1, min(w.T, mac_budget // max(1, per_frame))))
-
-
-def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
-    import oracle
-    oracle.build()
-    w = make_inputs(0)
-    if WORKLOAD == "adapter":
-        return run_reference_adapter(args, w)
-    # each step: the first frames of the workload, about 4e9 multiply-adds (a few seconds)
-    frames = oracle_frames(w, 4e9)
-    for _ in range(args.warmup):
-        cpu_oracle_step(w, frames)
-    tot, toks = 0.0, 0
-    for _ in range(args.steps):
-        dt, r = cpu_oracle_step(w, frames)
-        tot += dt
-        toks += r
-    value = toks / tot
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "n_kept": w.n, "sample": f"first {frames} of {w.T} frames per step"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
-                         "sample": f"index+fwd+bwd_data+bwd_weight on the first {frames} frames "
-                                   f"({int(w.frame_off[frames])} tokens) per step; 1 core used of "
-                                   f"{os.cpu_count()}"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line))
-    return 0
-
-
-def run_reference_adapter(args, w):
-    """Oracle index build + adapter forward on the first 8 frames of the long video per step."""
-    import oracle
-    frames = 8
-    r1 = int(w.frame_off[frames])
-
-    def one():
-        t0 = time.perf_counter()
-        sub_n, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W,
-                                         want_map=False)
-        oracle.adapter_fwd(w.X[:r1], sub_n, 0, r1, w.Wd, w.Wc, w.Wu)
-        return time.perf_counter() - t0
-
-    for _ in range(args.warmup):
-        one()
-    tot = sum(one() for _ in range(args.steps))
-    value = r1 * args.steps / tot
-    sample = (f"index build + adapter forward on the first {frames} of {w.T} frames ({r1} tokens) per step; "
-              f"single-threaded C, fp64; 1 core used of {os.cpu_count()}")
-    print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "n_kept": w.n, "sample": f"first {frames} of {w.T} frames per step"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
-                         "sample": sample},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }))
-    return 0
-
-
-# ----------------------------------------------------------------------------- B200 arm
-def run_b200(args):
-    import torch
-    import torch.distributed as dist
-
-    from sparse_convolution_pruned_b200 import svconv as sv
-    from sparse_convolution_pruned_b200.data_parallel import allreduce_grads
-
-    rank, local, world = dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    w = make_inputs(rank)  # weak scaling: each rank owns its own batch of frames
-    n, T, Cin, Cout = w.n, w.T, w.Cin, w.Cout
-
-    # pinned host inputs (the e2e leg copies these every step)
-    h_coords = torch.from_numpy(w.coords).pin_memory()
-    h_off = torch.from_numpy(w.frame_off).pin_memory()
-    h_X = torch.from_numpy(w.X).to(torch.bfloat16).pin_memory()
-    h_W = torch.from_numpy(w.Wt).to(torch.bfloat16).pin_memory()
-    h_dY = torch.from_numpy(w.dY).to(torch.bfloat16).pin_memory()
-    bias = torch.from_numpy(w.bias).to(dev) if w.bias is not None else None
-
-    coords = h_coords.to(dev)
-    off = h_off.to(dev)
-    X = h_X.to(dev)
-    Wt = h_W.to(dev)
-    dY = h_dY.to(dev)
-    nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
-    Y = torch.empty((n, Cout), dtype=torch.bfloat16, device=dev)
-    dX = torch.empty((n, Cin), dtype=torch.bfloat16, device=dev)
-    grads = torch.empty((Cout * 9 * Cin + Cout,), dtype=torch.float32, device=dev)
-    dW = grads[: Cout * 9 * Cin].view(Cout, 9, Cin)
-    db = grads[Cout * 9 * Cin:]
-    ws = torch.empty((max(16, sv.svconv_bwd_weight_workspace_size(sv.BF16, n, Cin, Cout),
-                          sv.svconv_bwd_workspace_size(sv.BF16, n, Cin, Cout)),), dtype=torch.uint8, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty((FLUSH_BYTES,), dtype=torch.uint8, device=dev)
-
-    stream = torch.cuda.Stream(device=dev)
-
-    def step_kernels():
-        sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
-        sv.svconv_fwd(X, nbr, Wt, bias, Y=Y)
-        # backward: data and weight gradients in one call (side by side at 64 channels)
-        sv.svconv_bwd(dY, X, nbr, Wt, dX=dX, dW=dW, db=db, workspace=ws)
-
-    launches_per_step = 5  # index, fwd, bwd_data, wgrad partials, wgrad reduce
-
-    with torch.cuda.stream(stream):
-        step_kernels()  # first call outside capture: caches device info and kernel attributes
-        stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-            step_kernels()
-        g_fwd = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_fwd, stream=stream, capture_error_mode="relaxed"):
-            sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
-            sv.svconv_fwd(X, nbr, Wt, bias, Y=Y)
-    torch.cuda.synchronize()
-
-    def one_step():
-        g.replay()
-        if world > 1:
-            allreduce_grads(grads)
-
-    def timed_loop(fn, steps, warmup, flush_l2=True):
-        with torch.cuda.stream(stream):
-            for _ in range(warmup):
-                if flush_l2:
-                    flush.zero_()
-                fn()
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            torch.cuda.synchronize()
-            evs = []
-            for _ in range(steps):
-                if flush_l2:
-                    flush.zero_()
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                evs.append((a, b))
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in evs)
-
-    with ClockSampler(local) as clk:
-        total_ms = timed_loop(one_step, args.steps, args.warmup)
-    clocks = clk.summary()
-    fwd_ms = timed_loop(g_fwd.replay, args.steps, args.warmup)
-    # the same step with the workload left in L2 between steps (reported beside the flushed number)
-    hot_ms = timed_loop(one_step, args.steps, args.warmup, flush_l2=False)
-
-    t = torch.tensor([total_ms, fwd_ms, hot_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_ms, hot_ms = float(t[0]), float(t[1]), float(t[2])
-
-    # per-kernel durations (events between the library calls on the launching stream)
-    names = ["build_index", "fwd", "bwd_data", "bwd_weight"]
-    calls = [lambda: sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status),
-             lambda: sv.svconv_fwd(X, nbr, Wt, bias, Y=Y),
-             lambda: sv.svconv_bwd_data(dY, nbr, Wt, dX=dX),
-             lambda: sv.svconv_bwd_weight(dY, X, nbr, dW=dW, db=db, workspace=ws)]
-    per = {k: 0.0 for k in names}
-    kreps = max(args.steps, 10)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            flush.zero_()
-            for c in calls:
-                c()
-        torch.cuda.synchronize()
-        recs = []
-        for _ in range(kreps):
-            # four flush passes (~160 us of GPU work) let the host enqueue every call
-            # and event below before the first kernel starts: no launch gaps inside
-            for _ in range(4):
-                flush.zero_()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-            ev[0].record(stream)
-            for i, c in enumerate(calls):
-                c()
-                ev[i + 1].record(stream)
-            recs.append(ev)
-        torch.cuda.synchronize()
-    for ev in recs:
-        for i, k in enumerate(names):
-            per[k] += ev[i].elapsed_time(ev[i + 1]) / kreps
-
-    # end-to-end through the public API with host buffers
-    h_Y = torch.empty((n, Cout), dtype=torch.bfloat16).pin_memory()
-    h_dX = torch.empty((n, Cin), dtype=torch.bfloat16).pin_memory()
-    h_grads = torch.empty_like(grads, device="cpu").pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (h_coords, h_off, h_X, h_W, h_dY))
-    d2h = sum(x.numel() * x.element_size() for x in (h_Y, h_dX, h_grads))
-
-    def e2e_step():
-        coords.copy_(h_coords, non_blocking=True)
-        off.copy_(h_off, non_blocking=True)
-        X.copy_(h_X, non_blocking=True)
-        Wt.copy_(h_W, non_blocking=True)
-        dY.copy_(h_dY, non_blocking=True)
-        step_kernels()
-        if world > 1:
-            allreduce_grads(grads)
-        h_Y.copy_(Y, non_blocking=True)
-        h_dX.copy_(dX, non_blocking=True)
-        h_grads.copy_(grads, non_blocking=True)
-
-    e2e_ms = timed_loop(e2e_step, args.steps, args.warmup)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t[0])
-
-    torch.cuda.synchronize()
-    st = int(status.item())
-    err = sv.svconv_read_error_word()
-    if st or err:
-        raise SystemExit(f"device status {st} / library error word {err}: results invalid")
-
-    # CPU baseline: the oracle as it stands, rank 0 at N=1 only, on a bounded sample
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        # about 1.6e10 multiply-adds of oracle work (10-15 s on one core)
-        frames = oracle_frames(w, 1.6e10)
-        macs = 3 * 9 * Cin * Cout * int(w.frame_off[frames])
-        reps = int(max(1, round(1.6e10 / macs)))
-        dt, toks = 0.0, 0
-        for _ in range(reps):
-            d, r = cpu_oracle_step(w, frames)
-            dt += d
-            toks += r
-        cpu = {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
-               "sample": f"index+fwd+bwd_data+bwd_weight on the first {frames} of {w.T} frames "
-                         f"({int(w.frame_off[frames])} tokens), {reps} time(s); single-threaded C, fp64; "
-                         f"1 core used of {os.cpu_count()}"}
-
-    if rank == 0:
-        peaks = load_peaks()
-        work = algorithmic_work(n, T, Cin, Cout)
-        if bias is not None:
-            work["fwd"]["bytes"] += 4 * Cout
-        kern = {k: dict(ms=per[k], **roofline_entry(k, work[k], per[k], peaks)) for k in names}
-        top = max(names, key=lambda k: per[k])
-        roof = dict(kern[top])
-        roof.pop("ms")
-        roof["kernel"] = top
-        roof["traffic"] = kernel_traffic(args.workload, top)
-        roof["peak_source"] = peaks["source"]
-        tokens = n * world
-        line = {
-            "metric": METRIC, "value": tokens * args.steps / (total_ms * 1e-3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": w.name, "n_kept_per_gpu": n, "T": T, "H": w.H, "W": w.W, "C_in": Cin,
-                       "C_out": Cout, "step": "build_index+fwd+bwd(data, weight: one svconv_bwd call)" +
-                                               ("+allreduce(dW,db)" if world > 1 else ""),
-                       "l2": f"flushed by a {FLUSH_BYTES >> 20} MiB write between timed steps",
-                       "graph": "step replayed from a CUDA graph", "parallelism": f"dp{world}"},
-            "fwd": {"value": tokens * args.steps / (fwd_ms * 1e-3), "unit": UNIT,
-                    "ms_per_step": fwd_ms / args.steps, "step": "build_index+fwd"},
-            "l2_hot": {"value": tokens * args.steps / (hot_ms * 1e-3), "unit": UNIT,
-                       "ms_per_step": hot_ms / args.steps, "note": "same step, no L2 flush between steps"},
-            "roofline": roof,
-            "kernels": kern,
-            "e2e": {"value": tokens * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line))
-    if world > 1:
-        del g, g_fwd
-        dist.destroy_process_group()
-    return 0
-
-
 def host_cpu():
     """CPU model and logical core count of this host (for the CPU-baseline record)."""
     model = "unknown"
@@ -503,21 +227,421 @@ def host_cpu():
     return {"model": model, "nproc": os.cpu_count()}
 
 
-# ----------------------------------------------------------------------------- adapter workload (a5)
-def run_adapter(args):
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_conv_step(w, frames, with_bwd):
+    """One oracle step on the first `frames` frames (frames are independent)."""
+    import oracle
+    r1 = int(w.frame_off[frames])
+    t0 = time.perf_counter()
+    nbr, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W, want_map=False)
+    oracle.fwd(w.X[:r1], nbr, w.Wt, w.bias)
+    if with_bwd:
+        oracle.bwd_data(w.dY[:r1], nbr, w.Wt)
+        oracle.bwd_weight(w.dY[:r1], w.X[:r1], nbr)
+    return time.perf_counter() - t0, r1
+
+
+# the single-threaded oracle does about 1.2e9 multiply-adds per second
+ORACLE_MACS_PER_S = 1.2e9
+
+
+def oracle_conv_frames(w, seconds, with_bwd):
+    """Leading frames whose oracle step takes about `seconds` (at least one frame)."""
+    per_token = (3 if with_bwd else 1) * 9 * w.Cin * w.Cout
+    per_frame = per_token * w.n / max(1, w.T)
+    return int(max(1, min(w.T, seconds * ORACLE_MACS_PER_S // max(1, per_frame))))
+
+
+def cpu_baseline_conv(w, with_bwd, seconds):
+    import oracle
+    oracle.build()
+    frames = oracle_conv_frames(w, seconds, with_bwd)
+    r = int(w.frame_off[frames])
+    macs = (3 if with_bwd else 1) * 9 * w.Cin * w.Cout * r
+    reps = int(max(1, round(seconds * ORACLE_MACS_PER_S / max(1, macs))))
+    dt, toks = 0.0, 0
+    for _ in range(reps):
+        d, rr = oracle_conv_step(w, frames, with_bwd)
+        dt += d
+        toks += rr
+    what = "index+fwd+bwd_data+bwd_weight" if with_bwd else "index+fwd"
+    return {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
+            "sample": f"{what} on the first {frames} of {w.T} frames ({r} tokens), {reps} time(s); "
+                      f"frames are independent, so the rate is the workload's; single-threaded C, fp64; "
+                      f"1 core used of {os.cpu_count()}"}
+
+
+def oracle_adapter_step(w, frames):
+    import oracle
+    r1 = int(w.frame_off[frames])
+    t0 = time.perf_counter()
+    sub_n, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W, want_map=False)
+    oracle.adapter_fwd(w.X[:r1], sub_n, 0, r1, w.Wd, w.Wc, w.Wu)
+    return time.perf_counter() - t0, r1
+
+
+def cpu_baseline_adapter(w, seconds):
+    import oracle
+    oracle.build()
+    per_frame = (w.D * w.R * 2 + 9 * w.R * w.R) * w.n / w.T
+    frames = int(max(1, min(w.T, seconds * ORACLE_MACS_PER_S // per_frame)))
+    dt, r1 = oracle_adapter_step(w, frames)
+    t1 = time.perf_counter()
+    oracle.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=True)
+    idx_ms = 1e3 * (time.perf_counter() - t1)
+    return {"value": r1 / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
+            "sample": f"index build + adapter forward on the first {frames} of {w.T} frames ({r1} tokens); "
+                      f"frames are independent; single-threaded C, fp64; 1 core used of {os.cpu_count()}",
+            "index_build_full_ms": idx_ms}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle on the host cores, on the headline workload, each step a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    key = args.workload or HEADLINE
+    w = make_inputs(key)
+    kind = WORKLOADS[key][2]
+    # whole run (warm-up + timed steps) within about two minutes of CPU time
+    per_step_s = max(0.05, min(3.0, 120.0 / (args.steps + args.warmup)))
+    if kind == "adapter":
+        per_frame = (w.D * w.R * 2 + 9 * w.R * w.R) * w.n / w.T
+        frames = int(max(1, min(w.T, per_step_s * ORACLE_MACS_PER_S // per_frame)))
+
+        def one():
+            return oracle_adapter_step(w, frames)
+    else:
+        with_bwd = kind == "fwd+bwd"
+        frames = oracle_conv_frames(w, per_step_s, with_bwd)
+
+        def one():
+            return oracle_conv_step(w, frames, with_bwd)
+    for _ in range(args.warmup):
+        one()
+    tot, toks = 0.0, 0
+    for _ in range(args.steps):
+        dt, r = one()
+        tot += dt
+        toks += r
+    value = toks / tot
+    sample = f"first {frames} of {w.T} frames ({int(w.frame_off[frames])} tokens) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n_kept": w.n, "step": kind, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
+                         "sample": f"{kind} step of the oracle on the {sample}; frames are independent; "
+                                   f"single-threaded C, fp64; 1 core used of {os.cpu_count()}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU timing helpers
+class Ctx:
+    """Per-process GPU state shared by the workload legs."""
+
+    def __init__(self, args, rank, local, world):
+        import torch
+        self.args, self.rank, self.local, self.world = args, rank, local, world
+        self.dev = torch.device("cuda", local)
+        self.stream = torch.cuda.Stream(device=self.dev)
+        self.flush = torch.empty((FLUSH_BYTES,), dtype=torch.uint8, device=self.dev)
+        self.peaks = load_peaks()
+
+    def timed(self, fn, steps, warmup, flush_l2=True):
+        """Sum of per-step CUDA-event times on the launching stream (barrier + synchronize on
+        both sides; the L2 flush, when asked for, runs before each step outside the events)."""
+        import torch
+        import torch.distributed as dist
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                if flush_l2:
+                    self.flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            if self.world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            evs = []
+            for _ in range(steps):
+                if flush_l2:
+                    self.flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(self.stream)
+                fn()
+                b.record(self.stream)
+                evs.append((a, b))
+            torch.cuda.synchronize()
+            if self.world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    def max_over_ranks(self, *vals):
+        import torch
+        import torch.distributed as dist
+        if self.world == 1:
+            return vals
+        t = torch.tensor(vals, dtype=torch.float64, device=self.dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return tuple(float(v) for v in t)
+
+    def per_kernel(self, calls, reps):
+        """Average event time of each call, queued behind ~160 us of flush work so that the host
+        has enqueued every call and event before the first kernel starts (no launch gaps)."""
+        import torch
+        with torch.cuda.stream(self.stream):
+            for _ in range(3):
+                self.flush.zero_()
+                for _, c in calls:
+                    c()
+            torch.cuda.synchronize()
+            recs = []
+            for _ in range(reps):
+                for _ in range(4):
+                    self.flush.zero_()
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+                ev[0].record(self.stream)
+                for i, (_, c) in enumerate(calls):
+                    c()
+                    ev[i + 1].record(self.stream)
+                recs.append(ev)
+            torch.cuda.synchronize()
+        out = {}
+        for i, (name, _) in enumerate(calls):
+            out[name] = sum(ev[i].elapsed_time(ev[i + 1]) for ev in recs) / reps
+        return out
+
+    def sustained(self, graph, est_ms, seconds):
+        """Back-to-back replays of `graph` for about `seconds`, with clock samples."""
+        import torch
+        reps = int(min(50000, max(10, math.ceil(seconds * 1e3 / max(est_ms, 1e-3)))))
+        with torch.cuda.stream(self.stream):
+            torch.cuda.synchronize()
+            with ClockSampler(self.local) as clk:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(self.stream)
+                for _ in range(reps):
+                    graph.replay()
+                b.record(self.stream)
+                torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        return reps, ms, clk.summary()
+
+
+def capture(stream, fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            fn()
+    return g
+
+
+def check_status(sv, status):
+    import torch
+    torch.cuda.synchronize()
+    st = int(status.item())
+    err = sv.svconv_read_error_word()
+    if st or err:
+        raise SystemExit(f"device status {st} / library error word {err}: results invalid")
+
+
+# ----------------------------------------------------------------------------- conv workloads
+def conv_leg(ctx, key, with_cpu, clock_window=False):
+    """One SparseConv2D workload: index build + forward [+ fused backward] per step."""
+    import torch
+
+    from sparse_convolution_pruned_b200 import svconv as sv
+    from sparse_convolution_pruned_b200.data_parallel import allreduce_grads
+
+    args, dev, stream, world = ctx.args, ctx.dev, ctx.stream, ctx.world
+    _, _, kind, dt_name = WORKLOADS[key]
+    with_bwd = kind == "fwd+bwd"
+    w = make_inputs(key, ctx.rank)  # weak scaling: each rank owns its own batch of frames
+    n, T, Cin, Cout = w.n, w.T, w.Cin, w.Cout
+    tdt = torch.float32 if dt_name == "f32" else torch.bfloat16
+    code = sv.F32 if dt_name == "f32" else sv.BF16
+    elem = 4 if dt_name == "f32" else 2
+
+    # pinned host inputs (the end-to-end leg copies these every step)
+    h_coords = torch.from_numpy(w.coords).pin_memory()
+    h_off = torch.from_numpy(w.frame_off).pin_memory()
+    h_X = torch.from_numpy(w.X).to(tdt).pin_memory()
+    h_W = torch.from_numpy(w.Wt).to(tdt).pin_memory()
+    h_dY = torch.from_numpy(w.dY).to(tdt).pin_memory()
+    h_b = torch.from_numpy(w.bias).pin_memory() if w.bias is not None else None
+    coords, off, X, Wt, dY = (t.to(dev) for t in (h_coords, h_off, h_X, h_W, h_dY))
+    bias = h_b.to(dev) if h_b is not None else None
+    nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
+    Y = torch.empty((n, Cout), dtype=tdt, device=dev)
+    dX = torch.empty((n, Cin), dtype=tdt, device=dev)
+    grads = torch.empty((Cout * 9 * Cin + Cout,), dtype=torch.float32, device=dev)
+    dW = grads[: Cout * 9 * Cin].view(Cout, 9, Cin)
+    db = grads[Cout * 9 * Cin:]
+    ws = torch.empty((max(16, sv.svconv_bwd_weight_workspace_size(code, n, Cin, Cout),
+                          sv.svconv_bwd_workspace_size(code, n, Cin, Cout)),), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def index():
+        sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
+
+    def fwd():
+        sv.svconv_fwd(X, nbr, Wt, bias, Y=Y)
+
+    def bwd():
+        # data and weight gradients in one call (side by side on disjoint SMs at 64 channels)
+        sv.svconv_bwd(dY, X, nbr, Wt, dX=dX, dW=dW, db=db, workspace=ws)
+
+    def step_kernels():
+        index()
+        fwd()
+        if with_bwd:
+            bwd()
+
+    wgrad_launches = 2  # tcgen05 / fp32 partials + fixed-order split reduce
+    launches = 2 + ((1 + wgrad_launches) if with_bwd else 0)
+
+    with torch.cuda.stream(stream):
+        step_kernels()  # first call outside capture: caches device info, kernel attributes, side streams
+        stream.synchronize()
+    g = capture(stream, step_kernels)
+    g_fwd = capture(stream, lambda: (index(), fwd())) if with_bwd else None
+    torch.cuda.synchronize()
+
+    def one_step():
+        g.replay()
+        if world > 1 and with_bwd:
+            allreduce_grads(grads)
+
+    clocks = None
+    sus = None
+    if clock_window:
+        # clock samples over the timed steps and the sustained replays right after them
+        with ClockSampler(ctx.local) as clk:
+            total_ms = ctx.timed(one_step, args.steps, args.warmup)
+            if args.sustained_s > 0:
+                sus = ctx.sustained(g, total_ms / args.steps, args.sustained_s)
+        clocks = clk.summary()
+    else:
+        total_ms = ctx.timed(one_step, args.steps, args.warmup)
+        if args.sustained_s > 0:
+            sus = ctx.sustained(g, total_ms / args.steps, args.sustained_s)
+    fwd_ms = ctx.timed(g_fwd.replay, args.steps, args.warmup) if with_bwd else total_ms
+    hot_ms = ctx.timed(one_step, args.steps, args.warmup, flush_l2=False)
+    total_ms, fwd_ms, hot_ms = ctx.max_over_ranks(total_ms, fwd_ms, hot_ms)
+
+    names = [("build_index", index), ("fwd", fwd)]
+    if with_bwd:
+        names += [("bwd_data", lambda: sv.svconv_bwd_data(dY, nbr, Wt, dX=dX)),
+                  ("bwd_weight", lambda: sv.svconv_bwd_weight(dY, X, nbr, dW=dW, db=db, workspace=ws))]
+    per = ctx.per_kernel(names, max(args.steps, 10))
+    if with_bwd:
+        per["bwd (fused call)"] = ctx.per_kernel([("bwd", bwd)], max(args.steps, 10))["bwd"]
+
+    # end to end through the Python API with pinned host buffers
+    h_Y = torch.empty((n, Cout), dtype=tdt).pin_memory()
+    h_dX = torch.empty((n, Cin), dtype=tdt).pin_memory()
+    h_grads = torch.empty_like(grads, device="cpu").pin_memory()
+    ins = [h_coords, h_off, h_X, h_W, h_dY] + ([h_b] if h_b is not None else [])
+    outs = [h_Y] + ([h_dX, h_grads] if with_bwd else [])
+    h2d = sum(x.numel() * x.element_size() for x in ins)
+    d2h = sum(x.numel() * x.element_size() for x in outs)
+
+    def e2e_step():
+        coords.copy_(h_coords, non_blocking=True)
+        off.copy_(h_off, non_blocking=True)
+        X.copy_(h_X, non_blocking=True)
+        Wt.copy_(h_W, non_blocking=True)
+        if bias is not None:
+            bias.copy_(h_b, non_blocking=True)
+        if with_bwd:
+            dY.copy_(h_dY, non_blocking=True)
+        step_kernels()
+        if world > 1 and with_bwd:
+            allreduce_grads(grads)
+        h_Y.copy_(Y, non_blocking=True)
+        if with_bwd:
+            h_dX.copy_(dX, non_blocking=True)
+            h_grads.copy_(grads, non_blocking=True)
+
+    if not with_bwd:
+        h2d -= h_dY.numel() * h_dY.element_size()
+    (e2e_ms,) = ctx.max_over_ranks(ctx.timed(e2e_step, args.steps, args.warmup))
+    check_status(sv, status)
+
+    cpu = cpu_baseline_conv(w, with_bwd, args.cpu_seconds) if with_cpu else None
+
+    peaks = ctx.peaks
+    alu = dt_name == "f32"
+    work = conv_work(n, T, Cin, Cout, elem, bias is not None)
+    kern = {}
+    for k in [nm for nm, _ in names]:
+        kern[k] = dict(ms=per[k], **roofline_entry(work[k], per[k], peaks, alu=alu and k != "build_index"))
+    if with_bwd:
+        kern["bwd (fused call)"] = {"ms": per["bwd (fused call)"],
+                                   "note": "svconv_bwd: both gradients in one call, as the step runs them"}
+    top = max((nm for nm, _ in names), key=lambda k: per[k])
+    roof = {k: v for k, v in kern[top].items() if k != "ms"}
+    roof["kernel"] = top
+    roof["traffic"] = kernel_traffic(key, top)
+    roof["peak_source"] = peaks["source"]
+    floors = sum(floor_seconds(work[k], peaks, alu=alu and k != "build_index") for k, _ in names)
+    step_ms = total_ms / args.steps
+    tokens = n * world
+    res = {
+        "workload": w.name, "n_kept_per_gpu": n, "T": T, "H": w.H, "W": w.W, "C_in": Cin, "C_out": Cout,
+        "dtype": dt_name, "value": tokens / (step_ms * 1e-3), "unit": UNIT, "ms_per_step": step_ms,
+        "step": "build_index+fwd" + ("+bwd(data, weight: one svconv_bwd call)" if with_bwd else "") +
+                ("+allreduce(dW,db)" if world > 1 and with_bwd else ""),
+        "l2": f"flushed by a {FLUSH_BYTES >> 20} MiB write between timed steps",
+        "roofline": roof,
+        "step_roofline": {"floor_ms": floors * 1e3, "frac": floors * 1e3 / step_ms,
+                          "note": "sum of the step's per-kernel floors / measured step time"},
+        "kernels": kern,
+        "l2_hot": {"value": tokens * args.steps / (hot_ms * 1e-3), "ms_per_step": hot_ms / args.steps,
+                   "note": "same step, no L2 flush between steps"},
+        "e2e": {"value": tokens * args.steps / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches_per_step": launches,
+        "cpu_baseline": cpu,
+    }
+    if with_bwd:
+        res["fwd"] = {"value": tokens * args.steps / (fwd_ms * 1e-3), "unit": UNIT,
+                      "ms_per_step": fwd_ms / args.steps, "step": "build_index+fwd"}
+    if sus is not None:
+        reps, ms, sclk = sus
+        res["sustained"] = {"steps": reps, "seconds": ms * 1e-3, "ms_per_step": ms / reps,
+                            "value": n * reps / (ms * 1e-3), "clocks": sclk,
+                            "note": "back-to-back graph replays, no L2 flush"}
+    if clocks is not None:
+        res["clocks"] = clocks
+    del g, g_fwd
+    return res
+
+
+# ----------------------------------------------------------------------------- adapter workload
+def adapter_leg(ctx, with_cpu, clock_window=False):
     """Long-video bottleneck adapter: one step = index build + chunked adapter forward.
 
-    X (n x 1024 bf16, 579 MB at the full size) is read and written in place each step,
-    far larger than L2, so no flush is needed between steps.
+    X (n x 1024 bf16, 579 MB) is read and written in place each step, far larger than L2,
+    so no flush is needed between steps.
     """
     import torch
-    import torch.distributed as dist
 
     from sparse_convolution_pruned_b200 import svconv as sv
 
-    rank, local, world = dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    w = make_inputs(rank)
+    args, dev, stream, world = ctx.args, ctx.dev, ctx.stream, ctx.world
+    w = make_inputs("adapter", ctx.rank)
     n, T, D, R = w.n, w.T, w.D, w.R
     chunk_T = args.adapter_chunk_frames  # frames per chunk (device memory grows with it; cap 1 GB)
     offs = w.frame_off.astype(np.int64)
@@ -526,6 +650,8 @@ def run_adapter(args):
     h_coords = torch.from_numpy(w.coords).pin_memory()
     h_off = torch.from_numpy(w.frame_off).pin_memory()
     h_X = torch.from_numpy(w.X).to(torch.bfloat16).pin_memory()
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated(dev) - ctx.flush.numel()
     torch.cuda.reset_peak_memory_stats(dev)
     coords = h_coords.to(dev)
     off = h_off.to(dev)
@@ -536,7 +662,6 @@ def run_adapter(args):
     nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     ws = torch.empty((max(16, sv.svconv_adapter_workspace_size(R, max_rows)),), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.Stream(device=dev)
 
     def index():
         sv.svconv_build_index(coords, off, T, w.H, w.W, nbr=nbr, status=status)
@@ -545,52 +670,35 @@ def run_adapter(args):
         sv.svconv_adapter_fwd(X, nbr, off, T, Wd, Wc, Wu, chunk_T=chunk_T, max_chunk_rows=max_rows,
                               workspace=ws, status=status)
 
-    n_chunks = (T + chunk_T - 1) // chunk_T
-    launches_per_step = 1 + 3 * n_chunks  # index; per chunk: down GEMM, conv, up GEMM
-
-    def timed(fn, steps, warmup):
-        with torch.cuda.stream(stream):
-            for _ in range(warmup):
-                fn()
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            torch.cuda.synchronize()
-            evs = []
-            for _ in range(steps):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                fn()
-                b.record(stream)
-                evs.append((a, b))
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in evs)
-
     def step():
         index()
         adapter()
 
+    n_chunks = (T + chunk_T - 1) // chunk_T
+    launches = 1 + 3 * n_chunks  # index; per chunk: down GEMM, conv, up GEMM
     with torch.cuda.stream(stream):
         step()
         stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-            step()
-        g_ad = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_ad, stream=stream, capture_error_mode="relaxed"):
-            adapter()
+    g = capture(stream, step)
+    g_ad = capture(stream, adapter)
     torch.cuda.synchronize()
-    peak = torch.cuda.max_memory_allocated(dev)
+    # device memory of the workload (the L2-flush buffer and earlier legs' leftovers excluded)
+    peak = torch.cuda.max_memory_allocated(dev) - ctx.flush.numel() - max(0, base)
 
-    with ClockSampler(local) as clk:
-        total_ms = timed(g.replay, args.steps, args.warmup)
-    clocks = clk.summary()
-    ad_ms = timed(g_ad.replay, args.steps, args.warmup) / args.steps
-    idx_ms = timed(index, args.steps, args.warmup) / args.steps
+    clocks = None
+    sus = None
+    if clock_window:
+        with ClockSampler(ctx.local) as clk:
+            total_ms = ctx.timed(g.replay, args.steps, args.warmup, flush_l2=False)
+            if args.sustained_s > 0:
+                sus = ctx.sustained(g, total_ms / args.steps, args.sustained_s)
+        clocks = clk.summary()
+    else:
+        total_ms = ctx.timed(g.replay, args.steps, args.warmup, flush_l2=False)
+        if args.sustained_s > 0:
+            sus = ctx.sustained(g, total_ms / args.steps, args.sustained_s)
+    ad_ms = ctx.timed(g_ad.replay, args.steps, args.warmup, flush_l2=False) / args.steps
+    idx_ms = ctx.timed(index, args.steps, args.warmup) / args.steps
 
     # end to end: the video's coordinates and features in from pinned host memory, the
     # updated features back out
@@ -606,69 +714,102 @@ def run_adapter(args):
         h_out.copy_(X, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_ms = timed(e2e, e2e_steps, 3)
-    t = torch.tensor([total_ms, e2e_ms, ad_ms, idx_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, ad_ms, idx_ms = (float(v) for v in t)
-    torch.cuda.synchronize()
-    st = int(status.item())
-    err = sv.svconv_read_error_word()
-    if st or err:
-        raise SystemExit(f"device status {st} / library error word {err}: results invalid")
+    e2e_ms = ctx.timed(e2e, e2e_steps, 3, flush_l2=False)
+    total_ms, e2e_ms, ad_ms, idx_ms = ctx.max_over_ranks(total_ms, e2e_ms, ad_ms, idx_ms)
+    check_status(sv, status)
 
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        # whole frames are independent: the oracle runs the first `frames` frames
-        frames = 8
-        r1 = int(w.frame_off[frames])
-        t0 = time.perf_counter()
-        sub_n, _, _ = oracle.build_index(w.coords[:r1], w.frame_off[: frames + 1], frames, w.H, w.W,
-                                         want_map=False)
-        oracle.adapter_fwd(w.X[:r1], sub_n, 0, r1, w.Wd, w.Wc, w.Wu)
-        dt = time.perf_counter() - t0
-        t1 = time.perf_counter()
-        oracle.build_index(w.coords, w.frame_off, T, w.H, w.W, want_map=True)
-        idx_cpu_ms = 1e3 * (time.perf_counter() - t1)
-        cpu = {"value": r1 / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "host": host_cpu(),
-               "sample": f"index build + adapter forward on the first {frames} of {T} frames ({r1} tokens); "
-                         f"single-threaded C, fp64; 1 core used of {os.cpu_count()}",
-               "index_build_full_ms": idx_cpu_ms}
+    cpu = cpu_baseline_adapter(w, args.cpu_seconds) if with_cpu else None
+    peaks = ctx.peaks
+    ad_work = adapter_work(n, D, R)
+    roof = {k: v for k, v in roofline_entry(ad_work, ad_ms, peaks).items()}
+    roof["kernel"] = f"adapter_fwd ({3 * n_chunks} tcgen05 GEMM launches, timed together)"
+    roof["traffic"] = kernel_traffic("adapter", "adapter_fwd")
+    roof["peak_source"] = peaks["source"]
+    # the adapter forward is a ~0.7 ms sequence of tensor-core launches: also against the sustained peak
+    roof["frac_of_sustained_peak"] = ad_work["flops"] / (ad_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]
+    idx_work = conv_work(n, T, R, R, 2, False)["build_index"]
+    step_ms = total_ms / args.steps
+    floors = floor_seconds(ad_work, peaks) + floor_seconds(idx_work, peaks)
+    tokens = n * world
+    res = {
+        "workload": w.name, "n_kept_per_gpu": n, "T": T, "H": w.H, "W": w.W, "D": D, "R": R, "dtype": "bf16",
+        "chunk_T": chunk_T, "value": tokens / (step_ms * 1e-3), "unit": UNIT, "ms_per_step": step_ms,
+        "step": "build_index+adapter_fwd (in place)",
+        "l2": "inputs larger than L2 (X read and written in place each step); no flush",
+        "peak_device_bytes": peak,
+        "roofline": roof,
+        "step_roofline": {"floor_ms": floors * 1e3, "frac": floors * 1e3 / step_ms,
+                          "note": "sum of the step's per-kernel floors / measured step time"},
+        "kernels": {"adapter_fwd": dict(ms=ad_ms, **roofline_entry(ad_work, ad_ms, peaks)),
+                    "build_index": dict(ms=idx_ms, **roofline_entry(idx_work, idx_ms, peaks))},
+        "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches_per_step": launches,
+        "cpu_baseline": cpu,
+    }
+    if sus is not None:
+        reps, ms, sclk = sus
+        res["sustained"] = {"steps": reps, "seconds": ms * 1e-3, "ms_per_step": ms / reps,
+                            "value": n * reps / (ms * 1e-3), "clocks": sclk,
+                            "note": "back-to-back graph replays (X larger than L2)"}
+    if clocks is not None:
+        res["clocks"] = clocks
+    del g, g_ad
+    return res
+
+
+def run_leg(ctx, key, with_cpu, clock_window=False):
+    if WORKLOADS[key][2] == "adapter":
+        return adapter_leg(ctx, with_cpu, clock_window)
+    return conv_leg(ctx, key, with_cpu, clock_window)
+
+
+# ----------------------------------------------------------------------------- B200 arm
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, local, world = dist_setup(args.gpus)
+    ctx = Ctx(args, rank, local, world)
+    head_key = args.workload or HEADLINE
+    with_cpu = world == 1 and not args.no_cpu_baseline
+
+    # the headline workload first: its timed steps and sustained replays carry the clock record
+    head = run_leg(ctx, head_key, with_cpu, clock_window=True)
+    configs = {head_key: head}
+    if world == 1 and not args.workload:
+        for key in ORDER:
+            if key != head_key:
+                configs[key] = run_leg(ctx, key, with_cpu)
 
     if rank == 0:
-        peaks = load_peaks()
-        flops = 2 * n * (D * R + 9 * R * R + R * D)
-        ad_work = {"bytes": 2 * n * D * 2 + 36 * n + 2 * (2 * D * R + 9 * R * R), "flops": flops}
-        roof = roofline_entry("adapter_fwd", ad_work, ad_ms, peaks)
-        roof["kernel"] = f"adapter_fwd ({3 * n_chunks} tcgen05 GEMM launches, timed together)"
-        roof["traffic"] = kernel_traffic(args.workload, "adapter_fwd")  # DRAM bytes of the 18 launches
-        roof["peak_source"] = peaks["source"]
-        idx_work = algorithmic_work(n, T, R, R)["build_index"]
-        tokens = n * world
         line = {
-            "metric": METRIC, "value": tokens * args.steps / (total_ms * 1e-3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
             "data": "synthetic",
-            "config": {"workload": w.name, "n_kept_per_gpu": n, "T": T, "H": w.H, "W": w.W, "D": D, "R": R,
-                       "chunk_T": chunk_T, "step": "build_index+adapter_fwd (in place)",
-                       "l2": "inputs larger than L2 (X read and written in place each step); no flush",
-                       "graph": "step replayed from a CUDA graph", "parallelism": f"dp{world}",
-                       "peak_device_bytes": peak},
-            "roofline": roof,
-            "kernels": {"adapter_fwd": dict(ms=ad_ms, **roofline_entry("adapter_fwd", ad_work, ad_ms, peaks)),
-                        "build_index": dict(ms=idx_ms, **roofline_entry("build_index", idx_work, idx_ms, peaks))},
-            "e2e": {"value": tokens * e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
+            "config": {"workload": head["workload"], "n_kept_per_gpu": head["n_kept_per_gpu"],
+                       "step": head["step"], "l2": head["l2"], "graph": "step replayed from a CUDA graph",
+                       "parallelism": f"dp{world}",
+                       "why_headline": "largest fwd+bwd configuration that fits one GPU"},
+            "roofline": head["roofline"],
+            "step_roofline": head["step_roofline"],
+            "kernels": head["kernels"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches_per_step"] * args.steps,
+            "clocks": dict(head.get("clocks") or {},
+                           window="the headline's timed steps and its sustained replays right after them"),
+            "cpu_baseline": head["cpu_baseline"],
         }
+        if "sustained" in head:
+            line["sustained"] = head["sustained"]
+        if "fwd" in head:
+            line["fwd"] = head["fwd"]
+        if len(configs) > 1:
+            line["configs"] = {k: {kk: vv for kk, vv in v.items()} for k, v in configs.items() if k != head_key}
         print(json.dumps(line))
     if world > 1:
-        del g, g_ad
+        torch.cuda.synchronize()
         dist.destroy_process_group()
     return 0
 
@@ -676,24 +817,27 @@ def run_adapter(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=6.0,
+                    help="CPU-oracle work per workload for the cpu_baseline objects (seconds, about)")
+    ap.add_argument("--sustained-s", type=float, default=1.0,
+                    help="seconds of back-to-back replays per workload for the sustained leg (0: none)")
     ap.add_argument("--adapter-chunk-frames", type=int, default=1024,
                     help="adapter workload: token frames per chunk of the chunked adapter forward "
-                         "(1024: 3 chunks, ~660 MiB peak; 512: 6 chunks, ~610 MiB, 17%% slower)")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="small_c",
-                    help="small_c (default: the headline configuration), large_c_fwd, large_c_bwd, adapter")
+                         "(1024: 3 chunks, ~660 MiB peak; 512: 6 chunks, ~610 MiB)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="time only this workload (as the top-level line); default: the headline "
+                         f"({HEADLINE}) plus every other workload under 'configs'")
     args = ap.parse_args()
-    global WORKLOAD
-    WORKLOAD = args.workload
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.steps < 1:
+        raise SystemExit("--steps must be >= 1")
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload == "adapter":
-        return run_adapter(args)
     return run_b200(args)
 
 

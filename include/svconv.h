@@ -138,9 +138,12 @@ SVCONV_API size_t svconv_bwd_weight_workspace_size(int dtype, int n, int Cin, in
  * allocation would synchronise the device).  It computes exactly what
  * svconv_bwd_weight computes, same arguments minus the workspace: the split
  * partials live in a fixed device array of SVCONV_NOALLOC_SCRATCH_BYTES inside the
- * library, which every GPU that loads the library holds until the process exits.
- *   - The first call on a device looks up that array's address; make it before
- *     any stream capture.
+ * library.  CUDA loads the library's device code on a device lazily, so the array
+ * is taken on a device when that happens, at the latest by the first call of this
+ * entry point there (an empty call, n = 0, counts), and is then held until the
+ * process exits.
+ *   - Make the first call on each device at start-up, before any stream capture:
+ *     it looks up the array's address and so commits the 16 MiB.
  *   - All calls share the array: calls that overlap on the GPU race.  Serialise them.
  *   - If the usual number of token splits does not fit, fewer are used (a different
  *     summation order, same tolerance); if one split's partials
@@ -163,13 +166,17 @@ SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
  *   bf16 with C_in = C_out = 64: the two gradients run side by side on disjoint
  *   groups of SMs, the weight gradient on a side stream of the library that is
  *   forked from and joined back to `stream` with events, so the call stays ordered
- *   on `stream` and can be captured in a CUDA graph.  The first such call on a
- *   device creates that stream and its two events: make it outside stream capture.
- *   Calls from several host threads are serialised inside the library.  dX is
- *   bitwise identical to svconv_bwd_data's; dW / db use fewer token splits than
- *   svconv_bwd_weight (another fixed summation order: deterministic, same
+ *   on `stream` and can be captured in a CUDA graph.  Each (device, caller stream)
+ *   pair gets its own side stream and events, created by the first such call on
+ *   that stream OUTSIDE stream capture; a call made while `stream` is being
+ *   captured before it has a side stream (or once 64 caller streams of a device
+ *   have one) runs the same two launches one after the other on `stream` instead,
+ *   with bitwise the same results.  Calls from several host threads on different
+ *   streams, one of them capturing, neither wait on nor enter each other's work.
+ *   dX is bitwise identical to svconv_bwd_data's; dW / db use fewer token splits
+ *   than svconv_bwd_weight (another fixed summation order: deterministic, same
  *   tolerance).  Other shapes and fp32 run the two calls in order on `stream`.
- *   Errors: as the two calls; SVCONV_ERR_CUDA if the side stream cannot be created.
+ *   Errors: as the two calls.
  */
 SVCONV_API int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
                           const void* Wt, void* dX, float* dW, float* db, void* workspace, size_t ws_bytes,

@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <vector>
 
 #include "svconv.h"
 #include "svconv_internal.h"
@@ -20,14 +21,20 @@
 namespace svc {
 namespace {
 
-constexpr int kMaxDev = 64;
+constexpr int kMaxSideStreams = 64;  // per device; further caller streams run the two kernels in order
 
+// One side stream (and its fork / join events) per (device, caller stream).  A side stream is
+// forked from and joined back to exactly one caller stream, so a stream capture on one caller
+// stream never pulls in, or waits on, work that another caller stream queued, and unrelated
+// caller streams are never ordered against each other through the library.
 struct SideStream {
+  int device = -1;
+  cudaStream_t caller = nullptr;
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
-SideStream g_side[kMaxDev];
-std::mutex g_side_mu;  // guards creation and each call's fork / launch / join sequence
+std::vector<SideStream> g_side;
+std::mutex g_side_mu;  // guards the table and each call's fork / launch / join sequence
 
 bool concurrent_shape(int dtype, int Cin, int Cout) { return dtype == SVCONV_BF16 && Cin == 64 && Cout == 64; }
 
@@ -42,21 +49,33 @@ void budgets(int* data_ctas, int* weight_ctas) {
   *weight_ctas = w;
 }
 
-// Side stream and events of the current device, created on first use (call with g_side_mu held).
-SideStream* side_stream() {
+// Side stream of (current device, caller), created on first use (call with g_side_mu held).
+// Returns nullptr when none can be used: the caller stream is being captured and has no side
+// stream yet (creating one inside a capture is not done), the table is full, or creation failed.
+SideStream* side_stream(cudaStream_t caller) {
   int d = 0;
-  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDev) return nullptr;
-  SideStream& r = g_side[d];
-  if (!r.stream) {
-    if (cudaStreamCreateWithFlags(&r.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) != cudaSuccess) {
-      cudaStreamDestroy(r.stream);
-      r.stream = nullptr;
-      return nullptr;
-    }
+  if (cudaGetDevice(&d) != cudaSuccess) return nullptr;
+  int per_dev = 0;
+  for (SideStream& r : g_side) {
+    if (r.device != d) continue;
+    if (r.caller == caller) return &r;
+    ++per_dev;
   }
-  return &r;
+  if (per_dev >= kMaxSideStreams) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return nullptr;
+  SideStream r;
+  r.device = d;
+  r.caller = caller;
+  if (cudaStreamCreateWithFlags(&r.stream, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+  if (cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming) != cudaSuccess) {
+    if (r.fork) cudaEventDestroy(r.fork);
+    cudaStreamDestroy(r.stream);
+    return nullptr;
+  }
+  g_side.push_back(r);
+  return &g_side.back();
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -97,8 +116,14 @@ int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int
   budgets(&dc, &wc);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_side_mu);
-  SideStream* side = side_stream();
-  if (!side) return SVCONV_ERR_CUDA;
+  SideStream* side = side_stream(s);
+  if (!side) {
+    // no side stream for this caller stream: the same two launches (same CTA budgets, so
+    // bitwise the same results) one after the other on the caller's stream
+    const int rc = tc_bwd_data(dY, nbr, n, Cin, Cout, Wt, dX, dc, s);
+    if (rc) return rc;
+    return tc_bwd_weight(dY, X, nbr, n, Cin, Cout, dW, db, static_cast<float*>(workspace), wc, s);
+  }
   // fork: the side stream waits for everything before this call on the caller's stream
   if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
     return SVCONV_ERR_CUDA;

@@ -7,11 +7,13 @@
 // would synchronise the device).  This variant keeps the partials in a fixed
 // file-scope device array instead, so the caller passes only inputs and outputs.
 //
-// The array is SVCONV_NOALLOC_SCRATCH_BYTES (16 MiB) per device and stays
-// resident on every GPU that loads the library until the process exits.  Its
-// device address is looked up once per device (cudaGetSymbolAddress, with that
-// device current) on the first call, so that first call should be made before
-// any stream capture.  All calls share the array: calls whose kernels overlap on
+// The array is SVCONV_NOALLOC_SCRATCH_BYTES (16 MiB) per device.  CUDA loads a
+// library's device code on a device lazily, so the array is committed on a device
+// when the library's module is first loaded there: at the latest by the first call
+// of this entry point on that device, which looks up the array's device address
+// (cudaGetSymbolAddress, with that device current) before anything else, even for
+// an empty input.  From then on it stays until the process exits.  Make that first
+// call at start-up, before any stream capture.  All calls share the array: calls whose kernels overlap on
 // the GPU (two streams, or two host threads) race and produce wrong gradients;
 // serialise them.  No initial contents are needed: every call rewrites every
 // partial it later reads.  If the default number of token splits does not fit,
@@ -70,6 +72,10 @@ extern "C" int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
   if (dtype == SVCONV_BF16 && (Cin % 64 != 0 || Cout % 64 != 0 || Cin > 4096 || Cout > 4096))
     return SVCONV_ERR_UNSUPPORTED;
   if (!sm100_device()) return SVCONV_ERR_DEVICE;
+  // Looked up first, so that any first call on a device (an empty one included) loads the
+  // library's module there and with it commits the scratch array.
+  float* partial = scratch_address();
+  if (!partial) return SVCONV_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (n == 0) {  // empty sum: zero gradients
     cudaError_t e = cudaMemsetAsync(dW, 0, sizeof(float) * 9 * (size_t)Cin * Cout, s);
@@ -90,9 +96,6 @@ extern "C" int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
   const size_t fit = kScratchFloats / per_split;
   if (fit < 1) return SVCONV_ERR_SIZE;  // one split's partial rows exceed the fixed scratch
   if ((size_t)splits > fit) splits = (int)fit;
-
-  float* partial = scratch_address();
-  if (!partial) return SVCONV_ERR_CUDA;
 
   cudaError_t e;
   if (dtype == SVCONV_F32) {

@@ -256,3 +256,33 @@ def test_adapter_vs_torch_composition(orc):
     H2 = bf(F.gelu(conv, approximate="none"))
     out = bf(X + H2 @ torch.from_numpy(a.Wu.astype(np.float64)).T)[r0:r1].numpy()
     np.testing.assert_allclose(got, out, rtol=0, atol=1e-9)
+
+
+# ------------------------------------------------------------------ frame-parallel oracle runs
+def test_frame_parallel_oracle_equals_the_direct_calls(orc):
+    """The full-size GPU checks run the oracle on frame ranges in worker processes; rows of
+    Y, dX and the adapter are then bit-identical to one direct call (frames are independent),
+    and the summed weight / bias gradients equal the direct sums up to fp64 rounding."""
+    import oracle_pool
+    from sparse_convolution_pruned_b200 import workloads as wl
+    w = wl.custom_conv(seed=61, T=9, H=6, W=7, keep_frac=0.5, Cin=8, Cout=12, dtype="f32", shuffle=True,
+                       empty_frames=(0, 4, 8))
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    got = oracle_pool.conv_full(w, ref_n)
+    assert np.array_equal(got["Y"], orc.fwd(w.X, ref_n, w.Wt, w.bias))
+    assert np.array_equal(got["dX"], orc.bwd_data(w.dY, ref_n, w.Wt))
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    np.testing.assert_allclose(got["dW"], rdW, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["db"], rdb, rtol=1e-12, atol=1e-12)
+    a = wl.adapter_bf16(seed=12, T=10, D=64, R=64)
+    an, _, _ = orc.build_index(a.coords, a.frame_off, a.T, a.H, a.W, want_map=False)
+    assert np.array_equal(oracle_pool.adapter_full(a, an), orc.adapter_fwd(a.X, an, 0, a.n, a.Wd, a.Wc, a.Wu))
+
+
+def test_frame_ranges_cover_every_frame_once():
+    import oracle_pool
+    off = np.array([0, 0, 5, 5, 9, 30, 31, 31, 40], np.int64)
+    for parts in (1, 2, 3, 5, 8, 50):
+        r = oracle_pool.frame_ranges(off, parts)
+        assert r[0][0] == 0 and r[-1][1] == len(off) - 1
+        assert all(a < b for a, b in r) and all(r[i][1] == r[i + 1][0] for i in range(len(r) - 1))
