@@ -758,6 +758,103 @@ def adapter_leg(ctx, with_cpu, clock_window=False):
     return res
 
 
+# ----------------------------------------------------------------------------- keep-rate crossover
+CROSSOVER_KEEPS = [0.1, 0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0]
+CROSSOVER_CHANNELS = [64, 256]
+
+
+def crossing(keeps, t_sparse, t_dense):
+    """Keep rate at which the sparse time meets the dense time (linear between sweep points);
+    None when the sparse path is faster at every swept keep rate."""
+    d = [a - b for a, b in zip(t_sparse, t_dense)]
+    for i in range(len(d)):
+        if d[i] >= 0:
+            if i == 0:
+                return keeps[0]
+            return keeps[i - 1] + (keeps[i] - keeps[i - 1]) * (-d[i - 1]) / (d[i] - d[i - 1])
+    return None
+
+
+def crossover_leg(ctx):
+    """SparseConv2D against the dense-reconstruction pipeline (scatter -> cuDNN conv2d ->
+    gather, PyTorch ops) over keep rates 0.1 .. 1.0 at C = 64 and C = 256 (T = 384 frames,
+    16 x 16 grid, blob-saliency top-k keep, bf16), forward and forward + backward."""
+    import torch
+
+    from sparse_convolution_pruned_b200 import svconv as sv
+    from sparse_convolution_pruned_b200 import workloads as wl
+    from sparse_convolution_pruned_b200.dense_recon import DenseRecon, torch_weight
+
+    torch.backends.cudnn.benchmark = True
+    args, dev, stream = ctx.args, ctx.dev, ctx.stream
+    steps = max(5, min(args.steps, 10))
+    out = {"setup": "T=384, 16x16 grid, blob-saliency top-k keep per frame, bf16, no bias; sparse = svconv_fwd "
+                    "(+ svconv_bwd) with the neighbour table built once per layout (the page reuses it across "
+                    "the layers of a pruning stage; 'with index' adds svconv_build_index); dense = scatter -> "
+                    "torch conv2d (cuDNN, channels-last, benchmark mode) -> gather, backward by autograd; "
+                    "every step replayed from a CUDA graph, L2 flushed between steps",
+           "keeps": CROSSOVER_KEEPS, "curves": {}}
+    for C in CROSSOVER_CHANNELS:
+        cur = {"sparse_fwd_ms": [], "sparse_fwd_with_index_ms": [], "dense_fwd_ms": [],
+               "sparse_fwd_bwd_ms": [], "dense_fwd_bwd_ms": [], "n_kept": []}
+        for keep in CROSSOVER_KEEPS:
+            k = int(round(keep * 256))
+            w = wl.small_c_bf16(seed=5, T=384, C=C, k=k)
+            coords = torch.from_numpy(w.coords).to(dev)
+            off = torch.from_numpy(w.frame_off).to(dev)
+            X = torch.from_numpy(w.X).to(torch.bfloat16).to(dev)
+            Wt = torch.from_numpy(w.Wt).to(torch.bfloat16).to(dev)
+            dY = torch.from_numpy(w.dY).to(torch.bfloat16).to(dev)
+            nbr = torch.empty((w.n, 9), dtype=torch.int32, device=dev)
+            Y = torch.empty((w.n, C), dtype=torch.bfloat16, device=dev)
+            dX = torch.empty_like(Y)
+            dW = torch.empty((C, 9, C), dtype=torch.float32, device=dev)
+            db = torch.empty((C,), dtype=torch.float32, device=dev)
+            ws = torch.empty((max(16, sv.svconv_bwd_workspace_size(sv.BF16, w.n, C, C)),), dtype=torch.uint8,
+                             device=dev)
+            wtorch = torch_weight(Wt)
+            dense = DenseRecon(coords, w.T, w.H, w.W)
+
+            def index():
+                sv.svconv_build_index(coords, off, w.T, w.H, w.W, nbr=nbr)
+
+            def s_fwd():
+                sv.svconv_fwd(X, nbr, Wt, None, Y=Y)
+
+            def s_fwd_bwd():
+                s_fwd()
+                sv.svconv_bwd(dY, X, nbr, Wt, dX=dX, dW=dW, db=db, workspace=ws)
+
+            with torch.cuda.stream(stream):
+                index()
+                s_fwd_bwd()
+                for _ in range(3):  # cuDNN algorithm selection and autograd warm-up outside capture
+                    dense.fwd(X, wtorch)
+                    dense.fwd_bwd(X, wtorch, dY)
+                stream.synchronize()
+            graphs = {
+                "sparse_fwd_ms": capture(stream, s_fwd),
+                "sparse_fwd_with_index_ms": capture(stream, lambda: (index(), s_fwd())),
+                "dense_fwd_ms": capture(stream, lambda: dense.fwd(X, wtorch)),
+                "sparse_fwd_bwd_ms": capture(stream, s_fwd_bwd),
+                "dense_fwd_bwd_ms": capture(stream, lambda: dense.fwd_bwd(X, wtorch, dY)),
+            }
+            for name, g in graphs.items():
+                (ms,) = ctx.max_over_ranks(ctx.timed(g.replay, steps, 3))
+                cur[name].append(ms / steps)
+            cur["n_kept"].append(w.n)
+            del graphs
+        cur["crossover_keep_fwd"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_ms"], cur["dense_fwd_ms"])
+        cur["crossover_keep_fwd_with_index"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_with_index_ms"],
+                                                        cur["dense_fwd_ms"])
+        cur["crossover_keep_fwd_bwd"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_bwd_ms"], cur["dense_fwd_bwd_ms"])
+        out["curves"][f"C{C}"] = cur
+    out["note"] = ("crossover_keep_* = keep rate where the sparse time meets the dense time (linear between "
+                   "sweep points); null = sparse faster at every swept keep rate.  The page reports 55% on its "
+                   "own (unstated) hardware")
+    return out
+
+
 def run_leg(ctx, key, with_cpu, clock_window=False):
     if WORKLOADS[key][2] == "adapter":
         return adapter_leg(ctx, with_cpu, clock_window)
@@ -781,6 +878,8 @@ def run_b200(args):
         for key in ORDER:
             if key != head_key:
                 configs[key] = run_leg(ctx, key, with_cpu)
+        if not args.no_crossover:
+            configs["crossover"] = crossover_leg(ctx)
 
     if rank == 0:
         line = {
@@ -828,6 +927,8 @@ def main():
     ap.add_argument("--adapter-chunk-frames", type=int, default=1024,
                     help="adapter workload: token frames per chunk of the chunked adapter forward "
                          "(1024: 3 chunks, ~660 MiB peak; 512: 6 chunks, ~610 MiB)")
+    ap.add_argument("--no-crossover", action="store_true",
+                    help="skip the keep-rate sweep against the dense-reconstruction baseline")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
                     help="time only this workload (as the top-level line); default: the headline "
                          f"({HEADLINE}) plus every other workload under 'configs'")

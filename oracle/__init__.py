@@ -59,6 +59,7 @@ def _load():
         lib.orc_adapter_fwd.argtypes = [P, P, I, I, I, I, P, P, P, P, P]
         lib.orc_dense_conv.argtypes = [P, I, I, I, I, P, P, P]
         lib.orc_bwd_bias.argtypes = [P, I, I, P]
+        lib.orc_xattn_aux.argtypes = [P, P, I, I, I, P, I, P]
         _lib = lib
     return _lib
 
@@ -165,6 +166,19 @@ def adapter_fwd(X, nbr, r0, r1, Wd, Wc, Wu, bc=None):
     out = np.empty((r1 - r0, D), dtype=np.float64)
     lib.orc_adapter_fwd(_p(X), _p(nbr), int(r0), int(r1), D, R, _p(_f64(Wd)), _p(_f64(Wc)),
                         _p(_f64(bc)), _p(_f64(Wu)), _p(out))
+    return out
+
+
+def xattn_aux(Hf, goff, aux, heads=1):
+    """Auxiliary tokens aux [G, A, R] updated by attention over the rows of their group
+    (Key Design 3); Hf [n, R] are the keys and values, goff [G+1] the groups' row bounds."""
+    lib = _load()
+    Hf = _f64(Hf)
+    goff = _i32(goff)
+    aux = _f64(aux)
+    G, A, R = aux.shape
+    out = np.empty((G, A, R), dtype=np.float64)
+    lib.orc_xattn_aux(_p(Hf), _p(goff), int(G), int(R), int(heads), _p(aux), int(A), _p(out))
     return out
 
 

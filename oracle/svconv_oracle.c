@@ -277,3 +277,51 @@ void orc_bwd_bias(const double *dY, int n, int Cout, double *db)
     for (int k = 0; k < n; ++k)
         for (int o = 0; o < Cout; ++o) db[o] += dY[(size_t)k * Cout + o];
 }
+
+/* Asymmetric cross-attention of auxiliary tokens over the sparse tokens (SV-TAD page, Key
+ * Design 3, "Asymmetric Cross-Attention for Temporal Recombination"): the auxiliary tokens
+ * (e.g. a CLS token) are the queries, the down-projected sparse visual features are the keys
+ * and the values, and only the auxiliary tokens are updated.
+ * Readings where the page gives only the name: scaled dot-product attention with softmax,
+ * no extra projections (the page names the down-projected features themselves as keys and
+ * values), the R channels split into `heads` heads of R / heads channels each scaled by
+ * 1 / sqrt(R / heads), and the result added to the auxiliary token (residual).  Group g
+ * (a video) owns sparse rows goff[g] .. goff[g+1]-1 and auxiliary tokens g*A .. g*A+A-1;
+ * a group without rows leaves its auxiliary tokens unchanged.
+ *   Hf [n][R], goff [G+1], aux [G][A][R], out [G][A][R]. */
+void orc_xattn_aux(const double *Hf, const int32_t *goff, int G, int R, int heads, const double *aux, int A,
+                   double *out)
+{
+    const int d = R / heads;
+    const double scale = 1.0 / sqrt((double)d);
+    for (int g = 0; g < G; ++g) {
+        const int r0 = goff[g], r1 = goff[g + 1];
+        for (int a = 0; a < A; ++a) {
+            const double *q = aux + ((size_t)g * A + a) * R;
+            double *o = out + ((size_t)g * A + a) * R;
+            for (int c = 0; c < R; ++c) o[c] = q[c];
+            if (r1 <= r0) continue;
+            for (int h = 0; h < heads; ++h) {
+                const int c0 = h * d;
+                /* softmax over the group's rows of the scaled scores, shifted by their maximum */
+                double m = -INFINITY;
+                for (int r = r0; r < r1; ++r) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += q[c0 + c] * Hf[(size_t)r * R + c0 + c];
+                    s *= scale;
+                    if (s > m) m = s;
+                }
+                double den = 0.0;
+                for (int c = 0; c < d; ++c) o[c0 + c] = 0.0;
+                for (int r = r0; r < r1; ++r) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += q[c0 + c] * Hf[(size_t)r * R + c0 + c];
+                    const double p = exp(s * scale - m);
+                    den += p;
+                    for (int c = 0; c < d; ++c) o[c0 + c] += p * Hf[(size_t)r * R + c0 + c];
+                }
+                for (int c = 0; c < d; ++c) o[c0 + c] = q[c0 + c] + o[c0 + c] / den;
+            }
+        }
+    }
+}

@@ -286,3 +286,62 @@ def test_frame_ranges_cover_every_frame_once():
         r = oracle_pool.frame_ranges(off, parts)
         assert r[0][0] == 0 and r[-1][1] == len(off) - 1
         assert all(a < b for a, b in r) and all(r[i][1] == r[i + 1][0] for i in range(len(r) - 1))
+
+
+# ------------------------------------------------------------------ asymmetric cross-attention
+def _xattn_case(seed, G=3, A=2, R=32, heads=2, sizes=(7, 0, 11)):
+    rng = np.random.default_rng(seed)
+    goff = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    H = rng.standard_normal((int(goff[-1]), R))
+    aux = rng.standard_normal((G, A, R))
+    return H, goff, aux
+
+
+def test_xattn_aux_equals_torch_sdpa(orc):
+    """Per group, torch's scaled_dot_product_attention in float64 (heads split the channels),
+    plus the residual; an empty group leaves its auxiliary tokens unchanged."""
+    import torch
+    import torch.nn.functional as F
+    for heads in (1, 2, 4):
+        H, goff, aux = _xattn_case(3 + heads, heads=heads)
+        G, A, R = aux.shape
+        d = R // heads
+        got = orc.xattn_aux(H, goff, aux, heads=heads)
+        for g in range(G):
+            r0, r1 = goff[g], goff[g + 1]
+            if r1 == r0:
+                assert np.array_equal(got[g], aux[g])
+                continue
+            q = torch.from_numpy(aux[g]).view(A, heads, d).permute(1, 0, 2)
+            kv = torch.from_numpy(H[r0:r1]).view(r1 - r0, heads, d).permute(1, 0, 2)
+            att = F.scaled_dot_product_attention(q, kv, kv).permute(1, 0, 2).reshape(A, R).numpy()
+            np.testing.assert_allclose(got[g], aux[g] + att, rtol=1e-12, atol=1e-12)
+
+
+def test_xattn_aux_closed_forms(orc):
+    rng = np.random.default_rng(8)
+    R = 16
+    H = rng.standard_normal((9, R))
+    # a group of one row: the softmax weight is 1, so the update is that row
+    goff = np.array([0, 1, 9], np.int32)
+    aux = rng.standard_normal((2, 1, R))
+    got = orc.xattn_aux(H, goff, aux)
+    np.testing.assert_allclose(got[0, 0], aux[0, 0] + H[0], rtol=0, atol=1e-14)
+    # a zero query scores every row 0: uniform weights, the update is the rows' mean
+    aux0 = np.zeros((2, 1, R))
+    got = orc.xattn_aux(H, goff, aux0)
+    np.testing.assert_allclose(got[1, 0], H[1:9].mean(0), rtol=0, atol=1e-14)
+    # a query far more aligned with one row than with the others (scores ~ 1e3 apart):
+    # the softmax saturates on that row (and nothing overflows)
+    Hs = rng.standard_normal((5, R))
+    q = 300.0 * Hs[3] / np.linalg.norm(Hs[3])
+    Hs[3] = 40.0 * Hs[3] / np.linalg.norm(Hs[3])
+    got = orc.xattn_aux(Hs, np.array([0, 5], np.int32), q.reshape(1, 1, R))
+    np.testing.assert_allclose(got[0, 0], q + Hs[3], rtol=0, atol=1e-9)
+
+
+def test_xattn_aux_row_order_does_not_matter(orc):
+    H, goff, aux = _xattn_case(13, G=2, sizes=(10, 6), heads=1)
+    perm = np.concatenate([np.random.default_rng(1).permutation(10), 10 + np.random.default_rng(2).permutation(6)])
+    np.testing.assert_allclose(orc.xattn_aux(H[perm], goff, aux), orc.xattn_aux(H, goff, aux), rtol=1e-12,
+                               atol=1e-12)
