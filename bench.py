@@ -54,10 +54,11 @@ WORKLOADS = {
     "tiny_f32": ("tiny_f32", 0, "fwd+bwd", "f32"),
     "small_c": ("small_c_bf16", 1, "fwd+bwd", "bf16"),
     "large_c_fwd": ("large_c_fwd_bf16", 2, "fwd", "bf16"),
+    "large_c_fwd_e4m3": ("large_c_fwd_e4m3", 2, "fwd", "e4m3"),
     "large_c_bwd": ("large_c_bwd_bf16", 3, "fwd+bwd", "bf16"),
     "adapter": ("adapter_bf16", 4, "adapter", "bf16"),
 }
-ORDER = ["tiny_f32", "small_c", "large_c_fwd", "large_c_bwd", "adapter"]
+ORDER = ["tiny_f32", "small_c", "large_c_fwd", "large_c_fwd_e4m3", "large_c_bwd", "adapter"]
 HEADLINE = "large_c_bwd"
 
 
@@ -78,15 +79,17 @@ def make_inputs(key, seed_offset=0):
 
 
 # ----------------------------------------------------------------------------- algorithmic work
-def conv_work(n, T, Cin, Cout, elem, bias):
+def conv_work(n, T, Cin, Cout, elem, bias, elem_out=None):
     """Per-launch algorithmic bytes and flops: unique data touched once (features, the
-    neighbour table at 36 B per token, weights, bias, fp32 weight gradients)."""
+    neighbour table at 36 B per token, weights, bias, fp32 weight gradients).  elem: bytes
+    per input / weight element; elem_out: bytes per forward output element (default elem)."""
+    eo = elem if elem_out is None else elem_out
     nbr = 36 * n
     w_bytes = 9 * Cin * Cout * elem
     fl = 2 * n * 9 * Cin * Cout
     return {
         "build_index": {"bytes": 12 * n + 4 * (T + 1) + nbr, "flops": 0},
-        "fwd": {"bytes": n * (Cin + Cout) * elem + nbr + w_bytes + (4 * Cout if bias else 0), "flops": fl},
+        "fwd": {"bytes": n * (Cin * elem + Cout * eo) + nbr + w_bytes + (4 * Cout if bias else 0), "flops": fl},
         "bwd_data": {"bytes": n * (Cin + Cout) * elem + nbr + w_bytes, "flops": fl},
         "bwd_weight": {"bytes": n * (Cin + Cout) * elem + nbr + 4 * (9 * Cin * Cout + Cout), "flops": fl},
     }
@@ -97,25 +100,34 @@ def adapter_work(n, D, R):
             "flops": 2 * n * (D * R + 9 * R * R + R * D)}
 
 
-def floor_seconds(work, peaks, alu=False):
+def flop_peak(peaks, alu=False, fp8=False):
+    """fp32 CUDA-core peak (alu), e4m3 tensor peak (measured bf16 x the nominal 4.5 / 2.25
+    ratio), or the measured bf16 tensor peak."""
+    if alu:
+        return FP32_ALU_TFLOPS
+    return peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+
+
+def floor_seconds(work, peaks, alu=False, fp8=False):
     t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    peak_fl = FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"]
+    peak_fl = flop_peak(peaks, alu, fp8)
     t_fl = work["flops"] / (peak_fl * 1e12) if work["flops"] else 0.0
     return max(t_mem, t_fl)
 
 
-def roofline_entry(work, ms, peaks, alu=False):
-    """The larger of the byte floor (HBM) and the flop floor (bf16 tensor, or fp32 ALU)."""
+def roofline_entry(work, ms, peaks, alu=False, fp8=False):
+    """The larger of the byte floor (HBM) and the flop floor (bf16 or e4m3 tensor, or fp32 ALU)."""
     sec = ms * 1e-3
     t_mem = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    peak_fl = FP32_ALU_TFLOPS if alu else peaks["bf16_tflops"]
+    peak_fl = flop_peak(peaks, alu, fp8)
     t_fl = work["flops"] / (peak_fl * 1e12) if work["flops"] else 0.0
     if t_fl > t_mem:
         achieved = work["flops"] / sec / 1e12
+        note = ("fp32 CUDA-core peak derived from 148 SMs x 128 lanes x FMA x 1.965 GHz" if alu else
+                "e4m3 dense = measured bf16 burst x 2 (nominal 4.5 / 2.25 PFLOP/s)" if fp8 else
+                "bf16 dense, burst (kernel timed alone)")
         return {"bound": "alu" if alu else "tensor", "achieved": achieved, "peak": peak_fl, "unit": "TFLOP/s",
-                "frac": achieved / peak_fl, "algorithmic": work["flops"],
-                "peak_note": ("fp32 CUDA-core peak derived from 148 SMs x 128 lanes x FMA x 1.965 GHz" if alu
-                              else "bf16 dense, burst (kernel timed alone)")}
+                "frac": achieved / peak_fl, "algorithmic": work["flops"], "peak_note": note}
     achieved = work["bytes"] / sec / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "algorithmic": work["bytes"]}
@@ -469,27 +481,31 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
     with_bwd = kind == "fwd+bwd"
     w = make_inputs(key, ctx.rank)  # weak scaling: each rank owns its own batch of frames
     n, T, Cin, Cout = w.n, w.T, w.Cin, w.Cout
-    tdt = torch.float32 if dt_name == "f32" else torch.bfloat16
-    code = sv.F32 if dt_name == "f32" else sv.BF16
-    elem = 4 if dt_name == "f32" else 2
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.float8_e4m3fn}[dt_name]
+    odt = torch.bfloat16 if dt_name == "e4m3" else tdt  # e4m3 inputs give a bf16 output
+    code = {"f32": sv.F32, "bf16": sv.BF16, "e4m3": sv.E4M3}[dt_name]
+    elem = {"f32": 4, "bf16": 2, "e4m3": 1}[dt_name]
+    elem_out = 2 if dt_name == "e4m3" else elem
 
     # pinned host inputs (the end-to-end leg copies these every step)
     h_coords = torch.from_numpy(w.coords).pin_memory()
     h_off = torch.from_numpy(w.frame_off).pin_memory()
     h_X = torch.from_numpy(w.X).to(tdt).pin_memory()
     h_W = torch.from_numpy(w.Wt).to(tdt).pin_memory()
-    h_dY = torch.from_numpy(w.dY).to(tdt).pin_memory()
+    h_dY = torch.from_numpy(w.dY).to(odt).pin_memory()
     h_b = torch.from_numpy(w.bias).pin_memory() if w.bias is not None else None
     coords, off, X, Wt, dY = (t.to(dev) for t in (h_coords, h_off, h_X, h_W, h_dY))
     bias = h_b.to(dev) if h_b is not None else None
     nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
-    Y = torch.empty((n, Cout), dtype=tdt, device=dev)
-    dX = torch.empty((n, Cin), dtype=tdt, device=dev)
+    Y = torch.empty((n, Cout), dtype=odt, device=dev)
+    dX = torch.empty((n, Cin), dtype=odt, device=dev)
     grads = torch.empty((Cout * 9 * Cin + Cout,), dtype=torch.float32, device=dev)
     dW = grads[: Cout * 9 * Cin].view(Cout, 9, Cin)
     db = grads[Cout * 9 * Cin:]
-    ws = torch.empty((max(16, sv.svconv_bwd_weight_workspace_size(code, n, Cin, Cout),
-                          sv.svconv_bwd_workspace_size(code, n, Cin, Cout)),), dtype=torch.uint8, device=dev)
+    ws_code = code if with_bwd else sv.F32
+    ws = torch.empty((max(16, sv.svconv_bwd_weight_workspace_size(ws_code, n, Cin, Cout),
+                          sv.svconv_bwd_workspace_size(ws_code, n, Cin, Cout)) if with_bwd else 16,),
+                     dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def index():
@@ -549,8 +565,8 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
         per["bwd (fused call)"] = ctx.per_kernel([("bwd", bwd)], max(args.steps, 10))["bwd"]
 
     # end to end through the Python API with pinned host buffers
-    h_Y = torch.empty((n, Cout), dtype=tdt).pin_memory()
-    h_dX = torch.empty((n, Cin), dtype=tdt).pin_memory()
+    h_Y = torch.empty((n, Cout), dtype=odt).pin_memory()
+    h_dX = torch.empty((n, Cin), dtype=odt).pin_memory()
     h_grads = torch.empty_like(grads, device="cpu").pin_memory()
     ins = [h_coords, h_off, h_X, h_W, h_dY] + ([h_b] if h_b is not None else [])
     outs = [h_Y] + ([h_dX, h_grads] if with_bwd else [])
@@ -583,10 +599,11 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
 
     peaks = ctx.peaks
     alu = dt_name == "f32"
-    work = conv_work(n, T, Cin, Cout, elem, bias is not None)
+    fp8 = dt_name == "e4m3"
+    work = conv_work(n, T, Cin, Cout, elem, bias is not None, elem_out)
     kern = {}
     for k in [nm for nm, _ in names]:
-        kern[k] = dict(ms=per[k], **roofline_entry(work[k], per[k], peaks, alu=alu and k != "build_index"))
+        kern[k] = dict(ms=per[k], **roofline_entry(work[k], per[k], peaks, alu=alu and k != "build_index", fp8=fp8))
     if with_bwd:
         kern["bwd (fused call)"] = {"ms": per["bwd (fused call)"],
                                    "note": "svconv_bwd: both gradients in one call, as the step runs them"}
@@ -595,7 +612,7 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
     roof["kernel"] = top
     roof["traffic"] = kernel_traffic(key, top)
     roof["peak_source"] = peaks["source"]
-    floors = sum(floor_seconds(work[k], peaks, alu=alu and k != "build_index") for k, _ in names)
+    floors = sum(floor_seconds(work[k], peaks, alu=alu and k != "build_index", fp8=fp8) for k, _ in names)
     step_ms = total_ms / args.steps
     tokens = n * world
     res = {
@@ -855,6 +872,122 @@ def crossover_leg(ctx):
     return out
 
 
+# ----------------------------------------------------------------------------- auxiliary cross-attention
+def xattn_leg(ctx, with_cpu):
+    """Auxiliary-token cross-attention (Key Design 3) at the long-video adapter's size: one
+    CLS token attending over 282,624 down-projected rows of R = 256 (standalone entry point),
+    and the chunked adapter forward with the cross-attention inside it."""
+    import torch
+
+    from sparse_convolution_pruned_b200 import svconv as sv
+    from sparse_convolution_pruned_b200 import workloads as wl
+
+    args, dev, stream = ctx.args, ctx.dev, ctx.stream
+    a = make_inputs("adapter", ctx.rank)
+    n, R, A = a.n, a.R, 1
+    rng = np.random.default_rng(40 + ctx.rank)
+    H_np = wl.round_to_bf16(rng.standard_normal((n, R)).astype(np.float32))
+    aux_np = wl.round_to_bf16(rng.standard_normal((1, A, R)).astype(np.float32))
+    h_H = torch.from_numpy(H_np).to(torch.bfloat16).pin_memory()
+    h_aux = torch.from_numpy(aux_np).to(torch.bfloat16).pin_memory()
+    goff = torch.tensor([0, n], dtype=torch.int32, device=dev)
+    H = h_H.to(dev)
+    aux = h_aux.to(dev)
+    out = torch.empty((1, A, R), dtype=torch.float32, device=dev)
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    ws = torch.empty((max(16, sv.svconv_xattn_workspace_size(1, n, A)),), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def xa():
+        sv.svconv_xattn_aux(H, goff, aux, max_group_rows=n, out=out, workspace=ws, status=status)
+
+    with torch.cuda.stream(stream):
+        xa()
+        stream.synchronize()
+    g = capture(stream, xa)
+    ms = ctx.timed(g.replay, args.steps, args.warmup) / args.steps
+    per = ctx.per_kernel([("xattn", xa)], max(args.steps, 10))["xattn"]
+
+    def e2e():
+        H.copy_(h_H, non_blocking=True)
+        aux.copy_(h_aux, non_blocking=True)
+        xa()
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_ms = ctx.timed(e2e, args.steps, args.warmup) / args.steps
+    ms, per, e2e_ms = ctx.max_over_ranks(ms, per, e2e_ms)
+
+    # the adapter with the cross-attention riding on its chunks
+    chunk_T = args.adapter_chunk_frames
+    offs = a.frame_off.astype(np.int64)
+    max_rows = int(max(offs[min(t + chunk_T, a.T)] - offs[t] for t in range(0, a.T, chunk_T)))
+    coords = torch.from_numpy(a.coords).to(dev)
+    off = torch.from_numpy(a.frame_off).to(dev)
+    X = torch.from_numpy(a.X).to(torch.bfloat16).to(dev)
+    Wd, Wc, Wu = (torch.from_numpy(v).to(torch.bfloat16).to(dev) for v in (a.Wd, a.Wc, a.Wu))
+    nbr = torch.empty((n, 9), dtype=torch.int32, device=dev)
+    aux1 = aux[0]
+    aux_out = torch.empty((A, R), dtype=torch.float32, device=dev)
+    ws2 = torch.empty((max(16, sv.svconv_adapter_xattn_workspace_size(a.T, R, chunk_T, max_rows, A)),),
+                      dtype=torch.uint8, device=dev)
+
+    def index():
+        sv.svconv_build_index(coords, off, a.T, a.H, a.W, nbr=nbr, status=status)
+
+    def ad_x():
+        sv.svconv_adapter_fwd_xattn(X, nbr, off, a.T, Wd, Wc, Wu, aux1, chunk_T=chunk_T, max_chunk_rows=max_rows,
+                                    aux_out=aux_out, workspace=ws2, status=status)
+
+    def ad():
+        sv.svconv_adapter_fwd(X, nbr, off, a.T, Wd, Wc, Wu, chunk_T=chunk_T, max_chunk_rows=max_rows,
+                              workspace=ws2, status=status)
+
+    with torch.cuda.stream(stream):
+        index()
+        ad_x()
+        stream.synchronize()
+    g_ax = capture(stream, ad_x)
+    g_a = capture(stream, ad)
+    ax_ms = ctx.timed(g_ax.replay, args.steps, args.warmup, flush_l2=False) / args.steps
+    a_ms = ctx.timed(g_a.replay, args.steps, args.warmup, flush_l2=False) / args.steps
+    ax_ms, a_ms = ctx.max_over_ranks(ax_ms, a_ms)
+    check_status(sv, status)
+
+    cpu = None
+    if with_cpu:
+        import oracle
+        oracle.build()
+        rows = 20000
+        t0 = time.perf_counter()
+        oracle.xattn_aux(H_np[:rows], np.array([0, rows], np.int32), aux_np)
+        dt = time.perf_counter() - t0
+        cpu = {"value": rows / dt, "unit": "key rows/s", "cores": 1, "kind": "oracle", "host": host_cpu(),
+               "sample": f"one query over the first {rows} of {n} rows (R = {R}); single-threaded C, fp64; "
+                         f"1 core used of {os.cpu_count()}"}
+    work = {"bytes": n * R * 2 + 2 * A * R + 4 * A * R, "flops": 4 * A * n * R}
+    roof = roofline_entry(work, per, ctx.peaks)
+    roof["kernel"] = "xattn_partial_kernel + xattn_combine_kernel"
+    roof["traffic"] = kernel_traffic("xattn", "xattn")
+    roof["peak_source"] = ctx.peaks["source"]
+    n_chunks = (a.T + chunk_T - 1) // chunk_T
+    del g, g_ax, g_a
+    return {
+        "workload": f"xattn_aux_n{n}_R{R}_A{A}_heads1 (rows of the long-video adapter's size)",
+        "value": n / (ms * 1e-3), "unit": "key rows/s", "ms_per_step": ms,
+        "step": "svconv_xattn_aux: one CLS token over one video's down-projected rows",
+        "l2": f"flushed by a {FLUSH_BYTES >> 20} MiB write between timed steps",
+        "roofline": roof, "kernels": {"xattn (both launches)": dict(ms=per, **roofline_entry(work, per, ctx.peaks))},
+        "e2e": {"value": n / (e2e_ms * 1e-3), "unit": "key rows/s", "h2d_bytes_per_step": n * R * 2 + A * R * 2,
+                "d2h_bytes_per_step": A * R * 4},
+        "gpu_launches_per_step": 2,
+        "cpu_baseline": cpu,
+        "in_adapter": {"adapter_fwd_xattn_ms": ax_ms, "adapter_fwd_ms": a_ms, "overhead_ms": ax_ms - a_ms,
+                       "chunk_T": chunk_T, "gpu_launches_per_step": 3 * n_chunks + n_chunks + 1,
+                       "note": "the adapter forward with the cross-attention partials taken after each chunk's "
+                               "down-projection (H1 still in L2) and merged after the last chunk"},
+    }
+
+
 def run_leg(ctx, key, with_cpu, clock_window=False):
     if WORKLOADS[key][2] == "adapter":
         return adapter_leg(ctx, with_cpu, clock_window)
@@ -878,6 +1011,7 @@ def run_b200(args):
         for key in ORDER:
             if key != head_key:
                 configs[key] = run_leg(ctx, key, with_cpu)
+        configs["xattn"] = xattn_leg(ctx, with_cpu)
         if not args.no_crossover:
             configs["crossover"] = crossover_leg(ctx)
 

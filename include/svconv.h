@@ -52,6 +52,7 @@ extern "C" {
 /* element types */
 #define SVCONV_F32 0
 #define SVCONV_BF16 1
+#define SVCONV_E4M3 2 /* svconv_fwd only: 8-bit float (4 exponent, 3 mantissa bits) X and W */
 
 /* host-side return codes */
 #define SVCONV_OK 0
@@ -97,6 +98,10 @@ SVCONV_API int svconv_build_index(const int32_t* coords, const int32_t* frame_of
  *   X [n][Cin], Y [n][Cout] of dtype; Wt [Cout][9][Cin] of dtype;
  *   bias [Cout] fp32 device or NULL.  Y must not alias X.
  *   fp32 limit: 9*Cin*Cout <= 49152.  bf16: Cin, Cout multiples of 64, Cout <= 4096.
+ *   SVCONV_E4M3 (large-channel inference): X [n][Cin] and Wt [Cout][9][Cin] hold e4m3
+ *   values (1 byte each), bias fp32, Y is BF16; products are exact and accumulate in
+ *   fp32 on the tensor cores (kind::f8f6f4, twice the bf16 rate).  Cin a multiple of
+ *   128 and Cout of 256 (both <= 4096); no scaling factors are applied.
  *   bf16 launches: persistent, at most one CTA per SM; output tiles of 256 columns run on
  *   clusters of two CTAs (a pair of SMs shares each 256-row tile), so the device must
  *   allow 2-CTA clusters for those shapes.
@@ -207,6 +212,54 @@ SVCONV_API int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* fr
                        const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T,
                        int max_chunk_rows, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
 SVCONV_API size_t svconv_adapter_workspace_size(int R, int max_chunk_rows);
+
+/*
+ * Asymmetric cross-attention of auxiliary tokens (SV-TAD page, Key Design 3,
+ * "Asymmetric Cross-Attention for Temporal Recombination": auxiliary tokens such as
+ * the CLS token are the queries, the down-projected sparse visual features the keys
+ * and values, and only the auxiliary tokens are updated).  Per group g (a video) and
+ * auxiliary token a, with the R channels split into `heads` heads of d = R / heads:
+ *     aux_out[g][a] = aux[g][a] + softmax_r(aux[g][a] . H[r] / sqrt(d)) H[r]
+ * over the group's rows r = group_off[g] .. group_off[g+1]-1 (per head); a group
+ * with no rows leaves its tokens unchanged.  No extra projections are applied.
+ *   H          [n][R] bf16 device (keys = values), 16-byte aligned.
+ *   group_off  [G+1] int32 DEVICE (CSR over the rows of H).
+ *   max_group_rows  upper bound on any group's rows; a larger group sets
+ *              SVCONV_STATUS_CHUNK_OVERFLOW and only its first rows are used.
+ *   aux        [G][A][R] bf16 device; aux_out [G][A][R] fp32 device.
+ *   workspace  >= svconv_xattn_workspace_size(G, max_group_rows, A) bytes; the
+ *              per-block softmax partials (max, sum, weighted row sum) live there
+ *              and are merged in a fixed order (bitwise reproducible).
+ *   dev_status int32 device or NULL (SVCONV_STATUS_* bits OR-ed in).
+ *   Limits: R a multiple of 8, 8 <= R <= 256; 1 <= A <= 16; R / heads a multiple
+ *   of 8 with R / heads / 8 a power of two.  CUDA cores (HBM-bound: each row of H
+ *   is read once).
+ */
+SVCONV_API int svconv_xattn_aux(const void* H, int n, int R, const int32_t* group_off, int G, int max_group_rows,
+                                const void* aux, int A, int heads, float* aux_out, void* workspace, size_t ws_bytes,
+                                int32_t* dev_status, void* stream);
+SVCONV_API size_t svconv_xattn_workspace_size(int G, int max_group_rows, int A);
+
+/*
+ * The chunked adapter forward of svconv_adapter_fwd with the auxiliary-token
+ * cross-attention inside it (Key Design 3: the cross-attention sits in the
+ * bottleneck adapter, over the down-projected features).  The whole sequence of T
+ * frames is one video: after each chunk's down-projection H1 = bf16(X Wd^T), the
+ * auxiliary tokens' softmax partials over that chunk's rows of H1 are taken (H1 is
+ * still in L2), and after the last chunk they are merged:
+ *     aux_out[a] = aux[a] + softmax_r(aux[a] . H1[r] / sqrt(d)) H1[r]  over all n rows,
+ * H1 being the down-projection of the adapter's INPUT X.  X is updated in place
+ * exactly as by svconv_adapter_fwd.
+ *   aux [A][R] bf16 device, aux_out [A][R] fp32 device; heads as svconv_xattn_aux.
+ *   workspace >= svconv_adapter_xattn_workspace_size(T, R, chunk_T, max_chunk_rows, A).
+ *   Other arguments and limits as svconv_adapter_fwd and svconv_xattn_aux.
+ */
+SVCONV_API int svconv_adapter_fwd_xattn(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D,
+                                        int R, const void* Wd, const void* Wc, const float* bc, const void* Wu,
+                                        int chunk_T, int max_chunk_rows, const void* aux, int A, int heads,
+                                        float* aux_out, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                        void* stream);
+SVCONV_API size_t svconv_adapter_xattn_workspace_size(int T, int R, int chunk_T, int max_chunk_rows, int A);
 
 /*
  * The library's own device error word (per device): kernels without a caller

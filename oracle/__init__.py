@@ -60,6 +60,7 @@ def _load():
         lib.orc_dense_conv.argtypes = [P, I, I, I, I, P, P, P]
         lib.orc_bwd_bias.argtypes = [P, I, I, P]
         lib.orc_xattn_aux.argtypes = [P, P, I, I, I, P, I, P]
+        lib.orc_down_proj.argtypes = [P, I, I, I, P, P]
         _lib = lib
     return _lib
 
@@ -180,6 +181,18 @@ def xattn_aux(Hf, goff, aux, heads=1):
     out = np.empty((G, A, R), dtype=np.float64)
     lib.orc_xattn_aux(_p(Hf), _p(goff), int(G), int(R), int(heads), _p(aux), int(A), _p(out))
     return out
+
+
+def down_proj(X, Wd):
+    """The adapter's first stage alone: bf16(X Wd^T), [n, R]."""
+    lib = _load()
+    X = _f64(X)
+    Wd = _f64(Wd)
+    n, D = X.shape
+    R = Wd.shape[0]
+    H1 = np.empty((n, R), dtype=np.float64)
+    lib.orc_down_proj(_p(X), int(n), int(D), int(R), _p(Wd), _p(H1))
+    return H1
 
 
 def dense_conv(G, Wt, bias=None):

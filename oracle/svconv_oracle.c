@@ -325,3 +325,16 @@ void orc_xattn_aux(const double *Hf, const int32_t *goff, int G, int R, int head
         }
     }
 }
+
+/* The adapter's down-projection on its own: H1 = bf16(X Wd^T) for rows 0 .. n-1, the
+ * same first stage as orc_adapter_fwd (the features the auxiliary tokens attend over).
+ *   X [n][D], Wd [R][D], H1 [n][R]. */
+void orc_down_proj(const double *X, int n, int D, int R, const double *Wd, double *H1)
+{
+    for (int r = 0; r < n; ++r)
+        for (int q = 0; q < R; ++q) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += X[(size_t)r * D + d] * Wd[(size_t)q * D + d];
+            H1[(size_t)r * R + q] = orc_round_bf16(acc);
+        }
+}

@@ -152,6 +152,8 @@ int svconv_fwd(int dtype, const void* X, const int32_t* nbr, int n, int Cin, int
   if (n < 0 || Cin <= 0 || Cout <= 0) return SVCONV_ERR_SIZE;
   if (n == 0) return SVCONV_OK;
   if (!X || !nbr || !Wt || !Y) return SVCONV_ERR_NULL;
+  if (dtype == SVCONV_E4M3 && (Cin % 128 != 0 || Cin > 4096 || Cout % 256 != 0 || Cout > 4096))
+    return SVCONV_ERR_UNSUPPORTED;
   int rc = check_device();
   if (rc) return rc;
   cudaStream_t s = (cudaStream_t)stream;
@@ -159,6 +161,26 @@ int svconv_fwd(int dtype, const void* X, const int32_t* nbr, int n, int Cin, int
     if ((long long)9 * Cin * Cout > 49152) return SVCONV_ERR_UNSUPPORTED;
     return cuda_rc(launch_f32_conv(false, static_cast<const float*>(X), nbr, n, Cin, Cout,
                                    static_cast<const float*>(Wt), Cin, Cout, bias, static_cast<float*>(Y), s));
+  }
+  if (dtype == SVCONV_E4M3) {
+    // e4m3 X and W, bf16 Y: the tensor-core gather on CTA pairs with K = 32 per MMA.  The
+    // kernel moves bytes, so rows of e4m3 are described as rows of half as many 2-byte units.
+    if (!aligned16(X) || !aligned16(Wt) || !aligned16(Y)) return SVCONV_ERR_ALIGN;
+    TcConvArgs a{};
+    a.A = X;
+    a.lda = Cin / 2;
+    a.a_rows = n;
+    a.nbr = nbr;
+    a.taps = 9;
+    a.Kc = Cin / 2;
+    a.M = n;
+    a.N = Cout;
+    a.bias = bias;
+    a.out = Y;
+    a.ldo = Cout;
+    a.out_rows = n;
+    a.f8 = 1;
+    return cuda_rc(launch_tc_conv(a, Wt, Cout, 9 * Cin / 2, 256, s));
   }
   if (dtype != SVCONV_BF16) return SVCONV_ERR_UNSUPPORTED;
   if (!bf16_channels_ok(Cin) || !bf16_channels_ok(Cout)) return SVCONV_ERR_UNSUPPORTED;
@@ -255,25 +277,30 @@ size_t svconv_adapter_workspace_size(int R, int max_chunk_rows) {
   return 2 * rows * (size_t)R * 2;  // H1 and H2, bf16
 }
 
-int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
-                       const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T,
-                       int max_chunk_rows, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
-  if (T < 0 || n < 0 || chunk_T <= 0 || max_chunk_rows <= 0) return SVCONV_ERR_SIZE;
-  if (!bf16_channels_ok(D) || !bf16_channels_ok(R)) return SVCONV_ERR_UNSUPPORTED;
-  if (n == 0 || T == 0) return SVCONV_OK;
-  if (!X || !nbr || !frame_off || !Wd || !Wc || !Wu) return SVCONV_ERR_NULL;
-  if (!aligned16(X) || !aligned16(Wd) || !aligned16(Wc) || !aligned16(Wu) || !aligned16(workspace))
-    return SVCONV_ERR_ALIGN;
-  const size_t need = svconv_adapter_workspace_size(R, max_chunk_rows);
-  if (!workspace || ws_bytes < need) return SVCONV_ERR_WORKSPACE;
-  int rc = check_device();
-  if (rc) return rc;
-  cudaStream_t s = (cudaStream_t)stream;
+}  // extern "C"
+
+namespace svc {
+namespace {
+
+// Auxiliary-token cross-attention riding on the adapter's chunks (nullptr: none).
+struct AdapterXattn {
+  const void* aux;
+  int A, heads;
+  float* aux_out;
+  float* part;
+  int blocks;    // partial blocks per chunk
+  int n_chunks;
+};
+
+int adapter_chunks(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
+                   const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T, int max_chunk_rows,
+                   void* workspace, int32_t* dev_status, const AdapterXattn* xa, cudaStream_t s) {
   const size_t rows_cap = ((size_t)max_chunk_rows + 127) / 128 * 128;
   void* H1 = workspace;
   void* H2 = static_cast<char*>(workspace) + rows_cap * (size_t)R * 2;
   int32_t* status = dev_status ? dev_status : device_error_word();
-  for (int t0 = 0; t0 < T; t0 += chunk_T) {
+  int chunk = 0;
+  for (int t0 = 0; t0 < T; t0 += chunk_T, ++chunk) {
     const int t1 = t0 + chunk_T < T ? t0 + chunk_T : T;
     // 1) H1 = X[rows] Wd^T  (dense, one tap)
     TcConvArgs d{};
@@ -294,6 +321,27 @@ int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, in
     d.status = status;
     cudaError_t e = launch_tc_conv(d, Wd, R, D, conv_bn(R), s);
     if (e != cudaSuccess) return SVCONV_ERR_CUDA;
+    // 1b) auxiliary tokens attend over this chunk's down-projected rows (partials per block)
+    if (xa) {
+      XattnLaunch x{};
+      x.H = H1;
+      x.h_rows = max_chunk_rows;
+      x.R = R;
+      x.heads = xa->heads;
+      x.lo = frame_off + t0;
+      x.hi = frame_off + t1;
+      x.h_sub = frame_off + t0;
+      x.G = 1;
+      x.max_rows = max_chunk_rows;
+      x.aux = xa->aux;
+      x.A = xa->A;
+      x.part = xa->part;
+      x.slot0 = chunk * xa->blocks;
+      x.slots_per_group = xa->n_chunks * xa->blocks;
+      x.status = status;
+      e = launch_xattn_partials(x, s);
+      if (e != cudaSuccess) return SVCONV_ERR_CUDA;
+    }
     // 2) H2 = GELU(SparseConv(H1) + bc), neighbour rows rebased to the chunk
     TcConvArgs c{};
     c.A = H1;
@@ -336,7 +384,111 @@ int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, in
     e = launch_tc_conv(u, Wu, D, R, conv_bn(D), s);
     if (e != cudaSuccess) return SVCONV_ERR_CUDA;
   }
+  if (xa)
+    return cuda_rc(launch_xattn_combine(xa->part, 1, xa->A, R, xa->n_chunks * xa->blocks, xa->aux, xa->aux_out, s));
   return SVCONV_OK;
+}
+
+int adapter_validate(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
+                     const void* Wd, const void* Wc, const void* Wu, int chunk_T, int max_chunk_rows,
+                     void* workspace, size_t ws_bytes, size_t need) {
+  if (T < 0 || n < 0 || chunk_T <= 0 || max_chunk_rows <= 0) return SVCONV_ERR_SIZE;
+  if (!bf16_channels_ok(D) || !bf16_channels_ok(R)) return SVCONV_ERR_UNSUPPORTED;
+  if (n == 0 || T == 0) return SVCONV_OK;
+  if (!X || !nbr || !frame_off || !Wd || !Wc || !Wu) return SVCONV_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Wd) || !aligned16(Wc) || !aligned16(Wu) || !aligned16(workspace))
+    return SVCONV_ERR_ALIGN;
+  if (!workspace || ws_bytes < need) return SVCONV_ERR_WORKSPACE;
+  return check_device();
+}
+
+}  // namespace
+}  // namespace svc
+
+extern "C" {
+
+int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
+                       const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T,
+                       int max_chunk_rows, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  const int rc = adapter_validate(X, nbr, frame_off, T, n, D, R, Wd, Wc, Wu, chunk_T, max_chunk_rows, workspace,
+                                  ws_bytes, svconv_adapter_workspace_size(R, max_chunk_rows));
+  if (rc || n == 0 || T == 0) return rc;
+  return adapter_chunks(X, nbr, frame_off, T, n, D, R, Wd, Wc, bc, Wu, chunk_T, max_chunk_rows, workspace, dev_status,
+                        nullptr, (cudaStream_t)stream);
+}
+
+size_t svconv_xattn_workspace_size(int G, int max_group_rows, int A) {
+  if (G <= 0 || max_group_rows < 0 || A <= 0) return 0;
+  return xattn_partial_bytes((size_t)G * xattn_blocks(max_group_rows), A);
+}
+
+int svconv_xattn_aux(const void* H, int n, int R, const int32_t* group_off, int G, int max_group_rows,
+                     const void* aux, int A, int heads, float* aux_out, void* workspace, size_t ws_bytes,
+                     int32_t* dev_status, void* stream) {
+  if (n < 0 || G < 0 || max_group_rows < 0) return SVCONV_ERR_SIZE;
+  if (!xattn_shape_ok(R, A, heads)) return SVCONV_ERR_UNSUPPORTED;
+  if (G == 0) return SVCONV_OK;
+  if (!group_off || !aux || !aux_out || (n > 0 && !H)) return SVCONV_ERR_NULL;
+  if (!aligned16(H) || !aligned16(aux) || !aligned16(aux_out) || !aligned16(workspace)) return SVCONV_ERR_ALIGN;
+  if (!workspace || ws_bytes < svconv_xattn_workspace_size(G, max_group_rows, A)) return SVCONV_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  XattnLaunch x{};
+  x.H = H;
+  x.h_rows = n;
+  x.R = R;
+  x.heads = heads;
+  x.lo = group_off;
+  x.hi = group_off + 1;
+  x.h_sub = nullptr;
+  x.G = G;
+  x.max_rows = max_group_rows;
+  x.aux = aux;
+  x.A = A;
+  x.part = static_cast<float*>(workspace);
+  x.slot0 = 0;
+  x.slots_per_group = xattn_blocks(max_group_rows);
+  x.status = dev_status ? dev_status : device_error_word();
+  cudaError_t e = launch_xattn_partials(x, s);
+  if (e != cudaSuccess) return SVCONV_ERR_CUDA;
+  return cuda_rc(launch_xattn_combine(x.part, G, A, R, x.slots_per_group, aux, aux_out, s));
+}
+
+size_t svconv_adapter_xattn_workspace_size(int T, int R, int chunk_T, int max_chunk_rows, int A) {
+  if (T <= 0 || R <= 0 || chunk_T <= 0 || max_chunk_rows <= 0 || A <= 0) return 0;
+  const size_t base = (svconv_adapter_workspace_size(R, max_chunk_rows) + 255) / 256 * 256;
+  const int n_chunks = (T + chunk_T - 1) / chunk_T;
+  return base + xattn_partial_bytes((size_t)n_chunks * xattn_blocks(max_chunk_rows), A);
+}
+
+int svconv_adapter_fwd_xattn(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
+                             const void* Wd, const void* Wc, const float* bc, const void* Wu, int chunk_T,
+                             int max_chunk_rows, const void* aux, int A, int heads, float* aux_out, void* workspace,
+                             size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!xattn_shape_ok(R, A, heads)) return SVCONV_ERR_UNSUPPORTED;
+  const int rc = adapter_validate(X, nbr, frame_off, T, n, D, R, Wd, Wc, Wu, chunk_T, max_chunk_rows, workspace,
+                                  ws_bytes, svconv_adapter_xattn_workspace_size(T, R, chunk_T, max_chunk_rows, A));
+  if (rc) return rc;
+  if (!aux || !aux_out) return SVCONV_ERR_NULL;
+  if (!aligned16(aux) || !aligned16(aux_out)) return SVCONV_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n == 0 || T == 0) {  // no rows: nothing to attend over, the auxiliary tokens are copied unchanged
+    const int rc2 = check_device();
+    if (rc2) return rc2;
+    return cuda_rc(launch_xattn_combine(nullptr, 1, A, R, 0, aux, aux_out, s));
+  }
+  AdapterXattn xa{};
+  xa.aux = aux;
+  xa.A = A;
+  xa.heads = heads;
+  xa.aux_out = aux_out;
+  xa.blocks = xattn_blocks(max_chunk_rows);
+  xa.n_chunks = T > 0 ? (T + chunk_T - 1) / chunk_T : 0;
+  const size_t base = (svconv_adapter_workspace_size(R, max_chunk_rows) + 255) / 256 * 256;
+  xa.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + base);
+  return adapter_chunks(X, nbr, frame_off, T, n, D, R, Wd, Wc, bc, Wu, chunk_T, max_chunk_rows, workspace, dev_status,
+                        &xa, s);
 }
 
 int svconv_read_error_word(int32_t* out) {

@@ -183,8 +183,11 @@ cudaError_t launch_f32_conv(bool mirror_bwd, const float* src, const int32_t* nb
   return cudaGetLastError();
 }
 
+// About 16 tokens per split: each thread's token loop is a chain of dependent loads
+// (neighbour index, then the feature row), so short loops keep the kernel off the
+// load-latency path at small n; at most 128 splits.
 size_t f32_wgrad_splits(int n) {
-  int sp = (n + 127) / 128;
+  int sp = (n + 15) / 16;
   if (sp > 128) sp = 128;
   if (sp < 1) sp = 1;
   return (size_t)sp;

@@ -112,6 +112,8 @@ struct TcConvArgs {
   int out_rows;           // rows of out / residual (range check of absolute output rows)
   int32_t* status;        // caller status word or nullptr (library word used otherwise)
   int max_ctas;           // CTA budget (0: one per SM)
+  int f8;                 // A and B hold e4m3 values; lda, Kc and the weight columns count PAIRS
+                          // of them (2-byte units), so byte offsets match the bf16 path
 };
 cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int w_cols, int bn, cudaStream_t s);
 
@@ -135,6 +137,28 @@ int tc_bwd_data(const void* dY, const int32_t* nbr, int n, int Cin, int Cout, co
                 cudaStream_t s);
 int tc_bwd_weight(const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout, float* dW, float* db,
                   float* partial, int ctas, cudaStream_t s);
+
+// ---------------------------------------------------------------- auxiliary-token cross-attention
+constexpr int kXattnMaxQueries = 16;
+struct XattnLaunch {
+  const void* H;            // bf16 keys / values [h_rows][R]
+  int h_rows, R, heads;
+  const int32_t* lo;        // device: group g owns rows lo[g] .. hi[g]-1
+  const int32_t* hi;
+  const int32_t* h_sub;     // device or nullptr: H row = row - *h_sub
+  int G, max_rows;          // groups; rows of the largest group (sets the partial blocks per group)
+  const void* aux;          // bf16 [G][A][R]
+  int A;
+  float* part;              // partial records, slot = g * slots_per_group + slot0 + block
+  int slot0, slots_per_group;
+  int* status;
+};
+bool xattn_shape_ok(int R, int A, int heads);
+size_t xattn_partial_bytes(int slots, int A);
+int xattn_blocks(int max_rows);
+cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s);
+cudaError_t launch_xattn_combine(const float* part, int G, int A, int R, int slots_per_group, const void* aux,
+                                 float* out, cudaStream_t s);
 
 // failure-detection self test
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s);

@@ -411,7 +411,7 @@ __device__ __forceinline__ bool mma_tile(TcBarriers* bar, MmaIssuer& m, int num_
 // A stage holds KBS K-blocks (the last stage of a tile fewer when num_kb is not a
 // multiple): A at 32-column steps in tensor memory, B at b_stage16 / KBS steps.
 // A_TMEM = false: dense GEMM, A stage s in shared memory as well (one K-block per stage).
-template <int GROUP, bool PAIR, int KBS = kGatherKb, bool A_TMEM = true>
+template <int GROUP, bool PAIR, int KBS = kGatherKb, bool A_TMEM = true, bool F8 = false>
 __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, int num_kb, uint32_t d,
                                                  volatile int* abort_flag, int* err, uint64_t timeout_ns) {
   static_assert(A_TMEM || KBS == 1, "dense stages hold one K-block");
@@ -441,7 +441,12 @@ __device__ __forceinline__ bool mma_tile_unified(TcBarriers* bar, MmaIssuer& m, 
           const uint32_t at = m.a_tmem0 + (uint32_t)(m.sa * KBS + h) * kTmemAStageCols;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            if constexpr (PAIR)
+            // F8: the same 32 bytes per row and step hold 32 e4m3 values (K = 32 per MMA)
+            if constexpr (PAIR && F8)
+              tc_mma_f8_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+            else if constexpr (F8)
+              tc_mma_f8_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
+            else if constexpr (PAIR)
               tc_mma_bf16_ts_pair(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
             else
               tc_mma_bf16_ts(d, at + k * 8, bd + (uint64_t)(k * m.b_k16), m.idesc, (kb0 + h) | k ? 1u : 0u);
@@ -674,9 +679,10 @@ __device__ __forceinline__ void epilogue_tma(const TcConvParams& p, uint32_t acc
 // B columns, and CTA rank 0 issues the MMAs for both.  Every SM then streams half of B
 // per 128 output rows.  Barriers that count both CTAs' producers (A and B stages,
 // accumulator release) live in rank 0; the MMA commits arrive in both CTAs.
-template <int BN, bool MIRROR, bool PAIR>
+template <int BN, bool MIRROR, bool PAIR, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_constant__ TcConvParams p) {
   static_assert(!PAIR || BN == 256, "CTA pairs run 256-column tiles");
+  static_assert(!F8 || !MIRROR, "e4m3 operands: forward gather with a K-major weight only");
   extern __shared__ uint8_t smem_raw[];
   const bool gather = p.nbr != nullptr;  // gathered A lives in tensor memory
   const int SA = p.stages_a, SB = p.stages_b;
@@ -1056,7 +1062,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
       MmaCfg c;
-      c.idesc = idesc_bf16_f32(kRows, BN, 0, MIRROR ? 1 : 0);
+      c.idesc = F8 ? idesc_e4m3_f32(kRows, BN, 0, 0) : idesc_bf16_f32(kRows, BN, 0, MIRROR ? 1 : 0);
       c.a_lbo = 16, c.a_sbo = 1024, c.a_step = 32;  // smem A (dense): K-major, 128-byte rows
       if (MIRROR) {
         c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // B: MN-major, 64-wide MN groups 8 KB apart
@@ -1076,7 +1082,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
         constexpr int kGroup = 1;
         bool ok;
         if (gather) {
-          ok = mma_tile_unified<kGroup, PAIR>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+          ok = mma_tile_unified<kGroup, PAIR, kGatherKb, true, F8>(bar, mi, num_kb, tmem_base + ab * BN, abort_flag,
+                                                                   err, p.timeout_ns);
         } else if (res_b) {
           const int nt = tile % n_tiles;
           const int next = tile + units;
@@ -1857,7 +1864,7 @@ static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
 }
 
 // grid: CTAs (PAIR: an even number, two per cluster).
-template <int BN, bool MIRROR, bool PAIR>
+template <int BN, bool MIRROR, bool PAIR, bool F8 = false>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
   const bool a_in_tmem = prm.nbr != nullptr;
   constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns per CTA
@@ -1884,7 +1891,7 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
   const size_t smem = smem_total(conv_geometry(a_in_tmem ? kBCols * kGatherKb : kBCols, prm.stages_a, prm.stages_b,
                                                a_in_tmem, prm.out_tma != 0));
   static int done[64];
-  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR, PAIR>, smem, done);
+  cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR, PAIR, F8>, smem, done);
   if (e != cudaSuccess) return e;
   if constexpr (PAIR) {
     // no more clusters than can be resident at once (the kernel loops over tiles)
@@ -1909,7 +1916,7 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, tc_conv_kernel<BN, MIRROR, PAIR>, &cfg);
+      e = cudaOccupancyMaxActiveClusters(&n, tc_conv_kernel<BN, MIRROR, PAIR, F8>, &cfg);
       if (e != cudaSuccess) return e;
       if (n < 1) return cudaErrorInvalidConfiguration;
       if (d >= 0 && d < 64) occ_smem[d] = (int)smem, occ_clusters[d] = n;
@@ -1918,9 +1925,9 @@ static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s)
       grid = 2 * occ_clusters[d];
     }
     lk.unlock();
-    return launch_pdl_cluster(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
+    return launch_pdl_cluster(tc_conv_kernel<BN, MIRROR, PAIR, F8>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
   } else
-    return launch_pdl(tc_conv_kernel<BN, MIRROR, PAIR>, dim3(grid), dim3(kThreads), smem, s, prm);
+    return launch_pdl(tc_conv_kernel<BN, MIRROR, PAIR, F8>, dim3(grid), dim3(kThreads), smem, s, prm);
 }
 
 template <bool MIRROR>
@@ -1936,6 +1943,9 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   TcConvParams prm;
   memset(&prm, 0, sizeof(prm));
   if (a.mirror != a.b_mn_major) return cudaErrorInvalidValue;  // the data gradient pairs both
+  // e4m3 operands: the forward gather on CTA pairs only (lda, Kc and w_cols count pairs of
+  // e4m3 values, i.e. 2-byte units, so every byte offset below is unchanged)
+  if (a.f8 && (a.mirror || !a.nbr || bn != 256 || a.max_ctas == 1)) return cudaErrorInvalidValue;
   if (a.nbr && a.taps != 9) return cudaErrorInvalidValue;
   // A operand: halo boxes of 64 rows (gather) or the 128-row tile itself (dense)
   if (!make_rows_tmap(&prm.tmap_a, a.A, (uint64_t)a.a_rows, (uint64_t)a.lda, a.nbr ? (uint32_t)kHaloBox : (uint32_t)kBM))
@@ -1991,7 +2001,7 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   if (a.max_ctas > 0 && grid > a.max_ctas) grid = a.max_ctas;
   if (grid > tiles) grid = tiles;
   // 64 gathered channels and 64 output columns, whole-table rows: W-resident small-channel kernel
-  if (a.nbr && a.Kc == 64 && a.N == 64 && bn == 64 && !a.row_lo && !a.a_abs && !a.nbr_abs && !a.out_abs)
+  if (a.nbr && a.Kc == 64 && a.N == 64 && bn == 64 && !a.row_lo && !a.a_abs && !a.nbr_abs && !a.out_abs && !a.f8)
     return a.mirror ? launch_small_inst<true>(prm, grid, s) : launch_small_inst<false>(prm, grid, s);
   if (pair) {
     // one cluster per 256-row tile, at most one CTA per SM
@@ -2000,6 +2010,7 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
     if (a.max_ctas > 0 && clusters > a.max_ctas / 2) clusters = a.max_ctas / 2;
     if (clusters > pair_tiles) clusters = pair_tiles;
     if (clusters < 1) clusters = 1;
+    if (a.f8) return launch_conv_inst<256, false, true, true>(prm, 2 * clusters, s);
     return a.mirror ? launch_conv_inst<256, true, true>(prm, 2 * clusters, s)
                     : launch_conv_inst<256, false, true>(prm, 2 * clusters, s);
   }

@@ -18,7 +18,7 @@ from typing import Optional, Tuple
 
 import torch
 
-F32, BF16 = 0, 1
+F32, BF16, E4M3 = 0, 1, 2
 OK = 0
 STATUS_BAD_COORD, STATUS_DUPLICATE, STATUS_BAD_FRAME, STATUS_BAD_OFFSETS = 1, 2, 4, 8
 STATUS_TIMEOUT, STATUS_BAD_INDEX, STATUS_CHUNK_OVERFLOW = 16, 32, 64
@@ -59,6 +59,14 @@ def lib() -> ctypes.CDLL:
         L.svconv_adapter_fwd.argtypes = [P, P, P, I, I, I, I, P, P, P, P, I, I, P, Z, P, P]
         L.svconv_adapter_workspace_size.argtypes = [I, I]
         L.svconv_adapter_workspace_size.restype = Z
+        L.svconv_xattn_aux.argtypes = [P, I, I, P, I, I, P, I, I, P, P, Z, P, P]
+        L.svconv_xattn_aux.restype = I
+        L.svconv_xattn_workspace_size.argtypes = [I, I, I]
+        L.svconv_xattn_workspace_size.restype = Z
+        L.svconv_adapter_fwd_xattn.argtypes = [P, P, P, I, I, I, I, P, P, P, P, I, I, P, I, I, P, P, Z, P, P]
+        L.svconv_adapter_fwd_xattn.restype = I
+        L.svconv_adapter_xattn_workspace_size.argtypes = [I, I, I, I, I]
+        L.svconv_adapter_xattn_workspace_size.restype = Z
         L.svconv_read_error_word.argtypes = [P]
         L.svconv_selftest_timeout.argtypes = [P, I, P]
         L.svconv_status_str.argtypes = [I]
@@ -112,6 +120,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return F32
     if t.dtype == torch.bfloat16:
         return BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -145,12 +155,13 @@ def svconv_build_index(coords: torch.Tensor, frame_off: torch.Tensor, T: int, H:
 
 def svconv_fwd(X: torch.Tensor, nbr: torch.Tensor, Wt: torch.Tensor, bias: Optional[torch.Tensor] = None, *,
                Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Y[k] = bias + sum_j W_j X[N[k, j]]; Wt is [C_out, 9, C_in]."""
+    """Y[k] = bias + sum_j W_j X[N[k, j]]; Wt is [C_out, 9, C_in].  e4m3 X / Wt give a bf16 Y."""
     _cuda(X, nbr, Wt, bias, Y)
     n, Cin = X.shape
     Cout = Wt.shape[0]
     if Y is None:
-        Y = torch.empty((n, Cout), dtype=X.dtype, device=X.device)
+        ydt = torch.bfloat16 if X.dtype == torch.float8_e4m3fn else X.dtype
+        Y = torch.empty((n, Cout), dtype=ydt, device=X.device)
     rc = lib().svconv_fwd(_dtype_code(X), _ptr(X), _ptr(nbr), n, Cin, Cout, _ptr(Wt), _ptr(bias), _ptr(Y),
                           _stream(X, stream))
     _check("svconv_fwd", rc)
@@ -262,6 +273,58 @@ def svconv_adapter_fwd(X: torch.Tensor, nbr: torch.Tensor, frame_off: torch.Tens
                                   workspace.numel() * workspace.element_size(), _ptr(status), _stream(X, stream))
     _check("svconv_adapter_fwd", rc)
     return X
+
+
+def svconv_xattn_workspace_size(G: int, max_group_rows: int, A: int) -> int:
+    return int(lib().svconv_xattn_workspace_size(int(G), int(max_group_rows), int(A)))
+
+
+def svconv_xattn_aux(H: torch.Tensor, group_off: torch.Tensor, aux: torch.Tensor, *, max_group_rows: int,
+                     heads: int = 1, out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                     status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """aux [G, A, R] bf16 attending over the rows of H [n, R] of their group -> fp32 [G, A, R]."""
+    _cuda(H, group_off, aux, out, workspace, status)
+    n, R = H.shape
+    G, A, _ = aux.shape
+    if out is None:
+        out = torch.empty((G, A, R), dtype=torch.float32, device=aux.device)
+    need = svconv_xattn_workspace_size(G, max_group_rows, A)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=aux.device)
+    rc = lib().svconv_xattn_aux(_ptr(H), n, R, _ptr(group_off), G, int(max_group_rows), _ptr(aux), A, int(heads),
+                                _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(status), _stream(aux, stream))
+    _check("svconv_xattn_aux", rc)
+    return out
+
+
+def svconv_adapter_xattn_workspace_size(T: int, R: int, chunk_T: int, max_chunk_rows: int, A: int) -> int:
+    return int(lib().svconv_adapter_xattn_workspace_size(int(T), int(R), int(chunk_T), int(max_chunk_rows), int(A)))
+
+
+def svconv_adapter_fwd_xattn(X: torch.Tensor, nbr: torch.Tensor, frame_off: torch.Tensor, T: int, Wd: torch.Tensor,
+                             Wc: torch.Tensor, Wu: torch.Tensor, aux: torch.Tensor, bc: Optional[torch.Tensor] = None, *,
+                             chunk_T: int, max_chunk_rows: int, heads: int = 1,
+                             aux_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None):
+    """The chunked adapter forward (X in place) plus the auxiliary tokens aux [A, R] attending
+    over the down-projected rows of the whole sequence -> (X, aux_out fp32 [A, R])."""
+    _cuda(X, nbr, frame_off, Wd, Wc, Wu, aux, bc, aux_out, workspace, status)
+    n, D = X.shape
+    R = Wd.shape[0]
+    A = aux.shape[0]
+    if aux_out is None:
+        aux_out = torch.empty((A, R), dtype=torch.float32, device=X.device)
+    need = svconv_adapter_xattn_workspace_size(T, R, chunk_T, max_chunk_rows, A)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=X.device)
+    rc = lib().svconv_adapter_fwd_xattn(_ptr(X), _ptr(nbr), _ptr(frame_off), int(T), n, D, R, _ptr(Wd), _ptr(Wc),
+                                        _ptr(bc), _ptr(Wu), int(chunk_T), int(max_chunk_rows), _ptr(aux), A,
+                                        int(heads), _ptr(aux_out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _ptr(status),
+                                        _stream(X, stream))
+    _check("svconv_adapter_fwd_xattn", rc)
+    return X, aux_out
 
 
 def svconv_read_error_word() -> int:

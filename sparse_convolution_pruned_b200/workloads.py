@@ -47,6 +47,15 @@ def round_to_bf16(x: np.ndarray) -> np.ndarray:
     return x
 
 
+def round_to_e4m3(x: np.ndarray) -> np.ndarray:
+    """Float32 samples rounded to the nearest value of the 8-bit float e4m3 (4 exponent, 3
+    mantissa bits, largest finite 448), using torch's float8_e4m3fn conversion.  Returns
+    float32 values exactly representable in e4m3.  Inputs lie well inside +-448."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float32).numpy()
+
+
 def _normal(rng: np.random.Generator, shape, var: float, bf16: bool) -> np.ndarray:
     a = rng.standard_normal(size=shape, dtype=np.float32)
     if var != 1.0:
@@ -195,6 +204,16 @@ def large_c_fwd_bf16(seed: int = 2, T: int = 384, C: int = 256) -> ConvWorkload:
                          rng=rng, seed=seed)
 
 
+def large_c_fwd_e4m3(seed: int = 2, T: int = 384, C: int = 256) -> ConvWorkload:
+    """The large-channel forward workload with X and W rounded to e4m3 (8-bit inference)."""
+    w = large_c_fwd_bf16(seed=seed, T=T, C=C)
+    w.X = round_to_e4m3(w.X)
+    w.Wt = round_to_e4m3(w.Wt)
+    w.dtype = "e4m3"
+    w.name = f"large_c_fwd_e4m3_T{T}_16x16_keep50_C{C}"
+    return w
+
+
 def large_c_bwd_bf16(seed: int = 3, T: int = 384, C: int = 256) -> ConvWorkload:
     """As the large-channel forward, but the keep ratio r_t ~ U(0.2, 0.8) varies per frame."""
     rng = np.random.default_rng(seed)
@@ -249,6 +268,7 @@ CONFIGS = {
     "tiny_f32": tiny_f32,
     "small_c_bf16": small_c_bf16,
     "large_c_fwd_bf16": large_c_fwd_bf16,
+    "large_c_fwd_e4m3": large_c_fwd_e4m3,
     "large_c_bwd_bf16": large_c_bwd_bf16,
     "adapter_bf16": adapter_bf16,
 }

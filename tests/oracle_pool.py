@@ -57,6 +57,12 @@ def _adapter_task(task):
     return oracle.adapter_fwd(X, sub_n, 0, X.shape[0], Wd, Wc, Wu)
 
 
+def _down_task(task):
+    import oracle
+    X, Wd = task
+    return oracle.down_proj(X, Wd)
+
+
 def _workers():
     return max(1, min(32, os.cpu_count() or 1))
 
@@ -92,4 +98,16 @@ def adapter_full(a, nbr):
         tasks.append((a.X[r0:r1], _rebase(nbr, r0, r1), a.Wd, a.Wc, a.Wu))
     with mp.get_context("spawn").Pool(workers) as pool:
         parts = pool.map(_adapter_task, tasks, chunksize=1)
+    return np.concatenate(parts, 0)
+
+
+def down_proj_full(X, Wd):
+    """Oracle down-projection bf16(X Wd^T) of every row, rows split over worker processes
+    (each row is independent)."""
+    workers = _workers()
+    n = X.shape[0]
+    cuts = np.linspace(0, n, 4 * workers + 1).astype(np.int64)
+    tasks = [(X[a:b], Wd) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+    with mp.get_context("spawn").Pool(workers) as pool:
+        parts = pool.map(_down_task, tasks, chunksize=1)
     return np.concatenate(parts, 0)

@@ -51,7 +51,13 @@ def test_host_validation_runs_before_any_device_call(L):
     assert L.svconv_adapter_fwd(fake, fake, fake, 4, 10, 1000, 256, fake, fake, None, fake, 2, 64, fake, 1 << 20,
                                 None, None) == -3
     # workspace sizes (pure host arithmetic for fp32)
-    assert sv.svconv_bwd_weight_workspace_size(sv.F32, 128, 16, 16) == 1 * (9 * 16 + 1) * 16 * 4
+    # fp32: one split per 16 tokens (at most 128), each split 9 C_in + 1 rows of C_out floats
+    assert sv.svconv_bwd_weight_workspace_size(sv.F32, 128, 16, 16) == 8 * (9 * 16 + 1) * 16 * 4
+    assert sv.svconv_bwd_weight_workspace_size(sv.F32, 100000, 16, 16) == 128 * (9 * 16 + 1) * 16 * 4
+    # the cross-attention partials: blocks of 256 rows, A records of 10 x 32 floats each
+    assert sv.svconv_xattn_workspace_size(3, 600, 2) == 3 * 3 * 2 * 10 * 32 * 4
+    # e4m3 forward: channel counts are checked before any device call
+    assert L.svconv_fwd(sv.E4M3, fake, fake, 10, 64, 256, fake, None, fake, None) == -3
     assert sv.svconv_bwd_weight_workspace_size(sv.F32, 0, 16, 16) == 0
     assert sv.svconv_adapter_workspace_size(256, 100) == 2 * 128 * 256 * 2
 

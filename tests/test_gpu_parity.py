@@ -390,3 +390,54 @@ def test_bad_neighbour_index_is_flagged_not_faulted(sv):
     sv.svconv_bwd_weight(X, X, nbr)
     assert sv.svconv_read_error_word() & sv.STATUS_BAD_INDEX
     assert sv.svconv_read_error_word() == 0  # reading clears it
+
+
+# ------------------------------------------------------------------ e4m3 forward (large channels)
+def run_e4m3_fwd(sv, w):
+    nbr, _, st = gpu_index(sv, w, want_map=False)
+    assert st == 0
+    X = dev(w.X).to(torch.float8_e4m3fn)
+    Wt = dev(w.Wt).to(torch.float8_e4m3fn)
+    assert torch.equal(X.float().cpu(), torch.from_numpy(w.X))  # the inputs are e4m3 values already
+    b = dev(w.bias) if w.bias is not None else None
+    Y = sv.svconv_fwd(X, nbr, Wt, b)
+    Y2 = sv.svconv_fwd(X, nbr, Wt, b)
+    torch.cuda.synchronize()
+    assert Y.dtype == torch.bfloat16 and torch.equal(Y, Y2)
+    return Y.float().cpu().numpy()
+
+
+E4M3_CASES = [
+    ("C256_T24", lambda: wl.large_c_fwd_e4m3(T=24)),
+    ("C128x256_ragged_shuffled", lambda: wl.custom_conv(seed=35, T=7, H=9, W=14, keep_frac=0.55, Cin=128, Cout=256,
+                                                        dtype="bf16", shuffle=True, empty_frames=(3,))),
+    ("C384x512_wide_grid", lambda: wl.custom_conv(seed=36, T=4, H=5, W=80, keep_frac=0.6, Cin=384, Cout=512,
+                                                  dtype="bf16")),
+]
+
+
+@pytest.mark.parametrize("name,make", E4M3_CASES, ids=[c[0] for c in E4M3_CASES])
+def test_e4m3_fwd(sv, orc, name, make):
+    w = make()
+    w.X, w.Wt = wl.round_to_e4m3(w.X), wl.round_to_e4m3(w.Wt)
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    check_bf16(run_e4m3_fwd(sv, w), orc.fwd(w.X, ref_n, w.Wt, w.bias), "Y e4m3")
+    assert sv.svconv_read_error_word() == 0
+
+
+def test_e4m3_fwd_full_size_complete(sv, orc):
+    import oracle_pool
+    w = wl.large_c_fwd_e4m3()
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    Y = run_e4m3_fwd(sv, w)
+    check_bf16(Y, oracle_pool.conv_full(w, ref_n, do_fwd=True, do_bwd=False)["Y"], "Y e4m3 full size")
+    assert sv.svconv_read_error_word() == 0
+
+
+def test_e4m3_rejects_unsupported_channels(sv):
+    X = torch.zeros((10, 64), dtype=torch.float8_e4m3fn, device="cuda")
+    nbr = torch.zeros((10, 9), dtype=torch.int32, device="cuda")
+    Wt = torch.zeros((256, 9, 64), dtype=torch.float8_e4m3fn, device="cuda")
+    with pytest.raises(sv.SvconvError) as e:
+        sv.svconv_fwd(X, nbr, Wt)  # C_in = 64 is not a multiple of 128
+    assert e.value.code == -3

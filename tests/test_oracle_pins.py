@@ -345,3 +345,13 @@ def test_xattn_aux_row_order_does_not_matter(orc):
     perm = np.concatenate([np.random.default_rng(1).permutation(10), 10 + np.random.default_rng(2).permutation(6)])
     np.testing.assert_allclose(orc.xattn_aux(H[perm], goff, aux), orc.xattn_aux(H, goff, aux), rtol=1e-12,
                                atol=1e-12)
+
+
+def test_down_proj_equals_torch_matmul_then_bf16(orc):
+    """The adapter's first stage: float64 matmul, then torch's round-to-nearest-even bf16 cast."""
+    import torch
+    rng = np.random.default_rng(21)
+    X = rng.standard_normal((37, 64))
+    Wd = rng.standard_normal((16, 64)) / 8
+    want = (torch.from_numpy(X) @ torch.from_numpy(Wd).T).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(orc.down_proj(X, Wd), want)
