@@ -812,7 +812,7 @@ def crossover_leg(ctx):
                     "every step replayed from a CUDA graph, L2 flushed between steps",
            "keeps": CROSSOVER_KEEPS, "curves": {}}
     for C in CROSSOVER_CHANNELS:
-        cur = {"sparse_fwd_ms": [], "sparse_fwd_with_index_ms": [], "dense_fwd_ms": [],
+        cur = {"sparse_fwd_ms": [], "sparse_fwd_with_index_ms": [], "dense_fwd_ms": [], "dense_conv_only_ms": [],
                "sparse_fwd_bwd_ms": [], "dense_fwd_bwd_ms": [], "n_kept": []}
         for keep in CROSSOVER_KEEPS:
             k = int(round(keep * 256))
@@ -831,6 +831,7 @@ def crossover_leg(ctx):
                              device=dev)
             wtorch = torch_weight(Wt)
             dense = DenseRecon(coords, w.T, w.H, w.W)
+            grid_in = dense.scatter(X).contiguous(memory_format=torch.channels_last)
 
             def index():
                 sv.svconv_build_index(coords, off, w.T, w.H, w.W, nbr=nbr)
@@ -853,6 +854,7 @@ def crossover_leg(ctx):
                 "sparse_fwd_ms": capture(stream, s_fwd),
                 "sparse_fwd_with_index_ms": capture(stream, lambda: (index(), s_fwd())),
                 "dense_fwd_ms": capture(stream, lambda: dense.fwd(X, wtorch)),
+                "dense_conv_only_ms": capture(stream, lambda: torch.nn.functional.conv2d(grid_in, wtorch, padding=1)),
                 "sparse_fwd_bwd_ms": capture(stream, s_fwd_bwd),
                 "dense_fwd_bwd_ms": capture(stream, lambda: dense.fwd_bwd(X, wtorch, dY)),
             }
@@ -865,10 +867,13 @@ def crossover_leg(ctx):
         cur["crossover_keep_fwd_with_index"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_with_index_ms"],
                                                         cur["dense_fwd_ms"])
         cur["crossover_keep_fwd_bwd"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_bwd_ms"], cur["dense_fwd_bwd_ms"])
+        cur["crossover_keep_fwd_vs_conv_only"] = crossing(CROSSOVER_KEEPS, cur["sparse_fwd_ms"],
+                                                          cur["dense_conv_only_ms"])
         out["curves"][f"C{C}"] = cur
     out["note"] = ("crossover_keep_* = keep rate where the sparse time meets the dense time (linear between "
-                   "sweep points); null = sparse faster at every swept keep rate.  The page reports 55% on its "
-                   "own (unstated) hardware")
+                   "sweep points); null = sparse faster at every swept keep rate.  dense_conv_only = the cuDNN "
+                   "convolution alone on an already scattered grid (no scatter, no gather).  The page reports 55% "
+                   "on its own (unstated) hardware")
     return out
 
 

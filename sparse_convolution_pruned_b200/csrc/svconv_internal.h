@@ -131,6 +131,13 @@ void tc_wgrad_plan_ctas(int n, int Cin, int Cout, int ctas, int* splits, int* ro
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s);
 cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s);
 
+// Single-pass backward at C_in = C_out = 64 (bf16): data gradient, weight-gradient partials
+// [tc_bwd_small_grid(n)][640][64] and their fixed-order reduce into dW / db.
+int tc_bwd_small_grid(int n);
+size_t tc_bwd_small_partial_floats(int n);
+cudaError_t launch_tc_bwd_small(const void* dY, const void* X, const int32_t* nbr, int n, const void* Wt, void* dX,
+                                float* partial, float* dW, float* db, cudaStream_t s);
+
 // bf16 tensor-core bodies of the data / weight gradients (arguments already validated);
 // max_ctas / ctas: CTA budget (0: all SMs).  Return SVCONV_* codes.
 int tc_bwd_data(const void* dY, const int32_t* nbr, int n, int Cin, int Cout, const void* Wt, void* dX, int max_ctas,

@@ -1456,7 +1456,7 @@ struct Regs16 {
   uint32_t v[16];
 };
 __device__ __noinline__ Regs16 wgrad_patch_far(Regs16 R, uint32_t sidx_s, const uint16_t* X16, int n, int Cin, int k0,
-                                               int hlo, int j, int ch0) {
+                                               int hlo, int j, int ch0, int win = kWgHaloRows) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
@@ -1466,7 +1466,7 @@ __device__ __noinline__ Regs16 wgrad_patch_far(Regs16 R, uint32_t sidx_s, const 
     for (int e = 0; e < 2; ++e) {
       const int tk = 16 * k4 + 8 * (m >> 1) + 2 * (lane & 3) + e;
       const int x = k0 + tk < n ? ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j)) : -1;
-      if (x >= 0 && x < n && (unsigned)(x - hlo) >= (unsigned)kWgHaloRows) {
+      if (x >= 0 && x < n && (unsigned)(x - hlo) >= (unsigned)win) {
         const uint32_t v = __ldg(X16 + (size_t)x * Cin + ch);
         R.v[r] = e == 0 ? ((R.v[r] & 0xFFFF0000u) | v) : ((R.v[r] & 0x0000FFFFu) | (v << 16));
       }
@@ -1772,6 +1772,396 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   }
 }
 
+// ============================================================================ single-pass backward, 64 channels
+// Both gradients of a C_in = C_out = 64 convolution in ONE pass over dY (SV-TAD page, Key
+// Design 2: the dedicated backward kernels; both are adjoints of the forward):
+//   dX[k]          = sum_j W_j^T dY[N[k][8-j]]                (mirrored gather, as tc_conv_small)
+//   dW^T[(j,i)][o] += sum_{k in tile} X[N[k][j]][i] dY[k][o]  (gathered X transposed, as tc_wgrad)
+// For each 128-token tile the loader brings the dY halo window (rows m0-32 .. m0+159), the X
+// halo window over the same rows and the tile's neighbour entries once.  The dY window feeds
+// the data gradient's gather AND, read in place as the MN-major B operand (its rows 32..159
+// are the tile's own tokens), the weight gradient's MMAs; so dY crosses L2 -> SM once.
+// The 640 x 64 fp32 weight-gradient accumulators (taps 0..8 and the db half, as in tc_wgrad)
+// stay in tensor memory for all tiles of the CTA and are written once at the end as the
+// CTA's split partial; the fixed-order split reduce turns them into dW and db.
+// Tensor memory: dW^T accumulators (5 x 64 columns), the dX accumulator (64), and a ring of
+// four 32-column A stages shared by both kinds of stage (19 per tile: 9 taps, 10 blocks).
+constexpr int kFbStages = 4;
+constexpr int kFbMTiles = 5;
+constexpr int kFbStagesPerTile = 9 + 2 * kFbMTiles;
+constexpr uint32_t kFbDxCol = kFbMTiles * 64;        // 320
+constexpr uint32_t kFbACol = kFbDxCol + 64;          // 384
+constexpr uint32_t kFbTmemCols = 512;
+constexpr uint32_t kFbHaloBytes = kConvHaloRows * 128;
+constexpr int kFbRowsPad = kFbMTiles * kBM;          // 640 partial rows
+
+struct FbParams {
+  CUtensorMap tmap_dy;  // dY [n][64], boxes {64, 64}
+  CUtensorMap tmap_x;   // X [n][64], boxes {64, 64}
+  CUtensorMap tmap_w;   // W as (i, j, o), box (64, 1, 64): W_j^T, MN-major
+  const __nv_bfloat16* dY;
+  const __nv_bfloat16* X;
+  const int32_t* nbr;
+  __nv_bfloat16* dX;
+  float* partial;       // [gridDim.x][640][64]
+  int* status;
+  unsigned long long timeout_ns;
+  int n;
+};
+
+struct __align__(16) FbBars {
+  uint32_t zero128[32];  // 128 zero bytes
+  uint64_t wfull;
+  uint64_t lfull[2], lempty[2];                   // tile slots: index entries + both halos
+  uint64_t afull[kFbStages], aempty[kFbStages];   // A stages in tensor memory
+  uint64_t tfull, tempty;                         // dX accumulator
+  uint64_t dwfull;                                // all weight-gradient MMAs of the CTA done
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__host__ __device__ constexpr size_t fb_smem_bytes() {
+  return 1024 + kSmallWBytes + 4 * (size_t)kFbHaloBytes + 2 * (size_t)kConvIdx * 4 + sizeof(FbBars);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) tc_bwd_small_kernel(const __grid_constant__ FbParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  uint8_t* sw = smem_raw + (((sbase + 1023u) & ~1023u) - sbase);
+  uint8_t* shalo = sw + kSmallWBytes;  // slot s: dY window at 2 s H, X window at (2 s + 1) H
+  int32_t* sidx = reinterpret_cast<int32_t*>(shalo + 4 * kFbHaloBytes);
+  FbBars* bar = reinterpret_cast<FbBars*>(reinterpret_cast<uint8_t*>(sidx) + 2 * kConvIdx * 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* err = p.status;
+  const int M = p.n;
+  const int num_tiles = (M + kBM - 1) / kBM;
+  auto dy_win = [&](int slot) { return smem_u32(shalo + (size_t)(2 * slot) * kFbHaloBytes); };
+  auto x_win = [&](int slot) { return smem_u32(shalo + (size_t)(2 * slot + 1) * kFbHaloBytes); };
+
+  auto issue_tile = [&](int tile, int slot) {
+    const int m0 = tile * kBM;
+    const int32_t* src = p.nbr + (size_t)m0 * 9;
+    const int lim = min(M - m0, kBM) * 9;
+    copy_index_entries(smem_u32(sidx + slot * kConvIdx), src, lim, ((reinterpret_cast<uintptr_t>(src) & 15u) == 0),
+                       &bar->lfull[slot], 2 * kFbHaloBytes);
+    if (lane == 0) {
+#pragma unroll
+      for (int q = 0; q < kConvHaloRows / kHaloBox; ++q) {
+        tma_load_2d(dy_win(slot) + q * kHaloBox * 128, &p.tmap_dy, &bar->lfull[slot], 0, m0 - kConvPad + q * kHaloBox);
+        tma_load_2d(x_win(slot) + q * kHaloBox * 128, &p.tmap_x, &bar->lfull[slot], 0, m0 - kConvPad + q * kHaloBox);
+      }
+    }
+    __syncwarp();
+  };
+
+  // ---- setup
+  uint32_t issued = 0;
+  if (warp == kHaloWarp) {
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bar->lfull[i], 33);              // 32 cp.async arrivals + the expect_tx arrival
+        mbar_init(&bar->lempty[i], kProdWarps + 1);  // the builder warps + the MMAs that read dY in place
+      }
+      fence_barrier_init();
+      fence_proxy_async_smem();
+      prefetch_tmap(&p.tmap_dy);
+      prefetch_tmap(&p.tmap_x);
+    }
+    __syncwarp();
+    pdl_wait();
+    for (int t = blockIdx.x; t < num_tiles && issued < 2; t += gridDim.x) issue_tile(t, (int)issued++);
+  } else if (warp == kBWarp) {
+    if (lane == 0) {
+      mbar_init(&bar->wfull, 1);
+      fence_barrier_init();
+      fence_proxy_async_smem();
+      pdl_wait();
+      mbar_arrive_expect_tx(&bar->wfull, kSmallWBytes);
+      const uint32_t dst = smem_u32(sw);
+      for (int j = 0; j < 9; ++j) tma_load_3d(dst + j * 8192, &p.tmap_w, &bar->wfull, 0, j, 0);
+    }
+    __syncwarp();
+  } else if (threadIdx.x == 0) {
+    for (int i = 0; i < 32; ++i) bar->zero128[i] = 0u;
+    for (int s = 0; s < kFbStages; ++s) {
+      mbar_init(&bar->afull[s], kProdWarps / 2);
+      mbar_init(&bar->aempty[s], 1);
+    }
+    mbar_init(&bar->tfull, 1);
+    mbar_init(&bar->tempty, kEpiWarps);
+    mbar_init(&bar->dwfull, 1);
+    bar->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bar->tmem_base, kFbTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t tmem_base = bar->tmem_base;
+  volatile int* abort_flag = &bar->abort_flag;
+
+  if (warp == kHaloWarp) {
+    // ------------------------------------------------------------ loader (tiles 2, 3, ...)
+    bool aborted = false;
+    uint32_t ti = issued;
+    for (int tile = blockIdx.x + (int)issued * gridDim.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      const int slot = ti & 1;
+      if (!warp_wait(&bar->lempty[slot], ring_parity(ti, 2) ^ 1u, abort_flag, err, p.timeout_ns)) {
+        aborted = true;
+        break;
+      }
+      issue_tile(tile, slot);
+      ++issued;
+    }
+    if (aborted) drain_ring(bar->lfull, issued, 2, err, p.timeout_ns);
+  } else if (warp == kBWarp) {
+    if (lane == 0) {  // W stays resident; its copy must land before the CTA can exit
+      volatile int never = 0;
+      mbar_wait(&bar->wfull, 0, &never, err, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp >= kEpiWarps && warp < kHaloWarp) {
+    // ------------------------------------------------------------ A builders
+    // Stage q of the CTA (19 per tile) goes to ring slot q % 4 and is built by the group of
+    // four warps q % 2.  Taps 0..8: thread (quarter, lane) writes token row 32 quarter + lane
+    // of dY[N[k][8-j]] (32x32b store).  Weight-gradient block (mt, tb): the transposed gather
+    // of tc_wgrad over tokens m0 + 64 tb .. + 63, half (quarter / 2) of M-tile mt, channels
+    // 32 (quarter % 2) .. + 31 (16x128b stores).
+    const int grp = (warp - kEpiWarps) >> 2;
+    const int quarter = warp & 3;
+    const uint32_t zero_row = smem_u32(bar->zero128);
+    const uint16_t* X16 = reinterpret_cast<const uint16_t*>(p.X);
+    uint32_t q = 0, ti = 0;
+    bool aborted = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !aborted; tile += gridDim.x, ++ti, q += kFbStagesPerTile) {
+      const int slot = ti & 1;
+      if (!warp_wait(&bar->lfull[slot], ring_parity(ti, 2), abort_flag, err, p.timeout_ns)) break;
+      const int m0 = tile * kBM;
+      const int hlo = m0 - kConvPad;
+      const uint32_t si_s = smem_u32(sidx + slot * kConvIdx);
+      for (int t = 0; t < kFbStagesPerTile; ++t) {
+        const uint32_t qq = q + (uint32_t)t;
+        if ((int)(qq & 1u) != grp) continue;
+        const int st = (int)(qq % kFbStages);
+        if (!warp_wait(&bar->aempty[st], ring_parity(qq, kFbStages) ^ 1u, abort_flag, err, p.timeout_ns)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();  // the MMAs that read this stage are complete
+        const uint32_t a_col = tmem_base + kFbACol + (uint32_t)st * kTmemAStageCols;
+        if (t < 9) {
+          const int j = t;
+          const int r = quarter * 32 + lane;
+          const bool row_ok = m0 + r < M;
+          const uint32_t halo = dy_win(slot);
+          const int raw = row_ok ? ld_shared_s32(si_s + 4u * (uint32_t)(r * 9 + (8 - j))) : -1;
+          const bool bad = (raw >= 0) & ((unsigned)raw >= (unsigned)M);
+          const int idx = bad ? -1 : raw;
+          const int h = idx - hlo;
+          const bool in_win = (idx >= 0) & ((unsigned)h < (unsigned)kConvHaloRows);
+          const uint32_t row = in_win ? halo + (uint32_t)h * 128u : zero_row;
+          const int swz = in_win ? (h & 7) : 0;
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 u = ld_shared_16(row + ((c ^ swz) << 4));
+            v[4 * c] = u.x, v[4 * c + 1] = u.y, v[4 * c + 2] = u.z, v[4 * c + 3] = u.w;
+          }
+          const bool far = (idx >= 0) & !in_win;
+          if (__any_sync(0xffffffffu, far | bad)) {
+            if (bad) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+            if (far) {
+              const __nv_bfloat16* src = p.dY + (size_t)idx * 64;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint4 u = ldg_16(src + c * 8);
+                v[4 * c] = u.x, v[4 * c + 1] = u.y, v[4 * c + 2] = u.z, v[4 * c + 3] = u.w;
+              }
+            }
+          }
+          tmem_st_32x32b_x32(a_col + ((uint32_t)(quarter * 32) << 16), v);
+        } else {
+          const int mt = (t - 9) >> 1, tb = (t - 9) & 1;
+          const int half = quarter >> 1;
+          const int cq = (quarter & 1) * 32;
+          const int j = 2 * mt + half;  // 9: the extra half (its row 0 gives db)
+          const int k0 = m0 + tb * kBK;
+          const uint32_t sidx_b = si_s + 4u * (uint32_t)(tb * kBK * 9);
+          if (j < 9) {
+            const uint32_t halo = x_win(slot);
+            const int mi = lane >> 3;
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+              const int c16 = cq + 16 * sub;
+              uint32_t R[16];
+              bool far = false, bad = false;
+              const int chunk = (c16 >> 3) + (mi & 1);
+#pragma unroll
+              for (int k4 = 0; k4 < 4; ++k4) {
+                const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
+                const int raw = ld_shared_s32(sidx_b + 4u * (uint32_t)(tk * 9 + j));
+                const bool tok_ok = k0 + tk < M;
+                bad |= tok_ok & (raw >= M);
+                const int x = (tok_ok & (raw < M)) ? raw : -1;
+                const int h = x - hlo;
+                const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kConvHaloRows);
+                far |= (x >= 0) & !in_win;
+                const uint32_t addr =
+                    in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_row;
+                ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
+              }
+              if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+              if (__any_sync(0xffffffffu, far)) {
+                Regs16 rr;
+#pragma unroll
+                for (int r2 = 0; r2 < 16; ++r2) rr.v[r2] = R[r2];
+                rr = wgrad_patch_far(rr, sidx_b, X16, M, 64, k0, hlo, j, c16, kConvHaloRows);
+#pragma unroll
+                for (int r2 = 0; r2 < 16; ++r2) R[r2] = rr.v[r2];
+              }
+              tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+            }
+          } else {
+            // row 0 of the extra half is 1 for every valid token: its accumulator row is db
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+              uint32_t R[16];
+#pragma unroll
+              for (int r2 = 0; r2 < 16; ++r2) R[r2] = 0u;
+              if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const int tk = k0 + 8 * k + 2 * lane;
+                  R[2 * k] = (tk < M ? 0x3F80u : 0u) | (tk + 1 < M ? 0x3F800000u : 0u);
+                }
+              }
+              tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+            }
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(&bar->afull[st]);
+      }
+      if (aborted) break;
+      warp_arrive(&bar->lempty[slot]);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer: 36 + 40 MMAs per tile
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, 64, 0, 1);  // A from tensor memory, B MN-major (W^T and dY)
+      const uint64_t bw0 = smem_desc_sw128(smem_u32(sw), 8192, 1024);
+      constexpr uint32_t k16 = 2048u >> 4;  // 16 K rows of an MN-major operand per MMA
+      bool ok = true;
+      if (mbar_wait(&bar->wfull, 0, abort_flag, err, p.timeout_ns)) {
+        uint32_t q = 0, ti = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++ti) {
+          const int slot = ti & 1;
+          if (!mbar_wait(&bar->tempty, (ti & 1u) ^ 1u, abort_flag, err, p.timeout_ns)) break;
+          const uint64_t bdy0 = smem_desc_sw128(dy_win(slot) + kConvPad * 128u, 8192, 1024);
+          for (int t = 0; t < kFbStagesPerTile; ++t, ++q) {
+            const int st = (int)(q % kFbStages);
+            if (!mbar_wait(&bar->afull[st], ring_parity(q, kFbStages), abort_flag, err, p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t at = tmem_base + kFbACol + (uint32_t)st * kTmemAStageCols;
+            if (t < 9) {
+              const uint64_t bd = bw0 + (uint64_t)((uint32_t)t * (8192u >> 4));
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16_ts(tmem_base + kFbDxCol, at + k * 8, bd + (uint64_t)(k * k16), idesc, (t | k) != 0 ? 1u : 0u);
+            } else {
+              const int mt = (t - 9) >> 1, tb = (t - 9) & 1;
+              const uint64_t bd = bdy0 + (uint64_t)((uint32_t)tb * (8192u >> 4));
+              const bool first = ti == 0 && tb == 0;  // the CTA's first block of this M-tile overwrites
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                tc_mma_bf16_ts(tmem_base + (uint32_t)mt * 64u, at + k * 8, bd + (uint64_t)(k * k16), idesc,
+                               (first && k == 0) ? 0u : 1u);
+            }
+            tc_commit(&bar->aempty[st]);
+            if (t == 8) tc_commit(&bar->tfull);
+          }
+          if (ok) tc_commit(&bar->lempty[slot]);  // the dW MMAs have read this slot's dY window
+        }
+      }
+      // every issued MMA (the weight-gradient accumulators in particular) is complete before
+      // the epilogue reads them and before tensor memory is released
+      tc_commit(&bar->dwfull);
+      volatile int never = 0;
+      mbar_wait(&bar->dwfull, 0, &never, err, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    uint32_t ti = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      if (!warp_wait(&bar->tfull, ti & 1u, abort_flag, err, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = tile * kBM + warp * 32 + lane;
+      uint32_t v[2][32];
+      const uint32_t acc = tmem_base + ((uint32_t)(warp * 32) << 16) + kFbDxCol;
+      tmem_ld_32x32b_x32(acc, v[0]);
+      tmem_ld_32x32b_x32(acc + 32, v[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      warp_arrive(&bar->tempty);
+      if (row < M) {
+        uint32_t packed[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int hh = e >> 4, c = (e & 15) * 2;
+          const __nv_bfloat162 h2 =
+              __floats2bfloat162_rn(__uint_as_float(v[hh][c]), __uint_as_float(v[hh][c + 1]));
+          packed[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint4* op = reinterpret_cast<uint4*>(p.dX + (size_t)row * 64);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          op[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+      }
+    }
+    // the CTA's weight-gradient partial: 5 M-tiles x 64 columns, this warp's 32 lanes of each
+    if (ok && warp_wait(&bar->dwfull, 0, abort_flag, err, p.timeout_ns)) {
+      tc_fence_after();
+      float* base = p.partial + (size_t)blockIdx.x * kFbRowsPad * 64;
+#pragma unroll 1
+      for (int mt = 0; mt < kFbMTiles; ++mt) {
+        uint32_t v[2][32];
+        const uint32_t acc = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)mt * 64u;
+        tmem_ld_32x32b_x32(acc, v[0]);
+        tmem_ld_32x32b_x32(acc + 32, v[1]);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(base + (size_t)(mt * kBM + warp * 32 + lane) * 64);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int hh = e >> 3, c = (e & 7) * 4;
+          dst[e] = make_float4(__uint_as_float(v[hh][c]), __uint_as_float(v[hh][c + 1]), __uint_as_float(v[hh][c + 2]),
+                               __uint_as_float(v[hh][c + 3]));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kFbTmemCols);
+  }
+}
+
 // ============================================================================ failure-detection self test
 __global__ void timeout_selftest_kernel(int32_t* status, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -2021,6 +2411,51 @@ cudaError_t launch_tc_conv(const TcConvArgs& a, const void* Wt, int w_rows, int 
   if (bn == 64)
     return a.mirror ? launch_conv_inst<64, true, false>(prm, grid, s) : launch_conv_inst<64, false, false>(prm, grid, s);
   return cudaErrorInvalidValue;
+}
+
+// Single-pass backward at 64 channels: as many CTAs as make every CTA carry the same number
+// of tiles (each CTA's partial covers its tiles; fewer CTAs, fewer partials to reduce).
+int tc_bwd_small_grid(int n) {
+  const int tiles = (n + kBM - 1) / kBM;
+  if (tiles <= 0) return 0;
+  const int sms = sm_count();
+  const int per = (tiles + sms - 1) / sms;
+  return (tiles + per - 1) / per;
+}
+
+size_t tc_bwd_small_partial_floats(int n) { return (size_t)tc_bwd_small_grid(n) * kFbRowsPad * 64; }
+
+cudaError_t launch_tc_bwd_small(const void* dY, const void* X, const int32_t* nbr, int n, const void* Wt, void* dX,
+                                float* partial, float* dW, float* db, cudaStream_t s) {
+  const int grid = tc_bwd_small_grid(n);
+  if (grid == 0) return cudaSuccess;
+  FbParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (!make_rows_tmap(&prm.tmap_dy, dY, (uint64_t)n, 64, (uint32_t)kHaloBox) ||
+      !make_rows_tmap(&prm.tmap_x, X, (uint64_t)n, 64, (uint32_t)kHaloBox))
+    return cudaErrorInvalidValue;
+  {
+    // W [o][j][i]: dims (i, j, o), box (64, 1, 64): tap j as an MN-major W_j^T
+    const uint64_t dims[3] = {64u, 9u, 64u};
+    const uint64_t strides[2] = {64u * 2, 64u * 9 * 2};
+    const uint32_t box[3] = {64u, 1u, 64u};
+    if (!make_tmap(&prm.tmap_w, Wt, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  prm.dY = static_cast<const __nv_bfloat16*>(dY);
+  prm.X = static_cast<const __nv_bfloat16*>(X);
+  prm.nbr = nbr;
+  prm.dX = static_cast<__nv_bfloat16*>(dX);
+  prm.partial = partial;
+  prm.status = device_error_word();
+  prm.timeout_ns = kDefaultTimeoutNs;
+  prm.n = n;
+  const size_t smem = fb_smem_bytes();
+  static int done[64];
+  cudaError_t e = ensure_smem_attr(tc_bwd_small_kernel, smem, done);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(tc_bwd_small_kernel, dim3(grid), dim3(kThreads), smem, s, prm);
+  if (e != cudaSuccess) return e;
+  return launch_wgrad_reduce(partial, grid, kFbRowsPad, 64, 64, 1, dW, db, s);
 }
 
 static int wgrad_bn(int Cout) { return Cout % 256 == 0 ? 256 : Cout % 128 == 0 ? 128 : 64; }

@@ -13,7 +13,7 @@
 //                         flight per warp), keeps an online softmax (running max m, sum l,
 //                         weighted row sum o) per query in registers, and the CTA merges its
 //                         8 warps and writes one partial (m, l, o) per query;
-//   xattn_combine_kernel  one warp per (group, query) merges the group's partials in a fixed
+//   xattn_combine_kernel  one CTA per (group, query) merges the group's partials in a fixed
 //                         order (deterministic) and adds the result to the auxiliary token.
 // Scores are formed in base 2 (the query is prescaled by log2(e) / sqrt(d)), so every
 // exponential is one exp2f.
@@ -201,33 +201,61 @@ __global__ void __launch_bounds__(kXaWarps * 32) xattn_partial_kernel(const __gr
   if (flags && threadIdx.x == 0 && b == 0) atomicOr(p.status, flags);
 }
 
+// Merge of a (group, query)'s partials: one CTA of 8 warps; warp w folds slots w, w + 8, ...
+// (four records in flight per lane) into a running (max, sum, weighted sum), then warp 0
+// merges the 8 warps in order.  The assignment and the order are fixed: deterministic.
+__device__ __forceinline__ void merge_state(float& M, float& L, float (&O)[8], float m, float l, const float (&o)[8]) {
+  if (l == 0.f) return;
+  const float mx = fmaxf(M, m);
+  const float a = exp2f(M - mx), b = exp2f(m - mx);  // M = -inf (nothing yet) gives a = 0
+  L = L * a + l * b;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) O[c] = O[c] * a + o[c] * b;
+  M = mx;
+}
+
 __global__ void __launch_bounds__(256) xattn_combine_kernel(const float* __restrict__ part, int G, int A, int R,
                                                             int slots_per_group, const __nv_bfloat16* __restrict__ aux,
                                                             float* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // (g, a)
+  __shared__ float s_state[kXaWarps][kXaRec][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.x / A, a = blockIdx.x - (blockIdx.x / A) * A;
   pdl_wait();
   pdl_trigger();
-  if (pair >= G * A) return;
-  const int g = pair / A, a = pair - g * A;
-  float M = -INFINITY;
-  for (int s = 0; s < slots_per_group; ++s) {
-    const size_t rec = (((size_t)g * slots_per_group + s) * A + a) * kXaRec * 32 + lane;
-    M = fmaxf(M, part[rec]);
-  }
-  float L = 0.f, O[8];
+  float M = -INFINITY, L = 0.f, O[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) O[c] = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < slots_per_group; ++s) {
-      const size_t rec = (((size_t)g * slots_per_group + s) * A + a) * kXaRec * 32 + lane;
-      const float ls = part[rec + 32];
-      if (ls == 0.f) continue;
-      const float f = exp2f(part[rec] - M);
-      L = fmaf(ls, f, L);
+  const size_t stride = (size_t)A * kXaRec * 32;  // between consecutive slots of the group
+  const float* base = part + (((size_t)g * slots_per_group) * A + a) * kXaRec * 32 + lane;
+  for (int s0 = warp; s0 < slots_per_group; s0 += 4 * kXaWarps) {
+    float m[4], l[4], o[4][8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) O[c] = fmaf(part[rec + (2 + c) * 32], f, O[c]);
+    for (int u = 0; u < 4; ++u) {
+      const int sl = s0 + u * kXaWarps;
+      const bool ok = sl < slots_per_group;
+      const float* r = base + (size_t)(ok ? sl : 0) * stride;
+      m[u] = ok ? r[0] : -INFINITY;
+      l[u] = ok ? r[32] : 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) o[u][c] = ok ? r[(2 + c) * 32] : 0.f;
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) merge_state(M, L, O, m[u], l[u], o[u]);
+  }
+  s_state[warp][0][lane] = M;
+  s_state[warp][1][lane] = L;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) s_state[warp][2 + c][lane] = O[c];
+  __syncthreads();
+  if (warp != 0) return;
+  M = -INFINITY, L = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) O[c] = 0.f;
+  for (int w = 0; w < kXaWarps; ++w) {
+    float o[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] = s_state[w][2 + c][lane];
+    merge_state(M, L, O, s_state[w][0][lane], s_state[w][1][lane], o);
   }
   if (lane * 8 >= R) return;
   float qv[8];
@@ -284,10 +312,9 @@ cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
 
 cudaError_t launch_xattn_combine(const float* part, int G, int A, int R, int slots_per_group, const void* aux,
                                  float* out, cudaStream_t s) {
-  const int pairs = G * A;
-  const int warps = 8;
-  return launch_pdl(xattn_combine_kernel, dim3((pairs + warps - 1) / warps), dim3(warps * 32), 0, s, part, G, A, R,
-                    slots_per_group, static_cast<const __nv_bfloat16*>(aux), out);
+  if (G * A == 0) return cudaSuccess;
+  return launch_pdl(xattn_combine_kernel, dim3(G * A), dim3(kXaWarps * 32), 0, s, part, G, A, R, slots_per_group,
+                    static_cast<const __nv_bfloat16*>(aux), out);
 }
 
 }  // namespace svc
