@@ -87,7 +87,7 @@ extern "C" {
  *              caller zeroes it).  Rows of tokens with bad coordinates are -1.
  *              Frames are validated independently, so when BAD_OFFSETS is set
  *              other bits may be set as well and nbr / M are undefined.
- *   Limits: H*W <= 16384, T >= 0, n >= 0.
+ *   Limits: H*W <= 16384, T >= 0, 0 <= n <= (2^31 - 1) / 9.
  */
 SVCONV_API int svconv_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n,
                        int32_t* nbr, int32_t* M, int32_t* dev_status, void* stream);

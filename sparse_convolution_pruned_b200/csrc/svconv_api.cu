@@ -141,6 +141,7 @@ const char* svconv_status_str(int code) {
 int svconv_build_index(const int32_t* coords, const int32_t* frame_off, int T, int H, int W, int n, int32_t* nbr,
                        int32_t* M, int32_t* dev_status, void* stream) {
   if (T < 0 || n < 0 || H <= 0 || W <= 0 || (long long)H * W > 16384) return SVCONV_ERR_SIZE;
+  if ((long long)n * 9 > 0x7fffffffLL) return SVCONV_ERR_SIZE;  // table entries are indexed with int32
   if (!frame_off || (n > 0 && (!coords || !nbr))) return SVCONV_ERR_NULL;
   int rc = check_device();
   if (rc) return rc;

@@ -24,27 +24,21 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   int32_t* sM = smem;
   int32_t* sCell = smem + HW;
   __shared__ int s_flags;
-  __shared__ int s_lo, s_hi;
   const int t = blockIdx.x;
   pdl_wait();
   pdl_trigger();
-  if (threadIdx.x == 0) {
-    int flags = 0;
-    int lo = frame_off[t], hi = frame_off[t + 1];
-    if (lo < 0 || hi < lo || hi > n) flags |= SVCONV_STATUS_BAD_OFFSETS;
-    if (t == 0 && lo != 0) flags |= SVCONV_STATUS_BAD_OFFSETS;
-    if (t == T - 1 && hi != n) flags |= SVCONV_STATUS_BAD_OFFSETS;
-    if (flags) lo = hi = 0;  // a segment that cannot be trusted is not touched
-    if (hi - lo > HW) {      // more tokens than cells: duplicates; only the first HW are mapped
-      flags |= SVCONV_STATUS_DUPLICATE;
-    }
-    s_flags = flags;
-    s_lo = lo;
-    s_hi = hi;
-  }
+  // every thread reads the frame's bounds itself (a broadcast load), so no extra barrier
+  // round trip is spent handing them out
+  int lo = __ldg(frame_off + t), hi = __ldg(frame_off + t + 1);
+  int flags = 0;
+  if (lo < 0 || hi < lo || hi > n) flags |= SVCONV_STATUS_BAD_OFFSETS;
+  if (t == 0 && lo != 0) flags |= SVCONV_STATUS_BAD_OFFSETS;
+  if (t == T - 1 && hi != n) flags |= SVCONV_STATUS_BAD_OFFSETS;
+  if (flags) lo = hi = 0;  // a segment that cannot be trusted is not touched
+  if (hi - lo > HW) flags |= SVCONV_STATUS_DUPLICATE;  // more tokens than cells: only the first HW are mapped
+  if (threadIdx.x == 0) s_flags = flags;
   for (int c = threadIdx.x; c < HW; c += blockDim.x) sM[c] = -1;
   __syncthreads();
-  const int lo = s_lo, hi = s_hi;
   const int cnt = hi - lo;
 
   // step 1: M[y_k][x_k] = k.  With duplicates the largest k wins (deterministic).
@@ -66,11 +60,11 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
 
   // step 2: the 9 lookups, one (k, j) entry per thread, coalesced writes.
   const int mapped = cnt < HW ? cnt : HW;
-  const long long total = (long long)cnt * 9;
+  const int total = cnt * 9;  // cnt <= n < 2^31 / 9 is checked on the host
   int32_t* out = nbr + (size_t)lo * 9;
-  for (long long e = threadIdx.x; e < total; e += blockDim.x) {
-    const int q = (int)(e / 9);
-    const int j = (int)(e - (long long)q * 9);
+  for (int e = threadIdx.x; e < total; e += blockDim.x) {
+    const int q = e / 9;
+    const int j = e - q * 9;
     int32_t v = -1;
     const int cell = q < mapped ? sCell[q] : -1;
     if (cell >= 0) {

@@ -2207,9 +2207,19 @@ static bool make_tmap(CUtensorMap* m, const void* base, int rank, const uint64_t
     bx[i] = box[i];
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
-  CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  auto encode = [&]() {
+    return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  CUresult r = encode();
+  if (r != CUDA_SUCCESS) {
+    // The encoder needs a current context.  A host thread whose first CUDA work is this call
+    // has none yet (device queries do not bind one): bind the current device's primary
+    // context to the thread and try once more.
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || cudaSetDevice(d) != cudaSuccess) return false;
+    r = encode();
+  }
   return r == CUDA_SUCCESS;
 }
 
