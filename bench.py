@@ -563,6 +563,13 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
     per = ctx.per_kernel(names, max(args.steps, 10))
     if with_bwd:
         per["bwd (fused call)"] = ctx.per_kernel([("bwd", bwd)], max(args.steps, 10))["bwd"]
+    single = with_bwd and dt_name == "bf16" and Cin == 64 and Cout == 64
+    if single:
+        ws1 = torch.empty((max(16, int(sv.lib().svconv_bwd_single_pass_workspace_size(n))),), dtype=torch.uint8,
+                          device=dev)
+        per["bwd (single pass)"] = ctx.per_kernel(
+            [("bwd1", lambda: sv.svconv_bwd_single_pass(dY, X, nbr, Wt, dX=dX, dW=dW, db=db, workspace=ws1))],
+            max(args.steps, 10))["bwd1"]
 
     # end to end through the Python API with pinned host buffers
     h_Y = torch.empty((n, Cout), dtype=odt).pin_memory()
@@ -607,6 +614,10 @@ def conv_leg(ctx, key, with_cpu, clock_window=False):
     if with_bwd:
         kern["bwd (fused call)"] = {"ms": per["bwd (fused call)"],
                                    "note": "svconv_bwd: both gradients in one call, as the step runs them"}
+    if single:
+        kern["bwd (single pass)"] = {"ms": per["bwd (single pass)"],
+                                    "note": "svconv_bwd_single_pass: both gradients from one pass over dY "
+                                            "(one kernel + the split reduce); not the step's schedule"}
     top = max((nm for nm, _ in names), key=lambda k: per[k])
     roof = {k: v for k, v in kern[top].items() if k != "ms"}
     roof["kernel"] = top

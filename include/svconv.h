@@ -168,21 +168,43 @@ SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
  *   db [Cout] fp32 (db may be NULL) are overwritten.
  *   workspace: device, at least svconv_bwd_workspace_size(...) bytes, 16-byte
  *   aligned, no initial contents required.
- *   bf16 with C_in = C_out = 64: ONE pass over dY computes both gradients (each
- *   128-token tile's dY window is loaded once and feeds the mirrored gather of dX and,
- *   in place, the MMAs of dW; the 640 x 64 fp32 dW accumulators stay in tensor memory
- *   for all tiles of a CTA and become that CTA's split partial), then the fixed-order
- *   split reduce.  Deterministic; dW / db use another split plan than
- *   svconv_bwd_weight (same tolerance).  Other shapes and fp32 run svconv_bwd_data and
- *   svconv_bwd_weight in order on `stream`.  The call only enqueues work on `stream`
- *   (no side streams, no host synchronisation), so it can be captured in a CUDA graph
- *   and used from several host threads on different streams.
+ *   bf16 with C_in = C_out = 64: the two gradients run side by side on disjoint
+ *   groups of SMs, the weight gradient on a side stream of the library that is
+ *   forked from and joined back to `stream` with events, so the call stays ordered
+ *   on `stream` and can be captured in a CUDA graph.  Each (device, caller stream)
+ *   pair gets its own side stream and events, created by the first such call on
+ *   that stream OUTSIDE stream capture; a call made while `stream` is being
+ *   captured before it has a side stream (or once 64 caller streams of a device
+ *   have one) runs the same two launches one after the other on `stream` instead,
+ *   with bitwise the same results.  Calls from several host threads on different
+ *   streams, one of them capturing, neither wait on nor enter each other's work.
+ *   dX is bitwise identical to svconv_bwd_data's; dW / db use fewer token splits
+ *   than svconv_bwd_weight (another fixed summation order: deterministic, same
+ *   tolerance).  Other shapes and fp32 run the two calls in order on `stream`.
  *   Errors: as the two calls.
  */
 SVCONV_API int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
                           const void* Wt, void* dX, float* dW, float* db, void* workspace, size_t ws_bytes,
                           void* stream);
 SVCONV_API size_t svconv_bwd_workspace_size(int dtype, int n, int Cin, int Cout);
+
+/*
+ * Both gradients of a bf16 convolution with C_in = C_out = 64 in ONE pass over dY
+ * (SV-TAD page, Key Design 2, the dedicated backward kernels): one kernel loads each
+ * 128-token tile's dY window once and uses it for the mirrored gather of dX and, in
+ * place, as the B operand of the dW MMAs; the 640 x 64 fp32 dW accumulators stay in
+ * tensor memory for every tile of a CTA and become that CTA's split partial; a
+ * fixed-order reduce over the partials gives dW and db.  Deterministic.  It reads dY
+ * and the neighbour table once instead of twice, but on this GPU the side-by-side
+ * schedule of svconv_bwd finishes sooner at the workloads measured, so svconv_bwd
+ * does not use it.
+ *   dY, X [n][64] bf16; Wt [64][9][64] bf16; dX [n][64] bf16; dW [64][9][64] fp32 and
+ *   db [64] fp32 (db may be NULL) overwritten; all device, 16-byte aligned.
+ *   workspace: >= svconv_bwd_single_pass_workspace_size(n) bytes, no initial contents.
+ */
+SVCONV_API int svconv_bwd_single_pass(const void* dY, const void* X, const int32_t* nbr, int n, const void* Wt,
+                                      void* dX, float* dW, float* db, void* workspace, size_t ws_bytes, void* stream);
+SVCONV_API size_t svconv_bwd_single_pass_workspace_size(int n);
 
 /*
  * Chunked bottleneck adapter forward (Key Design 2, "chunked execution" that

@@ -289,7 +289,7 @@ struct AdapterXattn {
   int A, heads;
   float* aux_out;
   float* part;
-  int blocks;    // partial blocks per chunk
+  int blocks;    // partial slots per chunk
   int n_chunks;
 };
 
@@ -420,7 +420,7 @@ int svconv_adapter_fwd(void* X, const int32_t* nbr, const int32_t* frame_off, in
 
 size_t svconv_xattn_workspace_size(int G, int max_group_rows, int A) {
   if (G <= 0 || max_group_rows < 0 || A <= 0) return 0;
-  return xattn_partial_bytes((size_t)G * xattn_blocks(max_group_rows), A);
+  return xattn_partial_bytes((size_t)G * xattn_slots(max_group_rows, G), A);
 }
 
 int svconv_xattn_aux(const void* H, int n, int R, const int32_t* group_off, int G, int max_group_rows,
@@ -449,7 +449,7 @@ int svconv_xattn_aux(const void* H, int n, int R, const int32_t* group_off, int 
   x.A = A;
   x.part = static_cast<float*>(workspace);
   x.slot0 = 0;
-  x.slots_per_group = xattn_blocks(max_group_rows);
+  x.slots_per_group = xattn_slots(max_group_rows, G);
   x.status = dev_status ? dev_status : device_error_word();
   cudaError_t e = launch_xattn_partials(x, s);
   if (e != cudaSuccess) return SVCONV_ERR_CUDA;
@@ -460,7 +460,7 @@ size_t svconv_adapter_xattn_workspace_size(int T, int R, int chunk_T, int max_ch
   if (T <= 0 || R <= 0 || chunk_T <= 0 || max_chunk_rows <= 0 || A <= 0) return 0;
   const size_t base = (svconv_adapter_workspace_size(R, max_chunk_rows) + 255) / 256 * 256;
   const int n_chunks = (T + chunk_T - 1) / chunk_T;
-  return base + xattn_partial_bytes((size_t)n_chunks * xattn_blocks(max_chunk_rows), A);
+  return base + xattn_partial_bytes((size_t)n_chunks * xattn_slots(max_chunk_rows, 1), A);
 }
 
 int svconv_adapter_fwd_xattn(void* X, const int32_t* nbr, const int32_t* frame_off, int T, int n, int D, int R,
@@ -484,7 +484,7 @@ int svconv_adapter_fwd_xattn(void* X, const int32_t* nbr, const int32_t* frame_o
   xa.A = A;
   xa.heads = heads;
   xa.aux_out = aux_out;
-  xa.blocks = xattn_blocks(max_chunk_rows);
+  xa.blocks = xattn_slots(max_chunk_rows, 1);
   xa.n_chunks = T > 0 ? (T + chunk_T - 1) / chunk_T : 0;
   const size_t base = (svconv_adapter_workspace_size(R, max_chunk_rows) + 255) / 256 * 256;
   xa.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + base);

@@ -162,7 +162,7 @@ struct XattnLaunch {
 };
 bool xattn_shape_ok(int R, int A, int heads);
 size_t xattn_partial_bytes(int slots, int A);
-int xattn_blocks(int max_rows);
+int xattn_slots(int max_rows, int G);  // partial slots (CTAs) per group
 cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s);
 cudaError_t launch_xattn_combine(const float* part, int G, int A, int R, int slots_per_group, const void* aux,
                                  float* out, cudaStream_t s);

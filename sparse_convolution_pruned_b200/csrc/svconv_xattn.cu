@@ -8,11 +8,12 @@
 // With a handful of queries per video this is not a dense contraction: every key row is read
 // once and used for A dot products and A weighted sums, 2 A flops per byte, far below the
 // tensor-core (and even the CUDA-core) ridge.  So it runs on CUDA cores and is sized for HBM:
-//   xattn_partial_kernel  one CTA per block of 256 consecutive rows of a group; each warp
-//                         streams rows (one 16-byte piece of a row per lane, four rows in
-//                         flight per warp), keeps an online softmax (running max m, sum l,
-//                         weighted row sum o) per query in registers, and the CTA merges its
-//                         8 warps and writes one partial (m, l, o) per query;
+//   xattn_partial_kernel  about one CTA per 512 rows (at most ~4 per SM), each folding every
+//                         gridDim.x-th chunk of ~16 KB of consecutive rows of a group; chunks
+//                         arrive in shared memory by bulk asynchronous copies, three deep;
+//                         each warp keeps an online softmax (running max m, sum l, weighted
+//                         row sum o) per query in registers, and the CTA merges its 8 warps
+//                         and writes one partial (m, l, o) per query;
 //   xattn_combine_kernel  one CTA per (group, query) merges the group's partials in a fixed
 //                         order (deterministic) and adds the result to the auxiliary token.
 // Scores are formed in base 2 (the query is prescaled by log2(e) / sqrt(d)), so every
@@ -28,11 +29,14 @@
 namespace svc {
 namespace {
 
-constexpr int kXaRows = 256;    // rows per partial block (one CTA)
+constexpr int kXaRowsPerCta = 512;  // rows per partial CTA aimed at (at most kXaCtaCap CTAs)
 constexpr int kXaWarps = 8;     // 256 threads
-constexpr int kXaUnroll = 4;    // rows in flight per warp
+constexpr int kXaStages = 3;    // staged chunks per CTA
+constexpr int kXaStageBytes = 16384;  // about one chunk of rows
 constexpr int kXaQB = 4;        // queries per pass held in registers
 constexpr int kXaRec = 10;      // per lane and query: m, l, o[8]
+constexpr int kXaCtaCap = 592;  // partial CTAs (slots) over all groups of one launch
+constexpr int kXaCombineWarps = 32;
 
 struct XattnParams {
   const __nv_bfloat16* H;  // keys / values [h_rows][R]
@@ -41,7 +45,8 @@ struct XattnParams {
   const int32_t* lo;       // group g owns rows lo[g] .. hi[g]-1 (row numbers before h_sub)
   const int32_t* hi;
   const int32_t* h_sub;    // nullptr, or H row = row - *h_sub (rows of a chunk stored from 0)
-  int rows_cap;            // rows covered per group: gridDim.x * kXaRows
+  int rows_cap;            // rows used per group at most (larger groups are flagged and clipped)
+  int chunk_rows;          // rows per staged chunk (a multiple of 32)
   const __nv_bfloat16* aux;  // [G][A][R]
   int A, q0, qb;           // this pass covers queries q0 .. q0+qb-1
   float qscale;            // log2(e) / sqrt(d)
@@ -75,12 +80,75 @@ __device__ __forceinline__ float head_sum(float v, int lanes_per_head) {
   return v;
 }
 
+// Fold one (max, sum, weighted sum) state into another (base-2 exponents).
+__device__ __forceinline__ void merge_state(float& M, float& L, float (&O)[8], float m, float l, const float (&o)[8]) {
+  if (l == 0.f) return;
+  const float mx = fmaxf(M, m);
+  const float a = exp2f(M - mx), b = exp2f(m - mx);  // M = -inf (nothing yet) gives a = 0
+  L = L * a + l * b;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) O[c] = O[c] * a + o[c] * b;
+  M = mx;
+}
+
+// Online-softmax update of one query's state with a batch of U rows (h: this lane's 8
+// channels of each row, s: the rows' base-2 scores, -inf for rows past the end).
+template <int U>
+__device__ __forceinline__ void online_update(float& m, float& l, float (&o)[8], const float (&s)[U],
+                                              const float (&h)[U][8]) {
+  float mx = m;
+#pragma unroll
+  for (int u = 0; u < U; ++u) mx = fmaxf(mx, s[u]);
+  if (mx == -INFINITY) return;  // no valid row in the batch yet
+  const float alpha = exp2f(m - mx);
+  float lsum = l * alpha;
+  float pr[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    pr[u] = exp2f(s[u] - mx);
+    lsum += pr[u];
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float acc = o[c] * alpha;
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc = fmaf(pr[u], h[u][c], acc);
+    o[c] = acc;
+  }
+  m = mx;
+  l = lsum;
+}
+
+// Lane 0 waits (bounded), the verdict is broadcast: control flow stays warp-uniform.
+__device__ __forceinline__ bool xa_warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, err, kDefaultTimeoutNs);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// CTA x of group g folds the chunks x, x + gridDim.x, ... of the group's rows into one state
+// per query and writes it as slot x.  Chunks (chunk_rows consecutive rows, about 16 KB) are
+// brought into shared memory by bulk asynchronous copies, kXaStages deep, so each CTA has
+// tens of KB in flight at a small register cost; warps then read their rows from shared
+// memory (one 16-byte piece per lane, 4 rows per batch: warp w takes rows 32 b + 4 w + u).
 template <int QB>
 __global__ void __launch_bounds__(kXaWarps * 32) xattn_partial_kernel(const __grid_constant__ XattnParams p) {
-  __shared__ float s_state[kXaWarps][QB][kXaRec][32];
+  extern __shared__ __align__(16) uint8_t xa_smem[];
+  __shared__ __align__(8) uint64_t full[kXaStages];
+  __shared__ int abort_flag;
+  constexpr int U = 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = blockIdx.y, b = blockIdx.x;
+  const int g = blockIdx.y;
   const bool active = lane * 8 < p.R;
+  const uint32_t row_bytes = (uint32_t)p.R * 2u;
+  const uint32_t stage_bytes = (uint32_t)p.chunk_rows * row_bytes;
+  int* err = p.status;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kXaStages; ++st) mbar_init(&full[st], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
 
@@ -95,8 +163,22 @@ __global__ void __launch_bounds__(kXaWarps * 32) xattn_partial_kernel(const __gr
     flags |= SVCONV_STATUS_CHUNK_OVERFLOW;
     hi = lo + p.rows_cap;
   }
-  const int r_begin = lo + b * kXaRows;
-  const int r_end = min(hi, r_begin + kXaRows);
+  const int n_chunks = (hi - lo + p.chunk_rows - 1) / p.chunk_rows;
+  const int mine = n_chunks > (int)blockIdx.x ? (n_chunks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const uint8_t* Hbytes = reinterpret_cast<const uint8_t*>(p.H);
+  auto issue = [&](int i) {  // chunk i of this CTA into stage i % kXaStages (thread 0)
+    const int c = (int)blockIdx.x + i * (int)gridDim.x;
+    const int r0 = lo + c * p.chunk_rows;
+    const int cnt = min(p.chunk_rows, hi - r0);
+    const uint32_t bytes = (uint32_t)cnt * row_bytes;
+    uint64_t* bar = &full[i % kXaStages];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_copy_g2s(smem_u32(xa_smem) + (uint32_t)(i % kXaStages) * stage_bytes,
+                  Hbytes + (size_t)(r0 - sub) * row_bytes, bytes, bar);
+  };
+  int issued = 0;
+  if (threadIdx.x == 0)
+    for (; issued < kXaStages && issued < mine; ++issued) issue(issued);
 
   // this lane's 8 channels of each query, prescaled so that scores are in base 2
   float q[QB][8];
@@ -121,103 +203,96 @@ __global__ void __launch_bounds__(kXaWarps * 32) xattn_partial_kernel(const __gr
     for (int c = 0; c < 8; ++c) o[a][c] = 0.f;
   }
 
-  const __nv_bfloat16* Hb = p.H + lane * 8;
-  for (int r0 = r_begin + warp * kXaUnroll; r0 < r_end; r0 += kXaWarps * kXaUnroll) {
-    float h[kXaUnroll][8];
-#pragma unroll
-    for (int u = 0; u < kXaUnroll; ++u) {
-      const int r = r0 + u;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (active && r < r_end) v = ldg_nc_16(Hb + (size_t)(r - sub) * p.R);
-      unpack8(v, h[u]);
+  bool aborted = false;
+  for (int i = 0; i < mine; ++i) {
+    const int st = i % kXaStages;
+    // every thread takes the same branch: a warp that passes its wait after another warp gave up
+    // must not run ahead into a barrier the others never reach
+    const bool ok = xa_warp_wait(&full[st], (uint32_t)((i / kXaStages) & 1), &abort_flag, err);
+    if (!__syncthreads_and(ok ? 1 : 0)) {
+      aborted = true;
+      break;
     }
+    const int r0 = lo + ((int)blockIdx.x + i * (int)gridDim.x) * p.chunk_rows;
+    const int cnt = min(p.chunk_rows, hi - r0);
+    const uint32_t base = smem_u32(xa_smem) + (uint32_t)st * stage_bytes + (uint32_t)lane * 16u;
+    for (int b = 0; b < cnt; b += kXaWarps * U) {
+      float h[U][8], sc_valid[U];
 #pragma unroll
-    for (int a = 0; a < QB; ++a) {
-      float s[kXaUnroll];
-      float mx = m[a];
-#pragma unroll
-      for (int u = 0; u < kXaUnroll; ++u) {
-        float d = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) d = fmaf(q[a][c], h[u][c], d);
-        s[u] = head_sum(d, p.lanes_per_head);
-        if (r0 + u >= r_end) s[u] = -INFINITY;  // past the block: weight 0
-        mx = fmaxf(mx, s[u]);
-      }
-      if (mx == -INFINITY) continue;  // no row yet (only possible on a block's empty tail)
-      const float alpha = exp2f(m[a] - mx);
-      float pr[kXaUnroll];
-      float lsum = l[a] * alpha;
-#pragma unroll
-      for (int u = 0; u < kXaUnroll; ++u) {
-        pr[u] = exp2f(s[u] - mx);
-        lsum += pr[u];
+      for (int u = 0; u < U; ++u) {
+        const int r = b + warp * U + u;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (active && r < cnt) v = ld_shared_16(base + (uint32_t)r * row_bytes);
+        unpack8(v, h[u]);
+        sc_valid[u] = r < cnt ? 0.f : -INFINITY;
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float acc = o[a][c] * alpha;
+      for (int a = 0; a < QB; ++a) {
+        float sc[U];
 #pragma unroll
-        for (int u = 0; u < kXaUnroll; ++u) acc = fmaf(pr[u], h[u][c], acc);
-        o[a][c] = acc;
+        for (int u = 0; u < U; ++u) {
+          float d = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) d = fmaf(q[a][c], h[u][c], d);
+          sc[u] = head_sum(d, p.lanes_per_head) + sc_valid[u];  // rows past the chunk: weight 0
+        }
+        online_update<U>(m[a], l[a], o[a], sc, h);
       }
-      m[a] = mx;
-      l[a] = lsum;
     }
+    __syncthreads();  // every warp is done with stage st
+    if (threadIdx.x == 0 && issued < mine) issue(issued++);
+  }
+  if (aborted) {
+    // after a wait ran out: let the copies still in flight land before the CTA exits
+    if (threadIdx.x == 0) {
+      volatile int never = 0;
+      for (int i = 0; i < issued; ++i) mbar_wait(&full[i % kXaStages], (uint32_t)((i / kXaStages) & 1), &never, err,
+                                                 kDefaultTimeoutNs);
+    }
+    __syncthreads();
+    return;
   }
 
+  // merge the warps in a fixed order through the (now idle) staging buffer
+  float* st_state = reinterpret_cast<float*>(xa_smem);  // [warp][QB][kXaRec][32]
 #pragma unroll
   for (int a = 0; a < QB; ++a) {
-    s_state[warp][a][0][lane] = m[a];
-    s_state[warp][a][1][lane] = l[a];
+    float* w0 = st_state + ((warp * QB + a) * kXaRec) * 32 + lane;
+    w0[0] = m[a];
+    w0[32] = l[a];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) s_state[warp][a][2 + c][lane] = o[a][c];
+    for (int c = 0; c < 8; ++c) w0[(2 + c) * 32] = o[a][c];
   }
   __syncthreads();
-  // merge the warps in a fixed order: thread (a, lane) of the first QB warps
   if (warp < QB && warp < p.qb) {
     const int a = warp;
-    float M = -INFINITY;
-    for (int w = 0; w < kXaWarps; ++w) M = fmaxf(M, s_state[w][a][0][lane]);
-    float L = 0.f, O[8];
+    float M = -INFINITY, L = 0.f, O[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) O[c] = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < kXaWarps; ++w) {
-        const float lw = s_state[w][a][1][lane];
-        if (lw == 0.f) continue;
-        const float f = exp2f(s_state[w][a][0][lane] - M);
-        L = fmaf(lw, f, L);
+    for (int w = 0; w < kXaWarps; ++w) {
+      const float* r = st_state + ((w * QB + a) * kXaRec) * 32 + lane;
+      float ow[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) O[c] = fmaf(s_state[w][a][2 + c][lane], f, O[c]);
-      }
+      for (int c = 0; c < 8; ++c) ow[c] = r[(2 + c) * 32];
+      merge_state(M, L, O, r[0], r[32], ow);
     }
-    const size_t slot = (size_t)g * p.slots_per_group + p.slot0 + b;
+    const size_t slot = (size_t)g * p.slots_per_group + p.slot0 + blockIdx.x;
     float* dst = p.part + ((slot * p.A + p.q0 + a) * kXaRec) * 32 + lane;
     dst[0] = M;
     dst[32] = L;
 #pragma unroll
     for (int c = 0; c < 8; ++c) dst[(2 + c) * 32] = O[c];
   }
-  if (flags && threadIdx.x == 0 && b == 0) atomicOr(p.status, flags);
+  if (flags && threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.status, flags);
 }
 
-// Merge of a (group, query)'s partials: one CTA of 8 warps; warp w folds slots w, w + 8, ...
+// Merge of a (group, query)'s partials: one CTA of 32 warps; warp w folds slots w, w + 32, ...
 // (four records in flight per lane) into a running (max, sum, weighted sum), then warp 0
-// merges the 8 warps in order.  The assignment and the order are fixed: deterministic.
-__device__ __forceinline__ void merge_state(float& M, float& L, float (&O)[8], float m, float l, const float (&o)[8]) {
-  if (l == 0.f) return;
-  const float mx = fmaxf(M, m);
-  const float a = exp2f(M - mx), b = exp2f(m - mx);  // M = -inf (nothing yet) gives a = 0
-  L = L * a + l * b;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) O[c] = O[c] * a + o[c] * b;
-  M = mx;
-}
-
-__global__ void __launch_bounds__(256) xattn_combine_kernel(const float* __restrict__ part, int G, int A, int R,
-                                                            int slots_per_group, const __nv_bfloat16* __restrict__ aux,
-                                                            float* __restrict__ out) {
-  __shared__ float s_state[kXaWarps][kXaRec][32];
+// merges the 32 warps in order.  The assignment and the order are fixed: deterministic.
+__global__ void __launch_bounds__(kXaCombineWarps * 32) xattn_combine_kernel(
+    const float* __restrict__ part, int G, int A, int R, int slots_per_group, const __nv_bfloat16* __restrict__ aux,
+    float* __restrict__ out) {
+  __shared__ float s_state[kXaCombineWarps][kXaRec][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = blockIdx.x / A, a = blockIdx.x - (blockIdx.x / A) * A;
   pdl_wait();
@@ -227,11 +302,11 @@ __global__ void __launch_bounds__(256) xattn_combine_kernel(const float* __restr
   for (int c = 0; c < 8; ++c) O[c] = 0.f;
   const size_t stride = (size_t)A * kXaRec * 32;  // between consecutive slots of the group
   const float* base = part + (((size_t)g * slots_per_group) * A + a) * kXaRec * 32 + lane;
-  for (int s0 = warp; s0 < slots_per_group; s0 += 4 * kXaWarps) {
+  for (int s0 = warp; s0 < slots_per_group; s0 += 4 * kXaCombineWarps) {
     float m[4], l[4], o[4][8];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int sl = s0 + u * kXaWarps;
+      const int sl = s0 + u * kXaCombineWarps;
       const bool ok = sl < slots_per_group;
       const float* r = base + (size_t)(ok ? sl : 0) * stride;
       m[u] = ok ? r[0] : -INFINITY;
@@ -251,7 +326,7 @@ __global__ void __launch_bounds__(256) xattn_combine_kernel(const float* __restr
   M = -INFINITY, L = 0.f;
 #pragma unroll
   for (int c = 0; c < 8; ++c) O[c] = 0.f;
-  for (int w = 0; w < kXaWarps; ++w) {
+  for (int w = 0; w < kXaCombineWarps; ++w) {
     float o[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) o[c] = s_state[w][2 + c][lane];
@@ -276,7 +351,14 @@ bool xattn_shape_ok(int R, int A, int heads) {
 
 size_t xattn_partial_bytes(int slots, int A) { return (size_t)slots * A * kXaRec * 32 * sizeof(float); }
 
-int xattn_blocks(int max_rows) { return max_rows <= 0 ? 1 : (max_rows + kXaRows - 1) / kXaRows; }
+// CTAs (= partial slots) per group: one per 512 rows of the largest group, at most kXaCtaCap
+// over all groups (about four per SM), so a long group is folded by few CTAs and leaves few
+// partials.  A fixed number, so the workspace size needs no device query.
+int xattn_slots(int max_rows, int G) {
+  const int cap = G > 0 && kXaCtaCap / G > 0 ? kXaCtaCap / G : 1;
+  const int b = max_rows <= 0 ? 1 : (max_rows + kXaRowsPerCta - 1) / kXaRowsPerCta;
+  return b < cap ? b : cap;
+}
 
 cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
   XattnParams p{};
@@ -287,8 +369,13 @@ cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
   p.lo = x.lo;
   p.hi = x.hi;
   p.h_sub = x.h_sub;
-  const int blocks = xattn_blocks(x.max_rows);
-  p.rows_cap = blocks * kXaRows;
+  p.rows_cap = x.max_rows > 0 ? x.max_rows : 0;
+  const int fit = kXaStageBytes / (x.R * 2) / 32 * 32;
+  p.chunk_rows = fit > 32 ? fit : 32;
+  const int slots = xattn_slots(x.max_rows, x.G);
+  size_t smem = (size_t)kXaStages * p.chunk_rows * x.R * 2;
+  const size_t state = (size_t)kXaWarps * kXaQB * kXaRec * 32 * sizeof(float);
+  if (smem < state) smem = state;
   p.aux = static_cast<const __nv_bfloat16*>(x.aux);
   p.A = x.A;
   p.qscale = (float)(1.4426950408889634 / std::sqrt((double)(x.R / x.heads)));
@@ -300,11 +387,11 @@ cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
     p.q0 = q0;
     p.qb = x.A - q0 < kXaQB ? x.A - q0 : kXaQB;
     cudaError_t e;
-    const dim3 grid(blocks, x.G);
+    const dim3 grid(slots, x.G);
     if (p.qb == 1)
-      e = launch_pdl(xattn_partial_kernel<1>, grid, dim3(kXaWarps * 32), 0, s, p);
+      e = launch_pdl(xattn_partial_kernel<1>, grid, dim3(kXaWarps * 32), smem, s, p);
     else
-      e = launch_pdl(xattn_partial_kernel<kXaQB>, grid, dim3(kXaWarps * 32), 0, s, p);
+      e = launch_pdl(xattn_partial_kernel<kXaQB>, grid, dim3(kXaWarps * 32), smem, s, p);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -313,8 +400,8 @@ cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
 cudaError_t launch_xattn_combine(const float* part, int G, int A, int R, int slots_per_group, const void* aux,
                                  float* out, cudaStream_t s) {
   if (G * A == 0) return cudaSuccess;
-  return launch_pdl(xattn_combine_kernel, dim3(G * A), dim3(kXaWarps * 32), 0, s, part, G, A, R, slots_per_group,
-                    static_cast<const __nv_bfloat16*>(aux), out);
+  return launch_pdl(xattn_combine_kernel, dim3(G * A), dim3(kXaCombineWarps * 32), 0, s, part, G, A, R,
+                    slots_per_group, static_cast<const __nv_bfloat16*>(aux), out);
 }
 
 }  // namespace svc

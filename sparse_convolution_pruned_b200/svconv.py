@@ -50,6 +50,10 @@ def lib() -> ctypes.CDLL:
         L.svconv_bwd_weight.argtypes = [I, P, P, P, I, I, I, P, P, P, Z, P]
         L.svconv_bwd.argtypes = [I, P, P, P, I, I, I, P, P, P, P, P, Z, P]
         L.svconv_bwd.restype = I
+        L.svconv_bwd_single_pass.argtypes = [P, P, P, I, P, P, P, P, P, Z, P]
+        L.svconv_bwd_single_pass.restype = I
+        L.svconv_bwd_single_pass_workspace_size.argtypes = [I]
+        L.svconv_bwd_single_pass_workspace_size.restype = Z
         L.svconv_bwd_workspace_size.argtypes = [I, I, I, I]
         L.svconv_bwd_workspace_size.restype = Z
         L.svconv_bwd_weight_noalloc.argtypes = [I, P, P, P, I, I, I, P, P, P]
@@ -250,6 +254,29 @@ def svconv_bwd(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tensor, Wt: torch.T
     rc = lib().svconv_bwd(dt, _ptr(dY), _ptr(X), _ptr(nbr), n, Cin, Cout, _ptr(Wt), _ptr(dX), _ptr(dW), _ptr(db),
                           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(X, stream))
     _check("svconv_bwd", rc)
+    return dX, dW, db
+
+
+def svconv_bwd_single_pass(dY: torch.Tensor, X: torch.Tensor, nbr: torch.Tensor, Wt: torch.Tensor, *,
+                           dX: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+                           db: Optional[torch.Tensor] = None, want_db: bool = True,
+                           workspace: Optional[torch.Tensor] = None, stream=None):
+    """(dX, dW, db) at C_in = C_out = 64 (bf16) from one pass over dY."""
+    _cuda(dY, X, nbr, Wt, dX, dW, db, workspace)
+    n = dY.shape[0]
+    if dX is None:
+        dX = torch.empty((n, 64), dtype=dY.dtype, device=dY.device)
+    if dW is None:
+        dW = torch.empty((64, 9, 64), dtype=torch.float32, device=X.device)
+    if db is None and want_db:
+        db = torch.empty((64,), dtype=torch.float32, device=X.device)
+    need = int(lib().svconv_bwd_single_pass_workspace_size(int(n)))
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=X.device)
+    rc = lib().svconv_bwd_single_pass(_ptr(dY), _ptr(X), _ptr(nbr), n, _ptr(Wt), _ptr(dX), _ptr(dW), _ptr(db),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(X, stream))
+    _check("svconv_bwd_single_pass", rc)
     return dX, dW, db
 
 

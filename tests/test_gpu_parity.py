@@ -441,3 +441,34 @@ def test_e4m3_rejects_unsupported_channels(sv):
     with pytest.raises(sv.SvconvError) as e:
         sv.svconv_fwd(X, nbr, Wt)  # C_in = 64 is not a multiple of 128
     assert e.value.code == -3
+
+
+# ------------------------------------------------------------------ single pass over dY (64 channels)
+SINGLE_PASS_CASES = [
+    ("small_c_config", lambda: wl.small_c_bf16()),
+    ("tiny_and_empty_frames", lambda: wl.custom_conv(seed=43, T=5, H=4, W=4, keep_frac=[0.0, 1 / 16, 0.0, 1.0, 0.5],
+                                                     Cin=64, Cout=64, dtype="bf16")),
+    ("shuffled_ragged", lambda: wl.custom_conv(seed=44, T=9, H=11, W=13, keep_frac=0.6, Cin=64, Cout=64, dtype="bf16",
+                                               shuffle=True, empty_frames=(4,))),
+    # W + 1 = 81 packed rows: neighbours outside the staged windows are read from global memory
+    ("wide_grid_5x80", lambda: wl.custom_conv(seed=45, T=6, H=5, W=80, keep_frac=0.6, Cin=64, Cout=64, dtype="bf16")),
+]
+
+
+@pytest.mark.parametrize("name,make", SINGLE_PASS_CASES, ids=[c[0] for c in SINGLE_PASS_CASES])
+def test_bwd_single_pass(sv, orc, name, make):
+    w = make()
+    nbr, _, st = gpu_index(sv, w, want_map=False)
+    assert st == 0
+    ref_n, _, _ = orc.build_index(w.coords, w.frame_off, w.T, w.H, w.W, want_map=False)
+    X, Wt, dY = dev(w.X, torch.bfloat16), dev(w.Wt, torch.bfloat16), dev(w.dY, torch.bfloat16)
+    dX, dW, db = sv.svconv_bwd_single_pass(dY, X, nbr, Wt)
+    dX2, dW2, db2 = sv.svconv_bwd_single_pass(dY, X, nbr, Wt)
+    torch.cuda.synchronize()
+    assert torch.equal(dX, dX2) and torch.equal(dW, dW2) and torch.equal(db, db2)  # deterministic
+    assert torch.equal(dX, sv.svconv_bwd_data(dY, nbr, Wt))  # same products, same order per output
+    check_bf16(dX.float().cpu().numpy(), orc.bwd_data(w.dY, ref_n, w.Wt), "dX")
+    rdW, rdb = orc.bwd_weight(w.dY, w.X, ref_n)
+    check_bf16(dW.cpu().numpy(), rdW, "dW")
+    check_bf16(db.cpu().numpy(), rdb, "db")
+    assert sv.svconv_read_error_word() == 0
