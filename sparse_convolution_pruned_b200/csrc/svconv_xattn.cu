@@ -388,10 +388,15 @@ cudaError_t launch_xattn_partials(const XattnLaunch& x, cudaStream_t s) {
     p.qb = x.A - q0 < kXaQB ? x.A - q0 : kXaQB;
     cudaError_t e;
     const dim3 grid(slots, x.G);
-    if (p.qb == 1)
-      e = launch_pdl(xattn_partial_kernel<1>, grid, dim3(kXaWarps * 32), smem, s, p);
-    else
-      e = launch_pdl(xattn_partial_kernel<kXaQB>, grid, dim3(kXaWarps * 32), smem, s, p);
+    // the staged chunks plus the kernel's static barriers exceed the default 48 KB limit
+    static int done1[64], done4[64];
+    if (p.qb == 1) {
+      e = ensure_smem_attr(xattn_partial_kernel<1>, smem, done1);
+      if (e == cudaSuccess) e = launch_pdl(xattn_partial_kernel<1>, grid, dim3(kXaWarps * 32), smem, s, p);
+    } else {
+      e = ensure_smem_attr(xattn_partial_kernel<kXaQB>, smem, done4);
+      if (e == cudaSuccess) e = launch_pdl(xattn_partial_kernel<kXaQB>, grid, dim3(kXaWarps * 32), smem, s, p);
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
