@@ -8,7 +8,7 @@
 // With a handful of queries per video this is not a dense contraction: every key row is read
 // once and used for A dot products and A weighted sums, 2 A flops per byte, far below the
 // tensor-core (and even the CUDA-core) ridge.  So it runs on CUDA cores and is sized for HBM:
-//   xattn_partial_kernel  about one CTA per 512 rows (at most ~4 per SM), each folding every
+//   xattn_partial_kernel  one wave of CTAs (3 per SM, >= 128 rows each), each folding every
 //                         gridDim.x-th chunk of ~16 KB of consecutive rows of a group; chunks
 //                         arrive in shared memory by bulk asynchronous copies, three deep;
 //                         each warp keeps an online softmax (running max m, sum l, weighted
@@ -29,13 +29,13 @@
 namespace svc {
 namespace {
 
-constexpr int kXaRowsPerCta = 512;  // rows per partial CTA aimed at (at most kXaCtaCap CTAs)
+constexpr int kXaRowsPerCta = 128;  // fewest rows per partial CTA (at most kXaCtaCap CTAs)
 constexpr int kXaWarps = 8;     // 256 threads
 constexpr int kXaStages = 3;    // staged chunks per CTA
 constexpr int kXaStageBytes = 16384;  // about one chunk of rows
 constexpr int kXaQB = 4;        // queries per pass held in registers
 constexpr int kXaRec = 10;      // per lane and query: m, l, o[8]
-constexpr int kXaCtaCap = 592;  // partial CTAs (slots) over all groups of one launch
+constexpr int kXaCtaCap = 444;  // partial CTAs (slots) over all groups: one wave of 3 per SM on 148 SMs
 constexpr int kXaCombineWarps = 32;
 
 struct XattnParams {
@@ -351,9 +351,10 @@ bool xattn_shape_ok(int R, int A, int heads) {
 
 size_t xattn_partial_bytes(int slots, int A) { return (size_t)slots * A * kXaRec * 32 * sizeof(float); }
 
-// CTAs (= partial slots) per group: one per 512 rows of the largest group, at most kXaCtaCap
-// over all groups (about four per SM), so a long group is folded by few CTAs and leaves few
-// partials.  A fixed number, so the workspace size needs no device query.
+// CTAs (= partial slots) per group: enough to fill the GPU once (each CTA keeps only its own
+// three chunks in flight, so the bytes in flight scale with the CTAs), at most kXaCtaCap over
+// all groups and at least 128 rows each.  A fixed number, so the workspace size needs no
+// device query.
 int xattn_slots(int max_rows, int G) {
   const int cap = G > 0 && kXaCtaCap / G > 0 ? kXaCtaCap / G : 1;
   const int b = max_rows <= 0 ? 1 : (max_rows + kXaRowsPerCta - 1) / kXaRowsPerCta;

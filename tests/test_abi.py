@@ -54,11 +54,11 @@ def test_host_validation_runs_before_any_device_call(L):
     # fp32: one split per 16 tokens (at most 128), each split 9 C_in + 1 rows of C_out floats
     assert sv.svconv_bwd_weight_workspace_size(sv.F32, 128, 16, 16) == 8 * (9 * 16 + 1) * 16 * 4
     assert sv.svconv_bwd_weight_workspace_size(sv.F32, 100000, 16, 16) == 128 * (9 * 16 + 1) * 16 * 4
-    # the cross-attention partials: one slot per 512 rows of the largest group (at most 592 over
+    # the cross-attention partials: one slot per 128 rows of the largest group (at most 444 over
     # all groups), A records of 10 x 32 floats per slot
-    assert sv.svconv_xattn_workspace_size(3, 600, 2) == 3 * 2 * 2 * 10 * 32 * 4
-    assert sv.svconv_xattn_workspace_size(1, 282624, 1) == 552 * 10 * 32 * 4
-    assert sv.svconv_xattn_workspace_size(4, 10 ** 7, 1) == 4 * 148 * 10 * 32 * 4
+    assert sv.svconv_xattn_workspace_size(3, 600, 2) == 3 * 5 * 2 * 10 * 32 * 4
+    assert sv.svconv_xattn_workspace_size(1, 282624, 1) == 444 * 10 * 32 * 4
+    assert sv.svconv_xattn_workspace_size(4, 10 ** 7, 1) == 4 * 111 * 10 * 32 * 4
     # e4m3 forward: channel counts are checked before any device call
     assert L.svconv_fwd(sv.E4M3, fake, fake, 10, 64, 256, fake, None, fake, None) == -3
     assert sv.svconv_bwd_weight_workspace_size(sv.F32, 0, 16, 16) == 0
