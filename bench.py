@@ -1021,7 +1021,11 @@ def run_b200(args):
     with_cpu = world == 1 and not args.no_cpu_baseline
 
     # the headline workload first: its timed steps and sustained replays carry the clock record
-    head = run_leg(ctx, head_key, with_cpu, clock_window=True)
+    if head_key == "xattn":  # the cross-attention leg alone (profiling runs)
+        head = xattn_leg(ctx, with_cpu)
+        head.update(dtype="bf16", n_kept_per_gpu=None, step_roofline=None)
+    else:
+        head = run_leg(ctx, head_key, with_cpu, clock_window=True)
     configs = {head_key: head}
     if world == 1 and not args.workload:
         for key in ORDER:
@@ -1040,9 +1044,10 @@ def run_b200(args):
             "config": {"workload": head["workload"], "n_kept_per_gpu": head["n_kept_per_gpu"],
                        "step": head["step"], "l2": head["l2"], "graph": "step replayed from a CUDA graph",
                        "parallelism": f"dp{world}",
-                       "why_headline": "largest fwd+bwd configuration that fits one GPU"},
+                       "why_headline": ("largest fwd+bwd configuration that fits one GPU" if not args.workload
+                                        else "the workload asked for with --workload")},
             "roofline": head["roofline"],
-            "step_roofline": head["step_roofline"],
+            "step_roofline": head.get("step_roofline"),
             "kernels": head["kernels"],
             "e2e": head["e2e"],
             "gpu_launches": head["gpu_launches_per_step"] * args.steps,
@@ -1079,7 +1084,7 @@ def main():
                          "(1024: 3 chunks, ~660 MiB peak; 512: 6 chunks, ~610 MiB)")
     ap.add_argument("--no-crossover", action="store_true",
                     help="skip the keep-rate sweep against the dense-reconstruction baseline")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["xattn"], default=None,
                     help="time only this workload (as the top-level line); default: the headline "
                          f"({HEADLINE}) plus every other workload under 'configs'")
     args = ap.parse_args()
