@@ -76,8 +76,8 @@ extern "C" {
 /*
  * Neighbour-index build (Key Design 1: the lookup map M per frame, filled with -1,
  * then M[y_k, x_k] = k; then N[k, j] = M[y_k+dy_j, x_k+dx_j], or -1 when the
- * neighbour was pruned or is out of bounds).  One CTA per frame keeps M in shared
- * memory; nothing returns to the host.
+ * neighbour was pruned or is out of bounds).  Each CTA keeps the maps of a few
+ * consecutive frames in shared memory; nothing returns to the host.
  *   coords     [n][3] int32 device, frame_off [T+1] int32 device.
  *   nbr        [n][9] int32 device, written.
  *   M          [T][H][W] int32 device or NULL; if given, written with the map

@@ -69,6 +69,9 @@ INDEX_CASES = [
     ("max_grid_128x128", lambda: wl.custom_conv(seed=8, T=2, H=128, W=128, keep_frac=0.3, Cin=4, Cout=4,
                                                 dtype="f32", shuffle=True)),
     ("single_row_1x40", lambda: wl.custom_conv(seed=9, T=4, H=1, W=40, keep_frac=0.5, Cin=4, Cout=4, dtype="f32")),
+    # thousands of frames: several frames per CTA, empty frames among them, shuffled tokens
+    ("many_frames_5x6", lambda: wl.custom_conv(seed=10, T=6000, H=5, W=6, keep_frac=0.5, Cin=4, Cout=4,
+                                               dtype="f32", shuffle=True, empty_frames=tuple(range(0, 6000, 7)))),
 ]
 
 
@@ -95,6 +98,37 @@ def test_index_adapter_size_and_empty(sv, orc):
     off = torch.zeros(5, dtype=torch.int32, device="cuda")
     nbr, M = sv.svconv_build_index(coords, off, 4, 3, 3, want_map=True, status=st)
     assert nbr.shape == (0, 9) and bool((M == -1).all()) and st.item() == 0
+
+
+def test_index_error_flags_in_multi_frame_ctas(sv, orc):
+    """Thousands of one-token frames (several frames per CTA); one frame at a time carries a bad
+    coordinate, a wrong frame number or a duplicate: flags equal the oracle's, and every other
+    frame's rows are still exact."""
+    T = 5000
+    coords = np.zeros((2 * T, 3), np.int32)
+    coords[:, 0] = np.repeat(np.arange(T), 2)
+    coords[0::2, 1], coords[0::2, 2] = 0, 0
+    coords[1::2, 1], coords[1::2, 2] = 0, 1
+    off = np.arange(0, 2 * T + 1, 2, dtype=np.int32)
+    for kind in ("coord", "frame", "dup"):
+        c = coords.copy()
+        k = 2 * 2501 + 1
+        if kind == "coord":
+            c[k, 2] = 9
+        elif kind == "frame":
+            c[k, 0] = 2500
+        else:
+            c[k, 1:] = c[k - 1, 1:]
+        ref_n, _, ref_st = orc.build_index(c, off, T, 3, 3, want_map=False)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nbr, _ = sv.svconv_build_index(dev(c), dev(off), T, 3, 3, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == ref_st, (kind, int(st.item()), ref_st)
+        got = nbr.cpu().numpy()
+        ok_rows = np.ones(2 * T, bool)
+        ok_rows[2 * 2500: 2 * 2502] = False  # the frames touched by the bad token
+        np.testing.assert_array_equal(got[ok_rows], ref_n[ok_rows])
+    assert sv.svconv_read_error_word() == 0
 
 
 def test_index_error_flags_match_oracle(sv, orc):
