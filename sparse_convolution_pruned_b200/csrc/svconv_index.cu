@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   const int HW = H * W;
   const int F = frames_per_cta;
   int32_t* sM = smem;               // [F][HW]
-  int32_t* sCell = smem + F * HW;   // [F][HW]
+  int32_t* sCell = smem + F * HW;   // [F][HW]: each token's (y << 16 | x), or -1
   __shared__ int s_lo[kIdxMaxFrames], s_cnt[kIdxMaxFrames], s_pre[kIdxMaxFrames + 1];
   __shared__ int s_flags;
   const int t0 = blockIdx.x * F;
@@ -77,8 +77,8 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
     } else if (y < 0 || y >= H || x < 0 || x >= W) {
       atomicOr(&s_flags, SVCONV_STATUS_BAD_COORD);
     } else {
-      cell = y * W + x;
-      atomicMax(&sM[f * HW + cell], k);
+      atomicMax(&sM[f * HW + y * W + x], k);
+      cell = (y << 16) | x;  // kept as (y, x): the lookups below need no division
     }
     if (q < HW) sCell[f * HW + q] = cell;
   }
@@ -95,11 +95,11 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
     const int q = i - s_pre[f];
     const int lo = s_lo[f];
     int32_t v = -1;
-    const int cell = q < HW ? sCell[f * HW + q] : -1;
-    if (cell >= 0) {
-      const int y = cell / W, x = cell - y * W;
+    const int yx = q < HW ? sCell[f * HW + q] : -1;
+    if (yx >= 0) {
+      const int y = yx >> 16, x = yx & 0xffff;
       const int32_t* Mf = sM + f * HW;
-      if (j == 4 && Mf[cell] != lo + q) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
+      if (j == 4 && Mf[y * W + x] != lo + q) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
       const int yy = y + j / 3 - 1, xx = x + j % 3 - 1;
       if (yy >= 0 && yy < H && xx >= 0 && xx < W) v = Mf[yy * W + xx];
     }
