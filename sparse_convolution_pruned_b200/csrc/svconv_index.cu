@@ -31,7 +31,9 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   int32_t* sM = smem;               // [F][HW]
   int32_t* sCell = smem + F * HW;   // [F][HW]: each token's (y << 16 | x), or -1
   __shared__ int s_lo[kIdxMaxFrames], s_cnt[kIdxMaxFrames], s_pre[kIdxMaxFrames + 1];
-  __shared__ int s_flags;
+  __shared__ int s_flags, s_contig;
+  __shared__ int32_t sStage[8 * 32 * 9];  // per warp: 32 rows of 9 entries
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * F;
   const int nf = min(F, T - t0);
   pdl_wait();
@@ -53,12 +55,14 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   for (int c = threadIdx.x; c < nf * HW; c += blockDim.x) sM[c] = -1;
   __syncthreads();
   if (threadIdx.x == 0) {
-    int acc = 0;
+    int acc = 0, contig = 1;
     for (int f = 0; f < nf; ++f) {
       s_pre[f] = acc;
       acc += s_cnt[f];
+      if (f > 0 && s_lo[f] != s_lo[f - 1] + s_cnt[f - 1]) contig = 0;
     }
     s_pre[nf] = acc;
+    s_contig = contig;
   }
   __syncthreads();
   const int total_tok = s_pre[nf];
@@ -84,26 +88,55 @@ __global__ void __launch_bounds__(256) build_index_kernel(const int32_t* __restr
   }
   __syncthreads();
 
-  // step 2: the 9 lookups, one (k, j) entry per thread.  With valid offsets the frames' rows
-  // are consecutive, so consecutive threads write consecutive entries.
-  const int total = total_tok * 9;  // tokens <= n <= (2^31 - 1) / 9 is checked on the host
-  for (int e = threadIdx.x; e < total; e += blockDim.x) {
-    const int i = e / 9;
-    const int j = e - i * 9;
-    int f = 0;
-    while (f + 1 < nf && s_pre[f + 1] <= i) ++f;
-    const int q = i - s_pre[f];
-    const int lo = s_lo[f];
-    int32_t v = -1;
-    const int yx = q < HW ? sCell[f * HW + q] : -1;
-    if (yx >= 0) {
-      const int y = yx >> 16, x = yx & 0xffff;
-      const int32_t* Mf = sM + f * HW;
-      if (j == 4 && Mf[y * W + x] != lo + q) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
-      const int yy = y + j / 3 - 1, xx = x + j % 3 - 1;
-      if (yy >= 0 && yy < H && xx >= 0 && xx < W) v = Mf[yy * W + xx];
+  // step 2: the 9 lookups, one token per thread (the frame search and the unpacking happen
+  // once per token; the taps unroll with constant offsets).  Each warp stages its 32 rows of
+  // 9 entries in shared memory (9 is odd, so the staging is free of bank conflicts) and, when
+  // the CTA's frames are contiguous in the table, writes them back as 9 coalesced stores.
+  int32_t* stage = sStage + warp * 32 * 9;
+  const bool contig = s_contig;
+  const int row0 = s_lo[0];
+  for (int base = warp * 32; base < total_tok; base += (int)blockDim.x) {
+    const int i = base + lane;
+    int32_t v[9];
+    int row = -1;
+    if (i < total_tok) {
+      int f = 0;
+      while (f + 1 < nf && s_pre[f + 1] <= i) ++f;
+      const int q = i - s_pre[f];
+      row = s_lo[f] + q;
+      const int yx = q < HW ? sCell[f * HW + q] : -1;
+      if (yx >= 0) {
+        const int y = yx >> 16, x = yx & 0xffff;
+        const int32_t* Mf = sM + f * HW;
+        if (Mf[y * W + x] != row) atomicOr(&s_flags, SVCONV_STATUS_DUPLICATE);
+#pragma unroll
+        for (int j = 0; j < 9; ++j) {
+          const int yy = y + j / 3 - 1, xx = x + j % 3 - 1;
+          v[j] = (yy >= 0 && yy < H && xx >= 0 && xx < W) ? Mf[yy * W + xx] : -1;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 9; ++j) v[j] = -1;
+      }
     }
-    nbr[(size_t)(lo + q) * 9 + j] = v;
+    if (contig) {
+      if (i < total_tok) {
+#pragma unroll
+        for (int j = 0; j < 9; ++j) stage[lane * 9 + j] = v[j];
+      }
+      __syncwarp();
+      const int cnt = min(32, total_tok - base) * 9;
+      int32_t* dst = nbr + (size_t)(row0 + base) * 9;
+#pragma unroll
+      for (int m = 0; m < 9; ++m) {
+        const int idx = lane + 32 * m;
+        if (idx < cnt) dst[idx] = stage[idx];
+      }
+      __syncwarp();
+    } else if (i < total_tok) {
+#pragma unroll
+      for (int j = 0; j < 9; ++j) nbr[(size_t)row * 9 + j] = v[j];
+    }
   }
   if (Mout) {
     for (int c = threadIdx.x; c < nf * HW; c += blockDim.x) Mout[(size_t)t0 * HW + c] = sM[c];
@@ -124,9 +157,10 @@ cudaError_t launch_build_index(const int32_t* coords, const int32_t* frame_off, 
   int F = (T + waves_ctas - 1) / waves_ctas;
   if (F < 1) F = 1;
   if (F > kIdxMaxFrames) F = kIdxMaxFrames;
-  while (F > 1 && (size_t)2 * sizeof(int32_t) * HW * F > 48 * 1024) --F;
+  while (F > 1 && (size_t)2 * sizeof(int32_t) * HW * F > 32 * 1024) --F;
   const size_t smem = 2 * sizeof(int32_t) * (size_t)HW * F;
-  if (smem > 48 * 1024) {
+  // beyond 48 KB of static (~10 KB) plus dynamic shared memory the kernel must opt in
+  if (smem > 36 * 1024) {
     static int done[64];
     cudaError_t e = ensure_smem_attr(build_index_kernel, smem, done);
     if (e != cudaSuccess) return e;
