@@ -78,8 +78,8 @@ constexpr int kConvHaloRows = kBM + 2 * kConvPad;  // conv halo window (A rows m
 constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
 constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
 __host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: index + halo slots in flight
-  return bn == 256 ? 4 : 8;                                // (covers ~2 us of load latency at small C)
-}
+  return bn == 256 ? 5 : 8;  // (covers ~2 us of load latency at small C; at 256 columns three builder
+}                            //  groups hold three slots and the loader runs ahead by two)
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
@@ -1490,6 +1490,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
   constexpr int kSlots = wgrad_slots(BN);
+  // Builder groups of four warps.  At 256 columns a CTA usually carries one unit, so its four
+  // epilogue warps would idle until the very end: they build A stages as a third group.
+  constexpr int kGroups = BN == 256 ? 3 : 2;
 
   const int m_tiles = p.rows_pad / kBM;
   const int n_tiles = p.Cout / BN;
@@ -1524,6 +1527,94 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     n0 = nt * BN;
     kb0 = (int)((long long)kbt * sp / p.splits);
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
+  };
+
+  // Builds the A stages of unit u's token blocks whose running index q satisfies
+  // q % kGroups == grp (q counts every block of the CTA, so the groups stay in step); false
+  // when a wait gave up.
+  auto build_unit = [&](int u, uint32_t& q, int grp) -> bool {
+    const int quarter = warp & 3;
+    const int half = quarter >> 1;
+    const int cq = (quarter & 1) * 32;
+    const uint32_t zero_addr = smem_u32(bar->zero16);
+    const uint16_t* X16 = reinterpret_cast<const uint16_t*>(p.X);
+    int sp, mt, n0, kb0, kb1;
+    decode(u, sp, mt, n0, kb0, kb1);
+    const int cb = mt / kWgTiles;
+    const int j = 2 * (mt % kWgTiles) + half;        // tap of this warp's half (9: the extra half)
+    const int kind = j < 9 ? 0 : (cb == 0 ? 1 : 2);  // gathered X, ones row, padding
+    for (int kb = kb0; kb < kb1; ++kb, ++q) {
+      if ((int)(q % (uint32_t)kGroups) != grp) continue;
+      const int slot = (int)(q % kSlots);
+      const int sa = (int)(q % kTmemAStages);
+      if (!warp_wait(&bar->ifull[slot], ring_parity(q, kSlots), abort_flag, err, p.timeout_ns) ||
+          !warp_wait(&bar->aempty[sa], ring_parity(q, kTmemAStages) ^ 1u, abort_flag, err, p.timeout_ns))
+        return false;
+      tc_fence_after();  // the MMAs that read this A stage are complete
+      const int k0 = kb * kBK;
+      const uint32_t a_col = tmem_base + kACol + (uint32_t)sa * kTmemAStageCols;
+      if (kind == 0) {
+        const uint32_t sidx_s = smem_u32(sm.idx + slot * kWgIdx);
+        const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
+        const int hlo = k0 - kWgPad;
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
+          uint32_t R[16];
+          bool far = false, bad = false;
+          const int chunk = (c16 >> 3) + (mi & 1);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            // branch-free: entries of tokens past n (stale slot contents) count as missing
+            const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
+            const int raw = ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j));
+            const bool tok_ok = k0 + tk < p.n;
+            bad |= tok_ok & (raw >= p.n);
+            const int x = (tok_ok & (raw < p.n)) ? raw : -1;
+            const int h = x - hlo;
+            const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kWgHaloRows);
+            far |= (x >= 0) & !in_win;
+            const uint32_t addr =
+                in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_addr;
+            ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
+          }
+          if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+          if (__any_sync(0xffffffffu, far)) {
+            // entries outside the halo window read as zero above: fetch them from global memory
+            Regs16 rr;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) rr.v[r] = R[r];
+            rr = wgrad_patch_far(rr, sidx_s, X16, p.n, p.Cin, k0, hlo, j, cb * kBK + c16);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) R[r] = rr.v[r];
+          }
+          tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+        }
+      } else if (kind == 1) {
+        // row 0 of the extra half is 1 for every valid token: its accumulator row is db
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          uint32_t R[16];
+#pragma unroll
+          for (int r = 0; r < 16; ++r) R[r] = 0u;
+          if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int tk = k0 + 8 * k + 2 * lane;
+              R[2 * k] = (tk < p.n ? 0x3F80u : 0u) | (tk + 1 < p.n ? 0x3F800000u : 0u);
+            }
+          }
+          tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+        }
+      }
+      // (padding halves are not written: their accumulator rows are never read)
+      tmem_st_wait();
+      tc_fence_before();
+      warp_arrive(&bar->afull[sa]);
+      warp_arrive(&bar->iempty[slot]);
+    }
+    return true;
   };
 
   if (warp == kHaloWarp) {
@@ -1581,100 +1672,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders (tensor memory)
-    // Two groups of four warps take alternate token blocks.  Warp w writes TMEM lanes
+    // Groups of four warps take turns over the token blocks (two groups, plus the epilogue
+    // warps as a third at 256 columns).  Warp w writes TMEM lanes
     // 32 (w % 4) .. + 31: half (w % 4) / 2 of the tile, channels 32 (w % 2) .. + 31 of
     // that half's tap, as two 16-lane pieces of 16 channels x 64 tokens.  For one
     // piece, ldmatrix k4 (k4 = 0..3) covers tokens 16 k4 .. + 15: lane i supplies the
     // halo row of token 16 k4 + 8 (i / 16) + i % 8, channels +8 ((i / 8) % 2); its four
     // registers are then registers 4 k4 .. 4 k4 + 3 of the 16x128b.x8 store.
     const int grp = (warp - kEpiWarps) >> 2;
-    const int quarter = warp & 3;
-    const int half = quarter >> 1;
-    const int cq = (quarter & 1) * 32;
-    const uint32_t zero_addr = smem_u32(bar->zero16);
-    const uint16_t* X16 = reinterpret_cast<const uint16_t*>(p.X);
     uint32_t q = 0;
-    bool aborted = false;
-    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-      int sp, mt, n0, kb0, kb1;
-      decode(u, sp, mt, n0, kb0, kb1);
-      const int cb = mt / kWgTiles;
-      const int j = 2 * (mt % kWgTiles) + half;        // tap of this warp's half (9: the extra half)
-      const int kind = j < 9 ? 0 : (cb == 0 ? 1 : 2);  // gathered X, ones row, padding
-      for (int kb = kb0; kb < kb1; ++kb, ++q) {
-        if ((int)(q & 1u) != grp) continue;
-        const int slot = (int)(q % kSlots);
-        const int sa = (int)(q % kTmemAStages);
-        if (!warp_wait(&bar->ifull[slot], ring_parity(q, kSlots), abort_flag, err, p.timeout_ns) ||
-            !warp_wait(&bar->aempty[sa], ring_parity(q, kTmemAStages) ^ 1u, abort_flag, err, p.timeout_ns)) {
-          aborted = true;
-          break;
-        }
-        tc_fence_after();  // the MMAs that read this A stage are complete
-        const int k0 = kb * kBK;
-        const uint32_t a_col = tmem_base + kACol + (uint32_t)sa * kTmemAStageCols;
-        if (kind == 0) {
-          const uint32_t sidx_s = smem_u32(sm.idx + slot * kWgIdx);
-          const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
-          const int hlo = k0 - kWgPad;
-          const int mi = lane >> 3;
-#pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
-            uint32_t R[16];
-            bool far = false, bad = false;
-            const int chunk = (c16 >> 3) + (mi & 1);
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-              // branch-free: entries of tokens past n (stale slot contents) count as missing
-              const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
-              const int raw = ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j));
-              const bool tok_ok = k0 + tk < p.n;
-              bad |= tok_ok & (raw >= p.n);
-              const int x = (tok_ok & (raw < p.n)) ? raw : -1;
-              const int h = x - hlo;
-              const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kWgHaloRows);
-              far |= (x >= 0) & !in_win;
-              const uint32_t addr =
-                  in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_addr;
-              ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
-            }
-            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-            if (__any_sync(0xffffffffu, far)) {
-              // entries outside the halo window read as zero above: fetch them from global memory
-              Regs16 rr;
-#pragma unroll
-              for (int r = 0; r < 16; ++r) rr.v[r] = R[r];
-              rr = wgrad_patch_far(rr, sidx_s, X16, p.n, p.Cin, k0, hlo, j, cb * kBK + c16);
-#pragma unroll
-              for (int r = 0; r < 16; ++r) R[r] = rr.v[r];
-            }
-            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
-          }
-        } else if (kind == 1) {
-          // row 0 of the extra half is 1 for every valid token: its accumulator row is db
-#pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            uint32_t R[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) R[r] = 0u;
-            if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int tk = k0 + 8 * k + 2 * lane;
-                R[2 * k] = (tk < p.n ? 0x3F80u : 0u) | (tk + 1 < p.n ? 0x3F800000u : 0u);
-              }
-            }
-            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
-          }
-        }
-        // (padding halves are not written: their accumulator rows are never read)
-        tmem_st_wait();
-        tc_fence_before();
-        warp_arrive(&bar->afull[sa]);
-        warp_arrive(&bar->iempty[slot]);
-      }
-    }
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x)
+      if (!build_unit(u, q, grp)) break;
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -1702,7 +1710,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   } else {
     // ------------------------------------------------------------ epilogue: fp32 partial rows
     uint32_t tc = 0;
+    uint32_t qe = 0;  // block counter of the third builder group
     for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+      if constexpr (kGroups == 3) {
+        if (!build_unit(u, qe, 2)) break;
+      }
       int sp, mt, n0, kb0, kb1;
       decode(u, sp, mt, n0, kb0, kb1);
       const uint32_t ab = tc % (uint32_t)kAcc;
@@ -2499,7 +2511,7 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
   prm.stages_a = kTmemAStages;
   prm.stages_b = 2;
   for (int b = 2; b <= kMaxStages; ++b)
-    if (smem_total(wgrad_geometry(BN, b)) <= 220 * 1024) prm.stages_b = b;
+    if (smem_total(wgrad_geometry(BN, b)) <= 226 * 1024) prm.stages_b = b;
   const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_b));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
