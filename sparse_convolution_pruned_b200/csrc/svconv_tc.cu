@@ -83,7 +83,7 @@ __host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: ind
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
-constexpr int kTmemAStages = 4;                    // weight gradient: A stages held in tensor memory
+__host__ __device__ constexpr int wgrad_a_stages(int bn) { return bn == 256 ? 8 : 4; }  // A stages in TMEM
 constexpr int kGatherKb = 2;                       // gather conv: K-blocks (of 64) per pipeline stage
 constexpr int kTmemAStageCols = kBK / 2;           // 64 bf16 per row = 32 TMEM columns
 
@@ -187,7 +187,7 @@ __host__ __device__ inline Geometry wgrad_geometry(int bn, int sb) {
 }
 __host__ __device__ constexpr int wgrad_acc_buffers(int bn) { return bn == 256 ? 1 : 2; }
 __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
-  return pow2_cols((uint32_t)(wgrad_acc_buffers(bn) * bn + kTmemAStages * kTmemAStageCols));
+  return pow2_cols((uint32_t)(wgrad_acc_buffers(bn) * bn + wgrad_a_stages(bn) * kTmemAStageCols));
 }
 
 __host__ __device__ inline size_t smem_total(const Geometry& g) {
@@ -1490,6 +1490,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
   constexpr int kSlots = wgrad_slots(BN);
+  constexpr int kAStages = wgrad_a_stages(BN);
   // Builder groups of four warps.  At 256 columns a CTA usually carries one unit, so its four
   // epilogue warps would idle until the very end: they build A stages as a third group.
   constexpr int kGroups = BN == 256 ? 3 : 2;
@@ -1501,7 +1502,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     // ifull: 32 cp.async arrivals of the loader lanes + its expect_tx arrival
-    init_barriers(bar, kTmemAStages, SB, kProdWarps / 2, kSlots, 33, kProdWarps / 2);
+    init_barriers(bar, kAStages, SB, kProdWarps / 2, kSlots, 33, kProdWarps / 2);
     prefetch_tmap(&p.tmap_x);
     prefetch_tmap(&p.tmap_dy);
   }
@@ -1546,9 +1547,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     for (int kb = kb0; kb < kb1; ++kb, ++q) {
       if ((int)(q % (uint32_t)kGroups) != grp) continue;
       const int slot = (int)(q % kSlots);
-      const int sa = (int)(q % kTmemAStages);
+      const int sa = (int)(q % kAStages);
       if (!warp_wait(&bar->ifull[slot], ring_parity(q, kSlots), abort_flag, err, p.timeout_ns) ||
-          !warp_wait(&bar->aempty[sa], ring_parity(q, kTmemAStages) ^ 1u, abort_flag, err, p.timeout_ns))
+          !warp_wait(&bar->aempty[sa], ring_parity(q, kAStages) ^ 1u, abort_flag, err, p.timeout_ns))
         return false;
       tc_fence_after();  // the MMAs that read this A stage are complete
       const int k0 = kb * kBK;
@@ -1690,7 +1691,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       c.idesc = idesc_bf16_f32(kBM, BN, 0, 1);  // A from tensor memory, B (dY) MN-major
       c.a_lbo = 0, c.a_sbo = 0, c.a_step = 0;
       c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // 64-wide N groups 8 KB apart, 16 K rows per step
-      MmaIssuer mi = make_issuer(sm, kBBytes, kTmemAStages, SB, c);
+      MmaIssuer mi = make_issuer(sm, kBBytes, kAStages, SB, c);
       mi.a_tmem0 = tmem_base + kACol;
       uint32_t tc = 0;
       bool issued = false;
@@ -2508,7 +2509,7 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
     const uint32_t box[2] = {32u, 32u};
     prm.part_tma = make_tmap(&prm.tmap_part, prm.partial, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 1 : 0;
   }
-  prm.stages_a = kTmemAStages;
+  prm.stages_a = wgrad_a_stages(BN);
   prm.stages_b = 2;
   for (int b = 2; b <= kMaxStages; ++b)
     if (smem_total(wgrad_geometry(BN, b)) <= 226 * 1024) prm.stages_b = b;
