@@ -67,8 +67,14 @@ __global__ void __launch_bounds__(256) f32_conv_kernel(const float* __restrict__
     const int c = (int)(e - (long long)k * Cdst);
     Dot2 acc;
     if (bias) acc.add(bias[c]);
+    // the nine neighbour indices first (independent loads), so that the row loads of the
+    // taps do not each wait for their own index load
+    int mm[9];
+#pragma unroll
+    for (int j = 0; j < 9; ++j) mm[j] = __ldg(nbr + (size_t)k * 9 + (mirror ? 8 - j : j));
+#pragma unroll
     for (int j = 0; j < 9; ++j) {
-      const int m = nbr[(size_t)k * 9 + (mirror ? 8 - j : j)];
+      const int m = mm[j];
       if (m < 0) continue;
       if (m >= n) {
         atomicOr(err, SVCONV_STATUS_BAD_INDEX);
