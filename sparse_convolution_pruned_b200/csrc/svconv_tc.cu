@@ -77,9 +77,13 @@ constexpr int kConvPad = 32;                       // conv halo margin: W + 1 <=
 constexpr int kConvHaloRows = kBM + 2 * kConvPad;  // conv halo window (A rows m0 - 32 .. m0 + 159)
 constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
 constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
-__host__ __device__ constexpr int wgrad_slots(int bn) {  // weight gradient: index + halo slots in flight
-  return bn == 256 ? 5 : 8;  // (covers ~2 us of load latency at small C; at 256 columns three builder
-}                            //  groups hold three slots and the loader runs ahead by two)
+// Weight gradient: index + halo slots in flight.  8 cover ~2 us of load latency at small C.  At
+// 256 columns three builder groups hold three slots and the loader runs ahead by the rest: two
+// on single CTAs (their 32 KB dY stages take the space), three on CTA pairs (16 KB dY stages).
+__host__ __device__ constexpr int wgrad_slots(int bn, bool pair = false) { return bn == 256 ? (pair ? 6 : 5) : 8; }
+// Weight gradient: stages whose barriers the MMA issuer checks before issuing them (at most
+// the number of dY stages).  On CTA pairs a batch of four keeps the M = 256 MMAs queued.
+__host__ __device__ constexpr int wgrad_mma_group(bool pair) { return pair ? 4 : 2; }
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
@@ -143,11 +147,12 @@ struct Carve {
   uint8_t* epi;    // dense epilogue staging: 2 boxes of 32 rows x 128 bytes per epilogue warp
   uint8_t* halo;   // conv: 2 halo buffers; weight gradient: 2 slots x 2 halos
   int32_t* idx;    // 2 neighbour-row slots
+  float* bias;     // conv: each epilogue warp's copy of the tile's bias columns
   TcBarriers* bar;
 };
 
 struct Geometry {
-  size_t a_bytes, b_bytes, halo_bytes, idx_bytes, epi_bytes;
+  size_t a_bytes, b_bytes, halo_bytes, idx_bytes, epi_bytes, bias_bytes;
 };
 
 __host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -156,11 +161,15 @@ __host__ __device__ constexpr size_t round_up(size_t x, size_t a) { return (x + 
 // ring, but two halo buffers and two index slots.  Dense path: an A ring by TMA, no halo.
 // epi_stage: the epilogue's staging boxes (TMA stores).
 constexpr uint32_t kEpiBoxBytes = 32 * 128;  // 32 rows x 64 bf16 columns
-__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem, bool epi_stage = false) {
+// The epilogue reads the bias from shared memory: at full shared-memory use almost none is
+// left as L1, so per-column loads from global memory would wait on L2 with the MMAs stalled.
+constexpr int kEpiBiasCols = 256;  // bias columns an epilogue warp holds (the widest tile)
+__host__ __device__ inline Geometry conv_geometry(int bn, int sa, int sb, bool a_in_tmem, bool epi_stage, bool bias) {
   return {a_in_tmem ? (size_t)0 : (size_t)sa * kABytes, (size_t)sb * bn * kBK * 2,
           a_in_tmem ? (size_t)2 * kConvHaloRows * 128 : (size_t)0,
           a_in_tmem ? round_up((size_t)2 * kConvIdx * 4, 16) : (size_t)0,
-          epi_stage ? (size_t)kEpiWarps * 2 * kEpiBoxBytes : (size_t)0};
+          epi_stage ? (size_t)kEpiWarps * 2 * kEpiBoxBytes : (size_t)0,
+          bias ? (size_t)kEpiWarps * kEpiBiasCols * 4 : (size_t)0};
 }
 
 // Tensor-memory plan of the conv kernel: accumulator buffers first, then the A stages.
@@ -181,9 +190,10 @@ __host__ __device__ constexpr int conv_tmem_a_stages(int bn) {
 }
 
 // Weight gradient: A lives in tensor memory; wgrad_slots(bn) slots of (index entries, halo).
-__host__ __device__ inline Geometry wgrad_geometry(int bn, int sb) {
-  return {(size_t)0, (size_t)sb * bn * kBK * 2, (size_t)wgrad_slots(bn) * kWgHaloRows * 128,
-          round_up((size_t)wgrad_slots(bn) * kWgIdx * 4, 16)};
+// pair: a CTA of a pair loads half of the bn dY columns per stage.
+__host__ __device__ inline Geometry wgrad_geometry(int bn, int sb, bool pair = false) {
+  return {(size_t)0, (size_t)sb * (pair ? bn / 2 : bn) * kBK * 2, (size_t)wgrad_slots(bn, pair) * kWgHaloRows * 128,
+          round_up((size_t)wgrad_slots(bn, pair) * kWgIdx * 4, 16)};
 }
 __host__ __device__ constexpr int wgrad_acc_buffers(int bn) { return bn == 256 ? 1 : 2; }
 __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
@@ -191,7 +201,7 @@ __host__ __device__ constexpr uint32_t wgrad_tmem_cols(int bn) {
 }
 
 __host__ __device__ inline size_t smem_total(const Geometry& g) {
-  return 1024 + g.a_bytes + g.b_bytes + g.epi_bytes + g.halo_bytes + g.idx_bytes + sizeof(TcBarriers);
+  return 1024 + g.a_bytes + g.b_bytes + g.epi_bytes + g.halo_bytes + g.idx_bytes + g.bias_bytes + sizeof(TcBarriers);
 }
 
 __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
@@ -203,7 +213,8 @@ __device__ __forceinline__ Carve carve(uint8_t* smem_raw, const Geometry& g) {
   c.epi = c.b + g.b_bytes;  // 1024-aligned: the A and B stages are multiples of 1 KB
   c.halo = c.epi + g.epi_bytes;
   c.idx = reinterpret_cast<int32_t*>(c.halo + g.halo_bytes);
-  c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
+  c.bias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(c.idx) + g.idx_bytes);
+  c.bar = reinterpret_cast<TcBarriers*>(reinterpret_cast<uint8_t*>(c.bias) + g.bias_bytes);
   return c;
 }
 
@@ -547,11 +558,20 @@ __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + copysignf(erf_abs, x));
 }
 
-// 32 accumulator columns (raw fp32 bits) + bias[col ..], then GELU when asked.
-__device__ __forceinline__ void epi_bias_gelu(const TcConvParams& p, const uint32_t (&v)[32], float (&f)[32], int col) {
+// 32 accumulator columns (raw fp32 bits) + bias[col ..], then GELU when asked.  bias_s: the
+// shared-memory address of bias[col] (16-byte aligned), or 0 to read p.bias from global memory.
+__device__ __forceinline__ void epi_bias_gelu(const TcConvParams& p, const uint32_t (&v)[32], float (&f)[32], int col,
+                                              uint32_t bias_s = 0u) {
 #pragma unroll
   for (int q = 0; q < 32; ++q) f[q] = __uint_as_float(v[q]);
-  if (p.bias) {
+  if (bias_s) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 b = ld_shared_16(bias_s + 16u * q);  // the same address in every lane: a broadcast
+      f[4 * q] += __uint_as_float(b.x), f[4 * q + 1] += __uint_as_float(b.y);
+      f[4 * q + 2] += __uint_as_float(b.z), f[4 * q + 3] += __uint_as_float(b.w);
+    }
+  } else if (p.bias) {
     if ((reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0) {  // col is a multiple of 32
       const float4* b4 = reinterpret_cast<const float4*>(p.bias + col);
 #pragma unroll
@@ -571,7 +591,8 @@ __device__ __forceinline__ void epi_bias_gelu(const TcConvParams& p, const uint3
 }
 
 template <int BN>
-__device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t acc, bool valid, size_t orow, int n0) {
+__device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t acc, bool valid, size_t orow, int n0,
+                                              uint32_t bias_s = 0u) {
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 64) {
     uint32_t v[2][32];
@@ -583,7 +604,7 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
     for (int hh = 0; hh < 2; ++hh) {
       const int c = c0 + 32 * hh;
       float f[32];
-      epi_bias_gelu(p, v[hh], f, n0 + c);
+      epi_bias_gelu(p, v[hh], f, n0 + c, bias_s ? bias_s + 4u * (uint32_t)c : 0u);
       if (p.residual) {
         const uint4* rp = reinterpret_cast<const uint4*>(p.residual + orow * p.ldo + n0 + c);
 #pragma unroll
@@ -627,7 +648,7 @@ __device__ __forceinline__ void epilogue_rows(const TcConvParams& p, uint32_t ac
 // be rows of out that this tile owns.  q counts the boxes this warp has issued.
 template <int BN, bool REDUCE, typename Release>
 __device__ __forceinline__ void epilogue_tma(const TcConvParams& p, uint32_t acc, uint32_t boxes, uint32_t& q,
-                                             int orow0, int n0, Release release) {
+                                             int orow0, int n0, uint32_t bias_s, Release release) {
   const int lane = threadIdx.x & 31;
   const uint32_t row_off = (uint32_t)lane * 128u;
   const uint32_t sw = (uint32_t)(lane & 7);
@@ -644,7 +665,7 @@ __device__ __forceinline__ void epilogue_tma(const TcConvParams& p, uint32_t acc
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float f[32];
-      epi_bias_gelu(p, v[hh], f, n0 + c0 + 32 * hh);
+      epi_bias_gelu(p, v[hh], f, n0 + c0 + 32 * hh, bias_s ? bias_s + 4u * (uint32_t)(c0 + 32 * hh) : 0u);
       uint32_t packed[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -690,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
   constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns this CTA loads per stage
   constexpr int kRows = PAIR ? 2 * kBM : kBM;  // output rows per tile
   // gather: a B stage holds kGatherKb K-blocks (geometry counts them as wider stages)
-  const Geometry geo = conv_geometry(gather ? kBCols * kGatherKb : kBCols, SA, SB, gather, tma_epi);
+  const Geometry geo = conv_geometry(gather ? kBCols * kGatherKb : kBCols, SA, SB, gather, tma_epi, p.bias != nullptr);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1117,10 +1138,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
     uint32_t tc = 0, nbox = 0;
     const int out_base = p.out_abs ? lo : 0;
     const uint32_t epi_boxes = smem_u32(sm.epi) + (uint32_t)warp * 2u * kEpiBoxBytes;
+    // this warp's copy of the tile's bias columns (the data gradient has no bias)
+    float* const bias_w = sm.bias + warp * kEpiBiasCols;
+    const uint32_t bias_s = (!MIRROR && p.bias) ? smem_u32(bias_w) : 0u;
+    int bias_n0 = -1;
+    static_assert(BN <= kEpiBiasCols, "bias staging holds one tile's columns");
     for (int tile = unit0; tile < num_tiles; tile += units, ++tc) {
       const uint32_t ab = tc % (uint32_t)n_acc;
       const int m0 = (tile / n_tiles) * kRows + row_off;
       const int n0 = (tile % n_tiles) * BN;
+      if (!MIRROR && p.bias && n0 != bias_n0) {
+        // while the tile's MMAs run, once every lane is done with the old columns
+        __syncwarp();
+        for (int c = lane; c < BN; c += 32) bias_w[c] = __ldg(p.bias + n0 + c);
+        __syncwarp();
+        bias_n0 = n0;
+      }
       const int row = m0 + warp * 32 + lane;
       const int orow_i = out_base + row;
       if (p.residual && row < M && orow_i >= 0 && orow_i < p.out_rows) {
@@ -1145,11 +1178,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_kernel(const __grid_const
       };
       if (tma_epi && __all_sync(0xffffffffu, valid)) {
         if (p.out_tma == 2)
-          epilogue_tma<BN, true>(p, acc, epi_boxes, nbox, orow_i - lane, n0, release);
+          epilogue_tma<BN, true>(p, acc, epi_boxes, nbox, orow_i - lane, n0, bias_s, release);
         else
-          epilogue_tma<BN, false>(p, acc, epi_boxes, nbox, orow_i - lane, n0, release);
+          epilogue_tma<BN, false>(p, acc, epi_boxes, nbox, orow_i - lane, n0, bias_s, release);
       } else {
-        epilogue_rows<BN>(p, acc, valid, (size_t)orow_i, n0);
+        epilogue_rows<BN>(p, acc, valid, (size_t)orow_i, n0, bias_s);
         release();
       }
     }
@@ -1449,6 +1482,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
 // exactly the (channel lane, token-pair column) order of tcgen05.st.16x128b, so A
 // is transposed and gathered on the way in, with no shared-memory stores.  B is
 // dY by TMA (MN-major).
+//
+// PAIR (256 columns, an even number of 128-row tiles): a cluster of two CTAs takes two
+// adjacent row tiles with M = 256 MMAs, each CTA building its own tile's A in its tensor
+// memory and loading half of the dY columns, so a dY tile crosses into the SMs once per
+// 256 rows instead of once per 128.  CTA rank 0 issues the MMAs; the A / B full barriers
+// and the accumulator release count both CTAs and live in rank 0; the MMA commits arrive
+// in both CTAs.  Halo and index slots stay per CTA.
 // Weight-gradient builder, rare path (kept out of line so the builders' loop stays small):
 // the 16 registers of a 16-channel piece hold zeros for entries outside the halo window;
 // fetch those elements from global memory.
@@ -1475,43 +1515,63 @@ __device__ __noinline__ Regs16 wgrad_patch_far(Regs16 R, uint32_t sidx_s, const 
   return R;
 }
 
-template <int BN>
+template <int BN, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_constant__ TcWgradParams p) {
+  static_assert(!PAIR || BN == 256, "CTA pairs run 256-column tiles");
   extern __shared__ uint8_t smem_raw[];
   const int SB = p.stages_b;
-  const Geometry geo = wgrad_geometry(BN, SB);
+  const Geometry geo = wgrad_geometry(BN, SB, PAIR);
   const Carve sm = carve(smem_raw, geo);
   TcBarriers* bar = sm.bar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* err = p.status;
-  constexpr uint32_t kBBytes = BN * kBK * 2;
+  constexpr int kBCols = PAIR ? BN / 2 : BN;  // dY columns this CTA loads per stage
+  constexpr uint32_t kBBytes = kBCols * kBK * 2;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // first unit of this CTA (pair)
+  const int ustride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;  // unit stride
+  // rank 0's copy of a barrier (PAIR)
+  auto lead = [](uint64_t* b) -> uint32_t { return mapa_shared(smem_u32(b), 0u); };
   constexpr int kAcc = wgrad_acc_buffers(BN);
   constexpr uint32_t kTmemCols = wgrad_tmem_cols(BN);
   constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
-  constexpr int kSlots = wgrad_slots(BN);
+  constexpr int kSlots = wgrad_slots(BN, PAIR);
   constexpr int kAStages = wgrad_a_stages(BN);
   // Builder groups of four warps.  At 256 columns a CTA usually carries one unit, so its four
   // epilogue warps would idle until the very end: they build A stages as a third group.
   constexpr int kGroups = BN == 256 ? 3 : 2;
 
   const int m_tiles = p.rows_pad / kBM;
+  const int m_units = PAIR ? m_tiles / 2 : m_tiles;  // row tiles (PAIR: pairs of adjacent tiles)
   const int n_tiles = p.Cout / BN;
-  const int num_units = m_tiles * n_tiles * p.splits;
+  const int num_units = m_units * n_tiles * p.splits;
   const int kbt = (p.n + kBK - 1) / kBK;  // token blocks in total
 
   if (threadIdx.x == 0) {
     // ifull: 32 cp.async arrivals of the loader lanes + its expect_tx arrival
-    init_barriers(bar, kAStages, SB, kProdWarps / 2, kSlots, 33, kProdWarps / 2);
+    // afull: one builder group of four warps (of each CTA of a pair); tempty: the epilogue warps (of both)
+    init_barriers(bar, kAStages, SB, (PAIR ? 2 : 1) * (kProdWarps / 2), kSlots, 33, kProdWarps / 2,
+                  (PAIR ? 2 : 1) * kEpiWarps);
     prefetch_tmap(&p.tmap_x);
     prefetch_tmap(&p.tmap_dy);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&bar->tmem_base, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&bar->tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&bar->tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrival
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   pdl_wait();  // inputs and outputs may belong to the kernel before this one
   pdl_trigger();
@@ -1519,12 +1579,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   volatile int* abort_flag = &bar->abort_flag;
 
   // unit -> (split, m-tile, n-tile); units of one split run side by side so the
-  // tiles of dY and the X rows they share are hot in L2.
+  // tiles of dY and the X rows they share are hot in L2.  PAIR: this CTA's tile of the pair.
   auto decode = [&](int u, int& sp, int& mt, int& n0, int& kb0, int& kb1) {
     const int nt = u % n_tiles;
     const int rest = u / n_tiles;
-    mt = rest % m_tiles;
-    sp = rest / m_tiles;
+    mt = PAIR ? 2 * (rest % m_units) + (int)rank : rest % m_units;
+    sp = rest / m_units;
     n0 = nt * BN;
     kb0 = (int)((long long)kbt * sp / p.splits);
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
@@ -1612,7 +1672,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       // (padding halves are not written: their accumulator rows are never read)
       tmem_st_wait();
       tc_fence_before();
-      warp_arrive(&bar->afull[sa]);
+      if (PAIR && !leader) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead(&bar->afull[sa]));
+      } else {
+        warp_arrive(&bar->afull[sa]);
+      }
       warp_arrive(&bar->iempty[slot]);
     }
     return true;
@@ -1622,7 +1687,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     // ------------------------------------------------------------ index entries + halo window, per token block
     uint32_t q = 0;
     bool aborted = false;
-    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+    for (int u = unit0; u < num_units && !aborted; u += ustride) {
       int sp, mt, n0, kb0, kb1;
       decode(u, sp, mt, n0, kb0, kb1);
       const int cb = mt / kWgTiles;
@@ -1651,7 +1716,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     // ------------------------------------------------------------ dY tiles
     uint32_t it = 0;
     bool aborted = false;
-    for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+    for (int u = unit0; u < num_units && !aborted; u += ustride) {
       int sp, mt, n0, kb0, kb1;
       decode(u, sp, mt, n0, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -1662,15 +1727,37 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         }
         if (lane == 0) {
           const uint32_t dst = smem_u32(sm.b + (size_t)sb * kBBytes);
-          mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
+          if constexpr (PAIR) {
+            // this CTA's half of the columns, counted on rank 0's barrier
+            if (leader) mbar_arrive_expect_tx(&bar->bfull[sb], 2u * kBBytes);
+            const uint32_t fb = lead(&bar->bfull[sb]);
 #pragma unroll
-          for (int q = 0; q < BN / 64; ++q)
-            tma_load_2d(dst + q * 8192, &p.tmap_dy, &bar->bfull[sb], n0 + q * 64, kb * kBK);
+            for (int q = 0; q < kBCols / 64; ++q)
+              tma_load_2d_pair(dst + q * 8192, &p.tmap_dy, fb, n0 + (int)rank * kBCols + q * 64, kb * kBK);
+          } else {
+            mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q)
+              tma_load_2d(dst + q * 8192, &p.tmap_dy, &bar->bfull[sb], n0 + q * 64, kb * kBK);
+          }
         }
         __syncwarp();
       }
     }
-    if (aborted) drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+    if (aborted) {
+      if (PAIR && !leader) {
+        // the full barriers live in the other CTA: give this warp's copies in flight time
+        // to land instead of waiting on a phase
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000u) {
+          }
+        }
+        __syncwarp();
+      } else {
+        drain_ring(bar->bfull, it, SB, err, p.timeout_ns);
+      }
+    }
   } else if (warp >= kEpiWarps && warp < kHaloWarp) {
     // ------------------------------------------------------------ A builders (tensor memory)
     // Groups of four warps take turns over the token blocks (two groups, plus the epilogue
@@ -1682,37 +1769,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     // registers are then registers 4 k4 .. 4 k4 + 3 of the 16x128b.x8 store.
     const int grp = (warp - kEpiWarps) >> 2;
     uint32_t q = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x)
+    for (int u = unit0; u < num_units; u += ustride)
       if (!build_unit(u, q, grp)) break;
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       MmaCfg c;
-      c.idesc = idesc_bf16_f32(kBM, BN, 0, 1);  // A from tensor memory, B (dY) MN-major
+      c.idesc = idesc_bf16_f32(PAIR ? 2 * kBM : kBM, BN, 0, 1);  // A from tensor memory, B (dY) MN-major
       c.a_lbo = 0, c.a_sbo = 0, c.a_step = 0;
       c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // 64-wide N groups 8 KB apart, 16 K rows per step
       MmaIssuer mi = make_issuer(sm, kBBytes, kAStages, SB, c);
       mi.a_tmem0 = tmem_base + kACol;
       uint32_t tc = 0;
       bool issued = false;
-      for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+      for (int u = unit0; u < num_units; u += ustride, ++tc) {
         int sp, mt, n0, kb0, kb1;
         decode(u, sp, mt, n0, kb0, kb1);
         const uint32_t ab = tc % (uint32_t)kAcc;
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, kAcc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile<true, 2>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns)) break;
-        tc_commit(&bar->tfull[ab]);
+        if (!mma_tile<true, wgrad_mma_group(PAIR), PAIR>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err,
+                                                        p.timeout_ns))
+          break;
+        if constexpr (PAIR) {
+          tc_commit_pair(&bar->tfull[ab]);
+        } else {
+          tc_commit(&bar->tfull[ab]);
+        }
       }
-      mma_drain(bar, issued, err, p.timeout_ns);
+      mma_drain<PAIR>(bar, issued, err, p.timeout_ns);
+    } else if (PAIR && lane == 0) {
+      // the other CTA's MMAs read this CTA's tensor and shared memory: wait for them to finish
+      volatile int never = 0;
+      mbar_wait(&bar->done, 0, &never, err, p.timeout_ns);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue: fp32 partial rows
     uint32_t tc = 0;
     uint32_t qe = 0;  // block counter of the third builder group
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++tc) {
+    for (int u = unit0; u < num_units; u += ustride, ++tc) {
       if constexpr (kGroups == 3) {
         if (!build_unit(u, qe, 2)) break;
       }
@@ -1727,7 +1824,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       // The CTA's last unit: its MMAs are done and no dY tile will be loaded any more, so the
       // dY ring is free and stages the partial rows for TMA stores (whole lines, no per-thread
       // row stores); other units store their rows directly.
-      if (p.part_tma && u + (int)gridDim.x >= num_units) {
+      if (p.part_tma && u + ustride >= num_units) {
         const uint32_t boxes = smem_u32(sm.b) + (uint32_t)warp * 2u * 4096u;
         const uint32_t sw = (uint32_t)(lane & 7);
         const int prow0 = sp * p.rows_pad + mt * kBM + warp * 32;
@@ -1771,17 +1868,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
           }
         }
       }
+      // hand the accumulator back to the MMA issuer (at rank 0 of a pair)
       tc_fence_before();
-      warp_arrive(&bar->tempty[ab]);
+      if (PAIR && !leader) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead(&bar->tempty[ab]));
+      } else {
+        warp_arrive(&bar->tempty[ab]);
+      }
     }
     if (p.part_tma && lane == 0) bulk_wait_group<0>();  // partial-row stores complete before the CTA exits
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    cluster_sync();  // no CTA leaves while the other may still arrive on or read its memory
+  } else {
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    } else {
+      tmem_dealloc(tmem_base, kTmemCols);
+    }
   }
 }
 
@@ -2248,12 +2359,12 @@ static bool make_rows_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint
 // K-blocks of B fit, take that many B stages (B then stays resident across a CTA's tiles
 // with the same columns) and as many A stages (2-4) as remain; otherwise up to 4 A stages
 // (short latency) and as many B stages (TMA from L2) as fit.
-static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
-  const size_t budget = 220 * 1024;
+static void pick_stages(int bn, int num_kb, bool epi, bool bias, int* sa, int* sb) {
+  const size_t budget = 224 * 1024;
   if (num_kb <= kMaxStages) {
     for (int a = 4; a >= 2; --a) {
       const int b = num_kb < 2 ? 2 : num_kb;
-      if (smem_total(conv_geometry(bn, a, b, false, epi)) <= budget) {
+      if (smem_total(conv_geometry(bn, a, b, false, epi, bias)) <= budget) {
         *sa = a;
         *sb = b;
         return;
@@ -2263,7 +2374,7 @@ static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
   for (int a = 4; a >= 2; a -= 2) {
     int b_best = 0;
     for (int b = 2; b <= kMaxStages; ++b) {
-      const Geometry g = conv_geometry(bn, a, b, false, epi);
+      const Geometry g = conv_geometry(bn, a, b, false, epi, bias);
       if (smem_total(g) <= budget) b_best = b;
     }
     if (b_best >= 3 || (a == 2 && b_best >= 2)) {
@@ -2277,67 +2388,73 @@ static void pick_stages(int bn, int num_kb, bool epi, int* sa, int* sb) {
 }
 
 // grid: CTAs (PAIR: an even number, two per cluster).
+// A persistent kernel on clusters of two loops over its tiles, so it gets no more clusters
+// than can be resident at once: *grid (CTAs, even) is clamped to twice that number.  Per
+// kernel and device the count is queried once for a shared-memory size (host threads may
+// launch concurrently).
+template <auto kernel>
+static cudaError_t clamp_pair_grid(size_t smem, int* grid) {
+  static int occ_smem[64], occ_clusters[64];
+  static std::mutex occ_mu;
+  int d = 0;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(occ_mu);
+  int n = (d >= 0 && d < 64 && occ_smem[d] == (int)smem) ? occ_clusters[d] : 0;
+  if (n == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(*grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    if (d >= 0 && d < 64) occ_smem[d] = (int)smem, occ_clusters[d] = n;
+  }
+  if (*grid > 2 * n) *grid = 2 * n;
+  return cudaSuccess;
+}
+
 template <int BN, bool MIRROR, bool PAIR, bool F8 = false>
 static cudaError_t launch_conv_inst(TcConvParams& prm, int grid, cudaStream_t s) {
   const bool a_in_tmem = prm.nbr != nullptr;
+  const bool has_bias = prm.bias != nullptr;  // the epilogue warps' bias copies
   constexpr int kBCols = PAIR ? BN / 2 : BN;  // B columns per CTA
   if (a_in_tmem) {
     // A stage s in tensor memory and B stage s in shared memory advance together: as many
     // stages as both the free tensor-memory columns and the shared-memory budget allow
     int sb = 2;
     for (int b = 2; b <= kMaxStages; ++b)
-      if (smem_total(conv_geometry(kBCols * kGatherKb, 0, b, true, prm.out_tma != 0)) <= 220 * 1024) sb = b;
+      if (smem_total(conv_geometry(kBCols * kGatherKb, 0, b, true, prm.out_tma != 0, has_bias)) <= 224 * 1024) sb = b;
     prm.stages_a = prm.stages_b = conv_tmem_a_stages(BN) < sb ? conv_tmem_a_stages(BN) : sb;
   } else {
     const int num_kb = prm.taps * (prm.Kc / kBK);
-    pick_stages(kBCols, num_kb, prm.out_tma != 0, &prm.stages_a, &prm.stages_b);
+    pick_stages(kBCols, num_kb, prm.out_tma != 0, has_bias, &prm.stages_a, &prm.stages_b);
     if (num_kb > prm.stages_b) {
       // B streams: A stage s and B stage s on one barrier pair, as many stages as fit
       int st = 2;
       for (int b = 2; b <= kMaxStages; ++b)
-        if (smem_total(conv_geometry(kBCols, b, b, false, prm.out_tma != 0)) <= 220 * 1024) st = b;
+        if (smem_total(conv_geometry(kBCols, b, b, false, prm.out_tma != 0, has_bias)) <= 224 * 1024) st = b;
       prm.stages_a = prm.stages_b = st;
       prm.dense_pair_ring = 1;
     }
   }
   // (the same geometry the kernel carves: gather B stages hold kGatherKb K-blocks)
   const size_t smem = smem_total(conv_geometry(a_in_tmem ? kBCols * kGatherKb : kBCols, prm.stages_a, prm.stages_b,
-                                               a_in_tmem, prm.out_tma != 0));
+                                               a_in_tmem, prm.out_tma != 0, has_bias));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_conv_kernel<BN, MIRROR, PAIR, F8>, smem, done);
   if (e != cudaSuccess) return e;
   if constexpr (PAIR) {
-    // no more clusters than can be resident at once (the kernel loops over tiles)
-    // per device: resident clusters at this shared-memory size (queried once; host threads may
-    // launch concurrently)
-    static int occ_smem[64], occ_clusters[64];
-    static std::mutex occ_mu;
-    int d = 0;
-    e = cudaGetDevice(&d);
+    e = clamp_pair_grid<tc_conv_kernel<BN, MIRROR, PAIR, F8>>(smem, &grid);
     if (e != cudaSuccess) return e;
-    std::unique_lock<std::mutex> lk(occ_mu);
-    if (d < 0 || d >= 64 || occ_smem[d] != (int)smem) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(grid);
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, tc_conv_kernel<BN, MIRROR, PAIR, F8>, &cfg);
-      if (e != cudaSuccess) return e;
-      if (n < 1) return cudaErrorInvalidConfiguration;
-      if (d >= 0 && d < 64) occ_smem[d] = (int)smem, occ_clusters[d] = n;
-      if (grid > 2 * n) grid = 2 * n;
-    } else if (grid > 2 * occ_clusters[d]) {
-      grid = 2 * occ_clusters[d];
-    }
-    lk.unlock();
     return launch_pdl_cluster(tc_conv_kernel<BN, MIRROR, PAIR, F8>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
   } else
     return launch_pdl(tc_conv_kernel<BN, MIRROR, PAIR, F8>, dim3(grid), dim3(kThreads), smem, s, prm);
@@ -2500,7 +2617,7 @@ void tc_wgrad_plan_ctas(int n, int Cin, int Cout, int ctas, int* splits, int* ro
   *bn = b;
 }
 
-template <int BN>
+template <int BN, bool PAIR = false>
 static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t s) {
   // partial rows [splits * rows_pad][Cout] fp32 through TMA stores (boxes of 32 rows x 32 columns)
   if ((reinterpret_cast<uintptr_t>(prm.partial) & 15u) == 0 && prm.Cout % 32 == 0) {
@@ -2512,12 +2629,39 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
   prm.stages_a = wgrad_a_stages(BN);
   prm.stages_b = 2;
   for (int b = 2; b <= kMaxStages; ++b)
-    if (smem_total(wgrad_geometry(BN, b)) <= 226 * 1024) prm.stages_b = b;
-  const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_b));
+    if (smem_total(wgrad_geometry(BN, b, PAIR)) <= 226 * 1024) prm.stages_b = b;
+  // the issuer waits on a batch of stages before it issues (and releases) any of them
+  if (prm.stages_b < wgrad_mma_group(PAIR) || prm.stages_a < wgrad_mma_group(PAIR)) return cudaErrorInvalidConfiguration;
+  const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_b, PAIR));
   static int done[64];
-  cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN>, smem, done);
+  cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN, PAIR>, smem, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tc_wgrad_kernel<BN>, dim3(grid), dim3(kThreads), smem, s, prm);
+  if constexpr (PAIR) {
+    e = clamp_pair_grid<tc_wgrad_kernel<BN, PAIR>>(smem, &grid);
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cluster(tc_wgrad_kernel<BN, PAIR>, dim3(grid), dim3(kThreads), smem, s, 2u, prm);
+  } else {
+    return launch_pdl(tc_wgrad_kernel<BN, PAIR>, dim3(grid), dim3(kThreads), smem, s, prm);
+  }
+}
+
+// Grid and instantiation for a plan: 256 columns over an even number of row tiles run on
+// CTA pairs (one cluster per pair of row tiles and split), otherwise one CTA per unit.
+static cudaError_t launch_wgrad_plan(TcWgradParams& prm, int bn, cudaStream_t s) {
+  const int m_tiles = prm.rows_pad / kBM;
+  if (bn == 256 && m_tiles % 2 == 0) {
+    const int pair_units = (m_tiles / 2) * (prm.Cout / bn) * prm.splits;
+    int clusters = sm_count() / 2;
+    if (clusters > pair_units) clusters = pair_units;
+    if (clusters < 1) clusters = 1;
+    return launch_wgrad_inst<256, true>(prm, 2 * clusters, s);
+  }
+  const int units = m_tiles * (prm.Cout / bn) * prm.splits;
+  int grid = sm_count();
+  if (grid > units) grid = units;
+  if (bn == 256) return launch_wgrad_inst<256>(prm, grid, s);
+  if (bn == 128) return launch_wgrad_inst<128>(prm, grid, s);
+  return launch_wgrad_inst<64>(prm, grid, s);
 }
 
 cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
@@ -2539,12 +2683,7 @@ cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
   prm.Cout = a.Cout;
   prm.splits = splits;
   prm.rows_pad = rows_pad;
-  const int units = (rows_pad / kBM) * (a.Cout / bn) * splits;
-  int grid = sm_count();
-  if (grid > units) grid = units;
-  if (bn == 256) return launch_wgrad_inst<256>(prm, grid, s);
-  if (bn == 128) return launch_wgrad_inst<128>(prm, grid, s);
-  return launch_wgrad_inst<64>(prm, grid, s);
+  return launch_wgrad_plan(prm, bn, s);
 }
 
 // Same kernel with a caller-chosen number of token splits (1 <= splits <= token
@@ -2569,12 +2708,7 @@ cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s) {
   prm.Cout = a.Cout;
   prm.splits = a.splits;
   prm.rows_pad = rows_pad;
-  const int units = (rows_pad / kBM) * (a.Cout / bn) * a.splits;
-  int grid = sm_count();
-  if (grid > units) grid = units;
-  if (bn == 256) return launch_wgrad_inst<256>(prm, grid, s);
-  if (bn == 128) return launch_wgrad_inst<128>(prm, grid, s);
-  return launch_wgrad_inst<64>(prm, grid, s);
+  return launch_wgrad_plan(prm, bn, s);
 }
 
 cudaError_t launch_timeout_selftest(int32_t* status, uint64_t timeout_ns, cudaStream_t s) {
