@@ -2,16 +2,23 @@
 // gradients of one SparseConv2D in a single call (SV-TAD page, Key Design 2: dedicated
 // backward kernels; the formulas are the adjoints of the forward).
 //
-// Both gradients read the same dY and neighbour table and do not depend on each other.
-// At 64 input and output channels both kernels are latency-bound (each CTA waits ~3 us
-// for its first operands and carries one or two tiles), so running them side by side on
-// disjoint groups of SMs finishes sooner than running them one after the other: the data
-// gradient takes about 3/8 of the SMs on the caller's stream, the weight gradient and its
-// split reduce the rest on a side stream owned by the library, joined back to the caller's
-// stream with events.  Other shapes, and fp32, run the two entry points in order on the
-// caller's stream.
+// Both gradients read the same dY and neighbour table and do not depend on each other, so
+// they can run side by side on disjoint groups of SMs: the data gradient on the caller's
+// stream, the weight gradient and its split reduce on a side stream owned by the library,
+// joined back to the caller's stream with events.
+// * 64 input and output channels: both kernels are latency-bound (each CTA waits ~3 us for
+//   its first operands and carries one or two tiles); the data gradient takes about 3/8 of
+//   the SMs (measured best split).
+// * Multiples of 256 channels (CTA-pair kernels): a cost model picks the split.  Each kernel
+//   alone on the whole GPU pays its start and end once, and the data gradient's 256-row tiles
+//   rarely fill the last wave of 74 clusters; side by side, the data gradient gets the
+//   clusters that leave its waves full and the weight gradient a whole number of token
+//   splits (fewer partials to reduce).
+// Other shapes, and fp32, run the two entry points in order on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -36,17 +43,59 @@ struct SideStream {
 std::vector<SideStream> g_side;
 std::mutex g_side_mu;  // guards the table and each call's fork / launch / join sequence
 
-bool concurrent_shape(int dtype, int Cin, int Cout) { return dtype == SVCONV_BF16 && Cin == 64 && Cout == 64; }
+// How svconv_bwd runs the two gradients: side by side with these CTA budgets, or in order.
+struct BwdPlan {
+  bool side_by_side = false;
+  int data_ctas = 0, weight_ctas = 0;
+};
 
-// CTA budgets: weight gradient 94 of 148 SMs, data gradient the rest (measured best split).
-void budgets(int* data_ctas, int* weight_ctas) {
+// Cost model of the 256-column CTA-pair kernels, in SM cycles of one cluster (per-stage clock
+// traces on B200): a data-gradient tile of 256 rows costs ~580 cycles per 64-deep K-block plus
+// ~3,300 at its boundary (the epilogue drains the single accumulator); a weight-gradient unit
+// ~850 cycles per 64-token block; a kernel ~15,000 cycles of start (first loads) and end (last
+// epilogue); the split reduce ~1 cycle per 1,800 bytes of fp32 partials.
+constexpr double kDxKbCycles = 580.0, kDxTileCycles = 3300.0, kDwBlockCycles = 850.0, kKernelCycles = 15000.0;
+constexpr double kReduceBytesPerCycle = 1800.0;
+
+BwdPlan plan_bwd(int dtype, int n, int Cin, int Cout) {
+  BwdPlan p;
+  if (dtype != SVCONV_BF16 || n <= 0) return p;
   const int sms = sm_count();
-  int w = sms * 94 / 148;
-  if (w < 5) w = 5;
-  int d = sms - w;
-  if (d < 1) d = 1;
-  *data_ctas = d;
-  *weight_ctas = w;
+  if (Cin == 64 && Cout == 64) {
+    // weight gradient 94 of 148 SMs, data gradient the rest
+    int w = sms * 94 / 148;
+    if (w < 5) w = 5;
+    int d = sms - w;
+    if (d < 1) d = 1;
+    p.side_by_side = true;
+    p.data_ctas = d;
+    p.weight_ctas = w;
+    return p;
+  }
+  // (widths the entry points accept: the side-by-side call skips their checks)
+  if (Cin % 256 != 0 || Cout % 256 != 0 || Cin > 4096 || Cout > 4096) return p;
+  const int clusters = sms / 2;
+  const double tiles = (double)((n + 255) / 256) * (Cin / 256);               // data-gradient pair tiles
+  const double tile_cycles = 9.0 * Cout / 64 * kDxKbCycles + kDxTileCycles;
+  const int units = (Cin / 64) * 5 / 2 * (Cout / 256);                         // weight pair units per split
+  const double blocks = (double)((n + 63) / 64);
+  const double split_bytes = (double)(Cin / 64) * 5 * 128 * Cout * 4;         // one split's fp32 partial
+  auto t_weight = [&](int s) { return std::ceil(blocks / s) * kDwBlockCycles + kKernelCycles + s * split_bytes / kReduceBytesPerCycle; };
+  auto t_data = [&](int c) { return std::ceil(tiles / c) * tile_cycles + kKernelCycles; };
+  int s_full, rows_pad, bn;
+  tc_wgrad_plan(n, Cin, Cout, &s_full, &rows_pad, &bn);
+  double best = t_data(clusters) + t_weight(s_full);  // one after the other, each on the whole GPU
+  for (int s = 1; units * s < clusters && s <= (int)blocks; ++s) {
+    const int cx = clusters - units * s;
+    const double t = std::max(t_data(cx), t_weight(s));
+    if (t < 0.97 * best) {
+      best = t;
+      p.side_by_side = true;
+      p.data_ctas = 2 * cx;
+      p.weight_ctas = 2 * units * s;
+    }
+  }
+  return p;
 }
 
 // Side stream of (current device, caller), created on first use (call with g_side_mu held).
@@ -88,17 +137,19 @@ using namespace svc;
 extern "C" {
 
 size_t svconv_bwd_workspace_size(int dtype, int n, int Cin, int Cout) {
-  if (!concurrent_shape(dtype, Cin, Cout) || n <= 0) return svconv_bwd_weight_workspace_size(dtype, n, Cin, Cout);
-  int dc, wc, splits, rows_pad, bn;
-  budgets(&dc, &wc);
-  tc_wgrad_plan_ctas(n, Cin, Cout, wc, &splits, &rows_pad, &bn);
+  if (n <= 0 || Cin <= 0 || Cout <= 0) return svconv_bwd_weight_workspace_size(dtype, n, Cin, Cout);
+  const BwdPlan plan = plan_bwd(dtype, n, Cin, Cout);
+  if (!plan.side_by_side) return svconv_bwd_weight_workspace_size(dtype, n, Cin, Cout);
+  int splits, rows_pad, bn;
+  tc_wgrad_plan_ctas(n, Cin, Cout, plan.weight_ctas, &splits, &rows_pad, &bn);
   return (size_t)splits * rows_pad * Cout * sizeof(float);
 }
 
 int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
                const void* Wt, void* dX, float* dW, float* db, void* workspace, size_t ws_bytes, void* stream) {
   if (n < 0 || Cin <= 0 || Cout <= 0) return SVCONV_ERR_SIZE;
-  if (!concurrent_shape(dtype, Cin, Cout) || n == 0) {
+  const BwdPlan plan = plan_bwd(dtype, n, Cin, Cout);
+  if (!plan.side_by_side) {
     const int rc = svconv_bwd_data(dtype, dY, nbr, n, Cin, Cout, Wt, dX, stream);
     if (rc) return rc;
     return svconv_bwd_weight(dtype, dY, X, nbr, n, Cin, Cout, dW, db, workspace, ws_bytes, stream);
@@ -112,8 +163,7 @@ int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int
   if (!aligned16(dY) || !aligned16(X) || !aligned16(Wt) || !aligned16(dX)) return SVCONV_ERR_ALIGN;
   if (!workspace || ws_bytes < svconv_bwd_workspace_size(dtype, n, Cin, Cout)) return SVCONV_ERR_WORKSPACE;
   if (!aligned16(workspace)) return SVCONV_ERR_ALIGN;
-  int dc, wc;
-  budgets(&dc, &wc);
+  const int dc = plan.data_ctas, wc = plan.weight_ctas;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lk(g_side_mu);
   SideStream* side = side_stream(s);

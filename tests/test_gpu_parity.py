@@ -247,6 +247,11 @@ def test_bf16_full_size_complete(sv, orc, make, with_bwd):
 
 FUSED_BWD_CASES = [
     ("small_c_concurrent", lambda: wl.small_c_bf16(), torch.bfloat16),
+    # 256-channel multiples: the two gradients side by side on disjoint SMs (CTA budgets from the
+    # cost model; the weight gradient with its own, smaller split count)
+    ("C256_T48_concurrent", lambda: wl.large_c_bwd_bf16(T=48), torch.bfloat16),
+    ("C512x256_concurrent", lambda: wl.custom_conv(seed=34, T=6, H=16, W=16, keep_frac=0.5, Cin=512, Cout=256,
+                                                   dtype="bf16", shuffle=True, empty_frames=(2,)), torch.bfloat16),
     ("C64_tiny_frames_concurrent", lambda: wl.custom_conv(seed=42, T=5, H=4, W=4, keep_frac=[0.0, 1 / 16, 0.0, 1.0, 0.5],
                                                           Cin=64, Cout=64, dtype="bf16"), torch.bfloat16),
     ("C128x192_sequential", lambda: wl.custom_conv(seed=31, T=7, H=9, W=14, keep_frac=0.55, Cin=128, Cout=192,
@@ -276,15 +281,17 @@ def test_fused_bwd(sv, orc, name, make, dtype):
     assert sv.svconv_read_error_word() == 0
 
 
-def test_fused_bwd_in_cuda_graph(sv):
-    w = wl.small_c_bf16(T=96)
+@pytest.mark.parametrize("make", [lambda: wl.small_c_bf16(T=96), lambda: wl.large_c_bwd_bf16(T=24)], ids=["C64", "C256"])
+def test_fused_bwd_in_cuda_graph(sv, make):
+    w = make()
     nbr, _, st = gpu_index(sv, w, want_map=False)
     X, Wt, dY = dev(w.X, torch.bfloat16), dev(w.Wt, torch.bfloat16), dev(w.dY, torch.bfloat16)
     ref = [t.clone() for t in sv.svconv_bwd(dY, X, nbr, Wt)]  # first call outside capture
     dX = torch.zeros_like(ref[0])
     dW = torch.zeros_like(ref[1])
     db = torch.zeros_like(ref[2])
-    ws = torch.empty(sv.svconv_bwd_workspace_size(sv.BF16, w.n, 64, 64), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(16, sv.svconv_bwd_workspace_size(sv.BF16, w.n, w.Cin, w.Cout)), dtype=torch.uint8,
+                     device="cuda")
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         g = torch.cuda.CUDAGraph()
