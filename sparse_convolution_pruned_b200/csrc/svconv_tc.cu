@@ -77,13 +77,13 @@ constexpr int kConvPad = 32;                       // conv halo margin: W + 1 <=
 constexpr int kConvHaloRows = kBM + 2 * kConvPad;  // conv halo window (A rows m0 - 32 .. m0 + 159)
 constexpr int kWgPad = 32;                         // weight-gradient halo margin: W + 1 <= 32 stays inside
 constexpr int kWgHaloRows = kBK + 2 * kWgPad;      // weight-gradient halo window (rows k0 - 32 .. k0 + 95)
-// Weight gradient: index + halo slots in flight.  8 cover ~2 us of load latency at small C.  At
-// 256 columns three builder groups hold three slots and the loader runs ahead by the rest: two
-// on single CTAs (their 32 KB dY stages take the space), three on CTA pairs (16 KB dY stages).
-__host__ __device__ constexpr int wgrad_slots(int bn, bool pair = false) { return bn == 256 ? (pair ? 6 : 5) : 8; }
-// Weight gradient: stages whose barriers the MMA issuer checks before issuing them (at most
-// the number of dY stages).  On CTA pairs a batch of four keeps the M = 256 MMAs queued.
-__host__ __device__ constexpr int wgrad_mma_group(bool pair) { return pair ? 4 : 2; }
+// Weight gradient: index + halo slots in flight (one per 64-token block).  8 cover ~2 us of
+// load latency at small C.  At 256 columns three builder groups hold three slots and the
+// loader runs ahead by two; the 32 KB dY (or dY-pair) stages take the rest of the space.
+__host__ __device__ constexpr int wgrad_slots(int bn, bool pair = false) { return bn == 256 ? 5 : 8; }
+// Weight gradient on CTA pairs: at most this many two-block stages fit next to the 256-column
+// accumulator in tensor memory (2 x 32 columns each).
+constexpr int kWgPairStagesMax = 4;
 constexpr int kWgTiles = 5;                        // weight gradient: 128-row tiles per 64-channel block
 constexpr int kConvIdx = kBM * 9;                  // neighbour entries of a conv tile
 constexpr int kWgIdx = kBK * 9;                    // neighbour entries of a 64-token block
@@ -124,7 +124,7 @@ struct TcConvParams {
 };
 
 struct TcWgradParams {
-  CUtensorMap tmap_x;   // X [n][Cin], halo boxes {64, 64}
+  CUtensorMap tmap_x;   // X [n][Cin], halo window boxes {64, 128}
   CUtensorMap tmap_dy;  // dY [n][Cout], box {64, 64}
   CUtensorMap tmap_part;  // part_tma: partial [splits * rows_pad][Cout] fp32, box {32, 32}
   const __nv_bfloat16* X;
@@ -190,9 +190,10 @@ __host__ __device__ constexpr int conv_tmem_a_stages(int bn) {
 }
 
 // Weight gradient: A lives in tensor memory; wgrad_slots(bn) slots of (index entries, halo).
-// pair: a CTA of a pair loads half of the bn dY columns per stage.
+// A dY stage is bn columns of one 64-token block, or on a CTA pair half of them for two blocks:
+// the same bytes.
 __host__ __device__ inline Geometry wgrad_geometry(int bn, int sb, bool pair = false) {
-  return {(size_t)0, (size_t)sb * (pair ? bn / 2 : bn) * kBK * 2, (size_t)wgrad_slots(bn, pair) * kWgHaloRows * 128,
+  return {(size_t)0, (size_t)sb * bn * kBK * 2, (size_t)wgrad_slots(bn, pair) * kWgHaloRows * 128,
           round_up((size_t)wgrad_slots(bn, pair) * kWgIdx * 4, 16)};
 }
 __host__ __device__ constexpr int wgrad_acc_buffers(int bn) { return bn == 256 ? 1 : 2; }
@@ -1488,7 +1489,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_conv_small_kernel(const __grid
 // memory and loading half of the dY columns, so a dY tile crosses into the SMs once per
 // 256 rows instead of once per 128.  CTA rank 0 issues the MMAs; the A / B full barriers
 // and the accumulator release count both CTAs and live in rank 0; the MMA commits arrive
-// in both CTAs.  Halo and index slots stay per CTA.
+// in both CTAs.  Halo and index slots stay per CTA.  A pair's stage holds two token blocks
+// (A: 2 x 32 tensor-memory columns; B: both blocks' dY halves) on ONE full / empty barrier
+// pair, as in the gather conv, so the issuing thread waits and commits once per 8 MMAs.
 // Weight-gradient builder, rare path (kept out of line so the builders' loop stays small):
 // the 16 registers of a 16-channel piece hold zeros for entries outside the halo window;
 // fetch those elements from global memory.
@@ -1538,7 +1541,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   constexpr uint32_t kACol = (uint32_t)(kAcc * BN);  // first column of the A stages
   constexpr uint32_t kHaloBufBytes = kWgHaloRows * 128;
   constexpr int kSlots = wgrad_slots(BN, PAIR);
-  constexpr int kAStages = wgrad_a_stages(BN);
+  // PAIR: stages of kKbs = 2 token blocks, A and B on one barrier pair (p.stages_a == p.stages_b)
+  constexpr int kKbs = PAIR ? 2 : 1;
+  const int kAStages = p.stages_a;
   // Builder groups of four warps.  At 256 columns a CTA usually carries one unit, so its four
   // epilogue warps would idle until the very end: they build A stages as a third group.
   constexpr int kGroups = BN == 256 ? 3 : 2;
@@ -1552,8 +1557,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     // ifull: 32 cp.async arrivals of the loader lanes + its expect_tx arrival
     // afull: one builder group of four warps (of each CTA of a pair); tempty: the epilogue warps (of both)
-    init_barriers(bar, kAStages, SB, (PAIR ? 2 : 1) * (kProdWarps / 2), kSlots, 33, kProdWarps / 2,
-                  (PAIR ? 2 : 1) * kEpiWarps);
+    // PAIR: afull also counts the weight loader's expect_tx arrival (rank 0)
+    init_barriers(bar, kAStages, PAIR ? 0 : SB, PAIR ? 2 * (kProdWarps / 2) + 1 : kProdWarps / 2, kSlots, 33,
+                  kProdWarps / 2, (PAIR ? 2 : 1) * kEpiWarps);
     prefetch_tmap(&p.tmap_x);
     prefetch_tmap(&p.tmap_dy);
   }
@@ -1590,10 +1596,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     kb1 = (int)((long long)kbt * (sp + 1) / p.splits);
   };
 
-  // Builds the A stages of unit u's token blocks whose running index q satisfies
-  // q % kGroups == grp (q counts every block of the CTA, so the groups stay in step); false
-  // when a wait gave up.
-  auto build_unit = [&](int u, uint32_t& q, int grp) -> bool {
+  // Builds the A stages of unit u whose running stage index qs satisfies qs % kGroups == grp
+  // (qs counts every stage of the CTA and qb every token block, so the groups stay in step);
+  // false when a wait gave up.
+  auto build_unit = [&](int u, uint32_t& qs, uint32_t& qb, int grp) -> bool {
     const int quarter = warp & 3;
     const int half = quarter >> 1;
     const int cq = (quarter & 1) * 32;
@@ -1604,72 +1610,79 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     const int cb = mt / kWgTiles;
     const int j = 2 * (mt % kWgTiles) + half;        // tap of this warp's half (9: the extra half)
     const int kind = j < 9 ? 0 : (cb == 0 ? 1 : 2);  // gathered X, ones row, padding
-    for (int kb = kb0; kb < kb1; ++kb, ++q) {
-      if ((int)(q % (uint32_t)kGroups) != grp) continue;
-      const int slot = (int)(q % kSlots);
-      const int sa = (int)(q % kAStages);
-      if (!warp_wait(&bar->ifull[slot], ring_parity(q, kSlots), abort_flag, err, p.timeout_ns) ||
-          !warp_wait(&bar->aempty[sa], ring_parity(q, kAStages) ^ 1u, abort_flag, err, p.timeout_ns))
-        return false;
-      tc_fence_after();  // the MMAs that read this A stage are complete
-      const int k0 = kb * kBK;
-      const uint32_t a_col = tmem_base + kACol + (uint32_t)sa * kTmemAStageCols;
-      if (kind == 0) {
-        const uint32_t sidx_s = smem_u32(sm.idx + slot * kWgIdx);
-        const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
-        const int hlo = k0 - kWgPad;
-        const int mi = lane >> 3;
-#pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
-          const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
-          uint32_t R[16];
-          bool far = false, bad = false;
-          const int chunk = (c16 >> 3) + (mi & 1);
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            // branch-free: entries of tokens past n (stale slot contents) count as missing
-            const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
-            const int raw = ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j));
-            const bool tok_ok = k0 + tk < p.n;
-            bad |= tok_ok & (raw >= p.n);
-            const int x = (tok_ok & (raw < p.n)) ? raw : -1;
-            const int h = x - hlo;
-            const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kWgHaloRows);
-            far |= (x >= 0) & !in_win;
-            const uint32_t addr =
-                in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_addr;
-            ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
-          }
-          if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
-          if (__any_sync(0xffffffffu, far)) {
-            // entries outside the halo window read as zero above: fetch them from global memory
-            Regs16 rr;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) rr.v[r] = R[r];
-            rr = wgrad_patch_far(rr, sidx_s, X16, p.n, p.Cin, k0, hlo, j, cb * kBK + c16);
-#pragma unroll
-            for (int r = 0; r < 16; ++r) R[r] = rr.v[r];
-          }
-          tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
-        }
-      } else if (kind == 1) {
-        // row 0 of the extra half is 1 for every valid token: its accumulator row is db
-#pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
-          uint32_t R[16];
-#pragma unroll
-          for (int r = 0; r < 16; ++r) R[r] = 0u;
-          if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int tk = k0 + 8 * k + 2 * lane;
-              R[2 * k] = (tk < p.n ? 0x3F80u : 0u) | (tk + 1 < p.n ? 0x3F800000u : 0u);
-            }
-          }
-          tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
-        }
+    for (int kbs = kb0; kbs < kb1; kbs += kKbs, ++qs) {
+      const int nb = min(kKbs, kb1 - kbs);  // token blocks in this stage
+      if ((int)(qs % (uint32_t)kGroups) != grp) {
+        qb += (uint32_t)nb;
+        continue;
       }
-      // (padding halves are not written: their accumulator rows are never read)
+      const int sa = (int)(qs % (uint32_t)kAStages);
+      if (!warp_wait(&bar->aempty[sa], ring_parity(qs, kAStages) ^ 1u, abort_flag, err, p.timeout_ns)) return false;
+      tc_fence_after();  // the MMAs that read this A stage are complete
+      for (int hb = 0; hb < nb; ++hb, ++qb) {
+        const int kb = kbs + hb;
+        const int slot = (int)(qb % kSlots);
+        if (!warp_wait(&bar->ifull[slot], ring_parity(qb, kSlots), abort_flag, err, p.timeout_ns)) return false;
+        const int k0 = kb * kBK;
+        const uint32_t a_col = tmem_base + kACol + (uint32_t)(sa * kKbs + hb) * kTmemAStageCols;
+        if (kind == 0) {
+          const uint32_t sidx_s = smem_u32(sm.idx + slot * kWgIdx);
+          const uint32_t halo = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
+          const int hlo = k0 - kWgPad;
+          const int mi = lane >> 3;
+  #pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const int c16 = cq + 16 * sub;  // first channel of these 16 lanes
+            uint32_t R[16];
+            bool far = false, bad = false;
+            const int chunk = (c16 >> 3) + (mi & 1);
+  #pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              // branch-free: entries of tokens past n (stale slot contents) count as missing
+              const int tk = 16 * k4 + 8 * (mi >> 1) + (lane & 7);
+              const int raw = ld_shared_s32(sidx_s + 4u * (uint32_t)(tk * 9 + j));
+              const bool tok_ok = k0 + tk < p.n;
+              bad |= tok_ok & (raw >= p.n);
+              const int x = (tok_ok & (raw < p.n)) ? raw : -1;
+              const int h = x - hlo;
+              const bool in_win = (x >= 0) & ((unsigned)h < (unsigned)kWgHaloRows);
+              far |= (x >= 0) & !in_win;
+              const uint32_t addr =
+                  in_win ? halo + (uint32_t)h * 128u + ((uint32_t)(chunk ^ (h & 7)) << 4) : zero_addr;
+              ldmatrix_x4_trans(addr, R[4 * k4], R[4 * k4 + 1], R[4 * k4 + 2], R[4 * k4 + 3]);
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(err, SVCONV_STATUS_BAD_INDEX);
+            if (__any_sync(0xffffffffu, far)) {
+              // entries outside the halo window read as zero above: fetch them from global memory
+              Regs16 rr;
+  #pragma unroll
+              for (int r = 0; r < 16; ++r) rr.v[r] = R[r];
+              rr = wgrad_patch_far(rr, sidx_s, X16, p.n, p.Cin, k0, hlo, j, cb * kBK + c16);
+  #pragma unroll
+              for (int r = 0; r < 16; ++r) R[r] = rr.v[r];
+            }
+            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+          }
+        } else if (kind == 1) {
+          // row 0 of the extra half is 1 for every valid token: its accumulator row is db
+  #pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            uint32_t R[16];
+  #pragma unroll
+            for (int r = 0; r < 16; ++r) R[r] = 0u;
+            if ((quarter & 1) == 0 && sub == 0 && lane < 4) {
+  #pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int tk = k0 + 8 * k + 2 * lane;
+                R[2 * k] = (tk < p.n ? 0x3F80u : 0u) | (tk + 1 < p.n ? 0x3F800000u : 0u);
+              }
+            }
+            tmem_st_16x128b_x8(a_col + ((uint32_t)(32 * quarter + 16 * sub) << 16), R);
+          }
+        }
+        // (padding halves are not written: their accumulator rows are never read)
+        warp_arrive(&bar->iempty[slot]);  // the halo and index rows are in registers / tensor memory
+      }
       tmem_st_wait();
       tc_fence_before();
       if (PAIR && !leader) {
@@ -1678,7 +1691,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       } else {
         warp_arrive(&bar->afull[sa]);
       }
-      warp_arrive(&bar->iempty[slot]);
     }
     return true;
   };
@@ -1704,9 +1716,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
                            &bar->ifull[slot], kHaloBufBytes);
         if (lane == 0) {
           const uint32_t hb = smem_u32(sm.halo + (size_t)slot * kHaloBufBytes);
-#pragma unroll
-          for (int b = 0; b < kWgHaloRows / kHaloBox; ++b)
-            tma_load_2d(hb + b * kHaloBox * 128, &p.tmap_x, &bar->ifull[slot], cb * kBK, k0 - kWgPad + b * kHaloBox);
+          // the whole window in one box: the loader's issue time per block, not bytes, paced
+          // the kernel (one copy fewer per block measured 3% faster)
+          tma_load_2d(hb, &p.tmap_x, &bar->ifull[slot], cb * kBK, k0 - kWgPad);
         }
         __syncwarp();
       }
@@ -1719,21 +1731,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     for (int u = unit0; u < num_units && !aborted; u += ustride) {
       int sp, mt, n0, kb0, kb1;
       decode(u, sp, mt, n0, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      for (int kb = kb0; kb < kb1; kb += kKbs, ++it) {
         const int sb = (int)(it % (uint32_t)SB);
-        if (!warp_wait(&bar->bempty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
+        uint64_t* const empty = PAIR ? bar->aempty : bar->bempty;  // PAIR: one ring with the A stages
+        if (!warp_wait(&empty[sb], ring_parity(it, SB) ^ 1u, abort_flag, err, p.timeout_ns)) {
           aborted = true;
           break;
         }
         if (lane == 0) {
-          const uint32_t dst = smem_u32(sm.b + (size_t)sb * kBBytes);
+          const uint32_t dst = smem_u32(sm.b + (size_t)sb * kKbs * kBBytes);
           if constexpr (PAIR) {
-            // this CTA's half of the columns, counted on rank 0's barrier
-            if (leader) mbar_arrive_expect_tx(&bar->bfull[sb], 2u * kBBytes);
-            const uint32_t fb = lead(&bar->bfull[sb]);
+            // this CTA's half of the columns of the stage's blocks, counted on rank 0's full barrier
+            const int nb = min(kKbs, kb1 - kb);
+            if (leader) mbar_arrive_expect_tx(&bar->afull[sb], 2u * (uint32_t)nb * kBBytes);
+            const uint32_t fb = lead(&bar->afull[sb]);
+            for (int h = 0; h < nb; ++h) {
 #pragma unroll
-            for (int q = 0; q < kBCols / 64; ++q)
-              tma_load_2d_pair(dst + q * 8192, &p.tmap_dy, fb, n0 + (int)rank * kBCols + q * 64, kb * kBK);
+              for (int q = 0; q < kBCols / 64; ++q)
+                tma_load_2d_pair(dst + h * kBBytes + q * 8192, &p.tmap_dy, fb, n0 + (int)rank * kBCols + q * 64,
+                                 (kb + h) * kBK);
+            }
           } else {
             mbar_arrive_expect_tx(&bar->bfull[sb], kBBytes);
 #pragma unroll
@@ -1745,9 +1762,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       }
     }
     if (aborted) {
-      if (PAIR && !leader) {
-        // the full barriers live in the other CTA: give this warp's copies in flight time
-        // to land instead of waiting on a phase
+      if (PAIR) {
+        // the full barriers live in rank 0 and also count the builders: give this warp's
+        // copies in flight time to land instead of waiting on a phase
         if (lane == 0) {
           const uint64_t t0 = globaltimer_ns();
           while (globaltimer_ns() - t0 < 200000u) {
@@ -1768,9 +1785,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
     // halo row of token 16 k4 + 8 (i / 16) + i % 8, channels +8 ((i / 8) % 2); its four
     // registers are then registers 4 k4 .. 4 k4 + 3 of the 16x128b.x8 store.
     const int grp = (warp - kEpiWarps) >> 2;
-    uint32_t q = 0;
+    uint32_t qs = 0, qb = 0;
     for (int u = unit0; u < num_units; u += ustride)
-      if (!build_unit(u, q, grp)) break;
+      if (!build_unit(u, qs, qb, grp)) break;
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
@@ -1778,7 +1795,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
       c.idesc = idesc_bf16_f32(PAIR ? 2 * kBM : kBM, BN, 0, 1);  // A from tensor memory, B (dY) MN-major
       c.a_lbo = 0, c.a_sbo = 0, c.a_step = 0;
       c.b_lbo = 8192, c.b_sbo = 1024, c.b_step = 2048;  // 64-wide N groups 8 KB apart, 16 K rows per step
-      MmaIssuer mi = make_issuer(sm, kBBytes, kAStages, SB, c);
+      MmaIssuer mi = make_issuer(sm, kKbs * kBBytes, kAStages, SB, c);
       mi.a_tmem0 = tmem_base + kACol;
       uint32_t tc = 0;
       bool issued = false;
@@ -1789,9 +1806,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
         if (!mbar_wait(&bar->tempty[ab], ring_parity(tc, kAcc) ^ 1u, abort_flag, err, p.timeout_ns)) break;
         tc_fence_after();
         issued = true;
-        if (!mma_tile<true, wgrad_mma_group(PAIR), PAIR>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err,
-                                                        p.timeout_ns))
-          break;
+        bool ok;
+        if constexpr (PAIR) {
+          ok = mma_tile_unified<1, true, kKbs>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        } else {
+          ok = mma_tile<true, 2>(bar, mi, kb1 - kb0, tmem_base + ab * BN, abort_flag, err, p.timeout_ns);
+        }
+        if (!ok) break;
         if constexpr (PAIR) {
           tc_commit_pair(&bar->tfull[ab]);
         } else {
@@ -1808,10 +1829,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_wgrad_kernel(const __grid_cons
   } else {
     // ------------------------------------------------------------ epilogue: fp32 partial rows
     uint32_t tc = 0;
-    uint32_t qe = 0;  // block counter of the third builder group
+    uint32_t qes = 0, qeb = 0;  // stage and block counters of the third builder group
     for (int u = unit0; u < num_units; u += ustride, ++tc) {
       if constexpr (kGroups == 3) {
-        if (!build_unit(u, qe, 2)) break;
+        if (!build_unit(u, qes, qeb, 2)) break;
       }
       int sp, mt, n0, kb0, kb1;
       decode(u, sp, mt, n0, kb0, kb1);
@@ -2626,12 +2647,18 @@ static cudaError_t launch_wgrad_inst(TcWgradParams& prm, int grid, cudaStream_t 
     const uint32_t box[2] = {32u, 32u};
     prm.part_tma = make_tmap(&prm.tmap_part, prm.partial, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 1 : 0;
   }
-  prm.stages_a = wgrad_a_stages(BN);
   prm.stages_b = 2;
   for (int b = 2; b <= kMaxStages; ++b)
     if (smem_total(wgrad_geometry(BN, b, PAIR)) <= 226 * 1024) prm.stages_b = b;
-  // the issuer waits on a batch of stages before it issues (and releases) any of them
-  if (prm.stages_b < wgrad_mma_group(PAIR) || prm.stages_a < wgrad_mma_group(PAIR)) return cudaErrorInvalidConfiguration;
+  if constexpr (PAIR) {
+    // one ring: A (tensor memory) and dY (shared memory) stages advance together
+    if (prm.stages_b > kWgPairStagesMax) prm.stages_b = kWgPairStagesMax;
+    prm.stages_a = prm.stages_b;
+  } else {
+    prm.stages_a = wgrad_a_stages(BN);
+    // the issuer checks two stages of each ring before it issues (and releases) either
+    if (prm.stages_b < 2) return cudaErrorInvalidConfiguration;
+  }
   const size_t smem = smem_total(wgrad_geometry(BN, prm.stages_b, PAIR));
   static int done[64];
   cudaError_t e = ensure_smem_attr(tc_wgrad_kernel<BN, PAIR>, smem, done);
@@ -2670,7 +2697,7 @@ cudaError_t launch_tc_wgrad(const TcWgradArgs& a, cudaStream_t s) {
   int splits, rows_pad, bn;
   tc_wgrad_plan(a.n, a.Cin, a.Cout, &splits, &rows_pad, &bn);
   if (splits != a.splits || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
-  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kHaloBox))
+  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kWgHaloRows))
     return cudaErrorInvalidValue;
   if (!make_rows_tmap(&prm.tmap_dy, a.dY, (uint64_t)a.n, (uint64_t)a.Cout, 64u)) return cudaErrorInvalidValue;
   prm.X = static_cast<const __nv_bfloat16*>(a.X);
@@ -2695,7 +2722,7 @@ cudaError_t launch_tc_wgrad_with_splits(const TcWgradArgs& a, cudaStream_t s) {
   tc_wgrad_plan(a.n, a.Cin, a.Cout, &plan_splits, &rows_pad, &bn);
   const int kbt = (a.n + kBK - 1) / kBK;
   if (a.splits < 1 || a.splits > kbt || rows_pad != a.rows_pad) return cudaErrorInvalidValue;
-  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kHaloBox))
+  if (!make_rows_tmap(&prm.tmap_x, a.X, (uint64_t)a.n, (uint64_t)a.Cin, (uint32_t)kWgHaloRows))
     return cudaErrorInvalidValue;
   if (!make_rows_tmap(&prm.tmap_dy, a.dY, (uint64_t)a.n, (uint64_t)a.Cout, 64u)) return cudaErrorInvalidValue;
   prm.X = static_cast<const __nv_bfloat16*>(a.X);
