@@ -168,7 +168,10 @@ SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
  *   db [Cout] fp32 (db may be NULL) are overwritten.
  *   workspace: device, at least svconv_bwd_workspace_size(...) bytes, 16-byte
  *   aligned, no initial contents required.
- *   bf16 with C_in = C_out = 64: the two gradients run side by side on disjoint
+ *   bf16 with C_in = C_out = 64, and bf16 with C_in, C_out multiples of 256 (up to
+ *   4096) when a cost model of the two kernels says it is shorter (CTA budgets from
+ *   the measured per-stage cycles; at C = 256 and ~49k tokens the data gradient gets
+ *   68 SMs and the weight gradient 80): the two gradients run side by side on disjoint
  *   groups of SMs, the weight gradient on a side stream of the library that is
  *   forked from and joined back to `stream` with events, so the call stays ordered
  *   on `stream` and can be captured in a CUDA graph.  Each (device, caller stream)
@@ -180,7 +183,8 @@ SVCONV_API int svconv_bwd_weight_noalloc(int dtype, const void* dY, const void* 
  *   streams, one of them capturing, neither wait on nor enter each other's work.
  *   dX is bitwise identical to svconv_bwd_data's; dW / db use fewer token splits
  *   than svconv_bwd_weight (another fixed summation order: deterministic, same
- *   tolerance).  Other shapes and fp32 run the two calls in order on `stream`.
+ *   tolerance; svconv_bwd_workspace_size gives the size for this call's split).
+ *   Other shapes and fp32 run the two calls in order on `stream`.
  *   Errors: as the two calls.
  */
 SVCONV_API int svconv_bwd(int dtype, const void* dY, const void* X, const int32_t* nbr, int n, int Cin, int Cout,
